@@ -1,0 +1,388 @@
+/*
+ * oracle.c -- plain, slow CPU oracle for the row-split int4 hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline / reference legs may load this library.  It shares no code,
+ * header, table or helper with the CUDA library in row_split_int4_b200/, and
+ * it never reads anything the CUDA library produced unless a test hands it
+ * that data on purpose (the per-stage checks feed each stage the same bf16
+ * input the GPU stage took).
+ *
+ * Everything here is the plain definition, computed in double precision:
+ *
+ *   qmm      y[m,n] = bf16_RNE( sum_{k<K} x[m,k] * (s[n,k/64]*q[n,k] + b[n,k/64]) )
+ *            -- the 4-bit affine, group-64 format of the checkpoint named in
+ *               TensorFold PR #1437 (Receipt: "4-bit affine with group 64");
+ *               each output row is reduced over the whole K by whoever owns it
+ *               (TensorFold PR #1433, step-1 body: the seam exchanges whole
+ *               output rows, each rank reduces over the full K).
+ *   glu      a = bf16_RNE( g * SiLU(u) ),  SiLU(u) = u / (1 + exp(-u))
+ *   gather   whole bf16 rows copied to their offsets, no arithmetic; a missing
+ *            half reads as the bf16 NaN 0x7FC0 (PR #1433 step-1 body: a broken
+ *            link surfaces as 0x7FC0).
+ *   argmax   linear scan, the lower id wins ties, any NaN/+-Inf flags the row
+ *            with bit 31 of the id word (PR #1433 step-1 body).
+ *   pick     any flagged word -> 0xFFFFFFFF, else the larger value, lower id on
+ *            ties (PR #1433 step-1 body; step-2 body: the pick is the better of
+ *            the two half-vocab winners).
+ *
+ * Readings taken where the pages are silent (all listed in the design doc):
+ *   nibble order  element k lives in byte k/2 of its row, low nibble for even k;
+ *   q             unsigned 0..15, no separate zero point (the bias carries it);
+ *   rounding      round-to-nearest-even straight from double to bf16, NaN -> 0x7FC0;
+ *   +-0           compare equal, so they tie and the lower id wins;
+ *   flagged word  value bits 0x7FC00000, id word 0x80000000 | first non-finite id.
+ *
+ * Build:  gcc -O2 -fopenmp -shared -fPIC oracle.c -o liboracle.so -lm
+ * (no -ffast-math: the double arithmetic must be IEEE).
+ *
+ * Planted controls: building with -DORC_PLANT=n makes one deliberate mistake,
+ * used only by tests/test_oracle_plants.py to show that the pins catch it:
+ *   1 the split rows of half h are the peer's rows      (a stage on the peer's half)
+ *   2 gather writes part 0 into every slot              (a gather writing its own half twice)
+ *   3 argmax breaks ties to the higher id
+ *   4 pick breaks ties to the higher id
+ *   5 argmax does not flag non-finite values
+ *   6 pick ignores the flag bit
+ *   7 dequant drops the bias term
+ *   8 dequant swaps the nibble order inside a byte
+ *   9 GLU uses SiLU(g)*u instead of g*SiLU(u)
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#ifndef ORC_PLANT
+#define ORC_PLANT 0
+#endif
+
+#define ORC_GROUP 64
+#define ORC_FLAG 0x80000000u
+#define ORC_SENTINEL 0xFFFFFFFFu
+#define ORC_NAN_BF16 0x7FC0u
+
+/* ---------------------------------------------------------------- bf16 -- */
+
+/* bf16 bit pattern -> double.  A bf16 is the top half of an fp32, so the
+ * widening is exact. */
+static double orc_bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* double -> bf16, round to nearest, ties to even, in one step (never through
+ * fp32, whose own rounding would round twice).  bf16: 1 sign bit, 8 exponent
+ * bits (bias 127), 7 stored mantissa bits; subnormals are kept; overflow
+ * rounds to +-Inf; NaN becomes 0x7FC0. */
+uint16_t orc_bf16_rne(double v)
+{
+    if (isnan(v))
+        return (uint16_t)ORC_NAN_BF16;
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80u);
+    int e2;
+    (void)frexp(a, &e2);          /* a = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;               /* a = 1.xxx * 2^E */
+    if (E < -126)
+        E = -126;                 /* subnormal: fixed spacing 2^-133 */
+    double scaled = ldexp(a, 7 - E);   /* a / 2^(E-7): exact power-of-two scaling */
+    double r = floor(scaled);
+    double frac = scaled - r;          /* exact: scaled < 2^9 */
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) == 1.0))
+        r += 1.0;
+    uint32_t ri = (uint32_t)r;
+    if (scaled < 128.0) {
+        /* subnormal range: bits are the mantissa count; 128 carries into
+         * the smallest normal, whose encoding is also 128 (0x0080). */
+        return (uint16_t)(sign | ri);
+    }
+    if (ri == 256u) {
+        E += 1;
+        ri = 128u;
+    }
+    if (E > 127)
+        return (uint16_t)(sign | 0x7F80u);
+    return (uint16_t)(sign | ((uint32_t)(E + 127) << 7) | (ri - 128u));
+}
+
+void orc_bf16_rne_array(const double *v, uint16_t *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = orc_bf16_rne(v[i]);
+}
+
+/* --------------------------------------------------------------- dequant -- */
+
+/* q of element k of one packed row (C1 reading: byte k/2, low nibble = even k). */
+static unsigned orc_nibble(const uint8_t *row, int64_t k)
+{
+    uint8_t byte = row[k >> 1];
+#if ORC_PLANT == 8
+    return (k & 1) ? (byte & 0xFu) : (byte >> 4);
+#else
+    return (k & 1) ? (byte >> 4) : (byte & 0xFu);
+#endif
+}
+
+/* w[n,k] = s[n,k/64] * q[n,k] + b[n,k/64], all in double.  With a bf16 scale
+ * (8 significant bits) and a 4-bit q the product is exact, and so is the sum
+ * with the bias whenever their exponents are within ~40 of each other. */
+double orc_dequant(const uint8_t *wq, const uint16_t *scales, const uint16_t *biases,
+                   int K, int64_t n, int64_t k)
+{
+    const int64_t G = K / ORC_GROUP;
+    double s = orc_bf16_to_f64(scales[n * G + k / ORC_GROUP]);
+    double b = orc_bf16_to_f64(biases[n * G + k / ORC_GROUP]);
+    double q = (double)orc_nibble(wq + n * (int64_t)(K / 2), k);
+#if ORC_PLANT == 7
+    (void)b;
+    return s * q;
+#else
+    return s * q + b;
+#endif
+}
+
+/* ------------------------------------------------------------------- qmm -- */
+
+/* For each activation row m and each listed weight row rows[i]:
+ *   y64[m,i]    = sum_k x[m,k] * w[rows[i],k]   (double, ascending k)
+ *   absdot[m,i] = sum_k |x[m,k] * w[rows[i],k]|
+ *   y[m,i]      = bf16_RNE(y64[m,i])
+ * x is bf16 [M][ldx]; wq is [N][K/2]; scales/biases are bf16 [N][K/64].
+ * y is [M][ldy]; y64/absdot are [M][nrows] and may be NULL.
+ * nthreads > 1 splits the rows over OpenMP threads; every row is still one
+ * thread's ascending-k sum, so the result does not depend on nthreads.
+ * Returns 0, or -1 on a bad argument. */
+int orc_qmm_rows(const uint16_t *x, int M, int K, int64_t ldx,
+                 const uint8_t *wq, const uint16_t *scales, const uint16_t *biases,
+                 const int64_t *rows, int64_t nrows,
+                 uint16_t *y, int64_t ldy, double *y64, double *absdot, int nthreads)
+{
+    if (M < 0 || K < 0 || K % ORC_GROUP != 0 || nrows < 0 || ldx < K || ldy < nrows)
+        return -1;
+    const int64_t G = K / ORC_GROUP;
+    const int64_t rowbytes = K / 2;
+#pragma omp parallel for schedule(dynamic, 16) num_threads(nthreads > 0 ? nthreads : 1) if (nthreads > 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t n = rows[i];
+        const uint8_t *qrow = wq + n * rowbytes;
+        for (int m = 0; m < M; ++m) {
+            const uint16_t *xr = x + (int64_t)m * ldx;
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double s = orc_bf16_to_f64(scales[n * G + k / ORC_GROUP]);
+                double b = orc_bf16_to_f64(biases[n * G + k / ORC_GROUP]);
+                double q = (double)orc_nibble(qrow, k);
+#if ORC_PLANT == 7
+                double w = s * q;
+                (void)b;
+#else
+                double w = s * q + b;
+#endif
+                double p = orc_bf16_to_f64(xr[k]) * w;
+                acc += p;
+                aacc += fabs(p);
+            }
+            y[(int64_t)m * ldy + i] = orc_bf16_rne(acc);
+            if (y64)
+                y64[(int64_t)m * nrows + i] = acc;
+            if (absdot)
+                absdot[(int64_t)m * nrows + i] = aacc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------- GLU -- */
+
+/* a = bf16_RNE(g * SiLU(u)), SiLU(u) = u / (1 + exp(-u)), in double.  g and u
+ * are the bf16-rounded outputs of the gate row and the up row with the same
+ * index.  a64 (may be NULL) receives the unrounded double. */
+void orc_glu(const uint16_t *g, const uint16_t *u, uint16_t *a, double *a64, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double gv = orc_bf16_to_f64(g[i]);
+        double uv = orc_bf16_to_f64(u[i]);
+#if ORC_PLANT == 9
+        double r = (gv / (1.0 + exp(-gv))) * uv;
+#else
+        double r = gv * (uv / (1.0 + exp(-uv)));
+#endif
+        a[i] = orc_bf16_rne(r);
+        if (a64)
+            a64[i] = r;
+    }
+}
+
+/* ---------------------------------------------------------------- gather -- */
+
+/* The row range that half h of nparts owns in a matrix of N rows: contiguous
+ * equal spans [h*N/nparts, (h+1)*N/nparts) (TensorFold PR #1433 step-2 body:
+ * 2,560 of 5,120, 8,704 of 17,408, 124,160 of 248,320; rank 0 starts at 0).
+ * Returns -1 when N does not split evenly. */
+int orc_half_rows(int h, int nparts, int64_t N, int64_t *row0, int64_t *nrows)
+{
+    if (nparts <= 0 || h < 0 || h >= nparts || N < 0 || N % nparts != 0)
+        return -1;
+    int64_t w = N / nparts;
+#if ORC_PLANT == 1
+    h = (h + 1) % nparts;
+#endif
+    *row0 = (int64_t)h * w;
+    *nrows = w;
+    return 0;
+}
+
+/* dst[m, off_h + j] = part_h[m, j] with off_h = widths[0] + ... + widths[h-1];
+ * part h is dense [M][widths[h]].  A NULL part fills its columns with the bf16
+ * NaN 0x7FC0.  Pure copy, no arithmetic. */
+void orc_gather_rows(uint16_t *dst, int64_t ld_dst, const uint16_t *const *parts,
+                     const int64_t *widths, int nparts, int M)
+{
+    int64_t off = 0;
+    for (int h = 0; h < nparts; ++h) {
+#if ORC_PLANT == 2
+        const uint16_t *src = parts[0];
+        const int64_t sw = widths[0];
+#else
+        const uint16_t *src = parts[h];
+        const int64_t sw = widths[h];
+#endif
+        for (int m = 0; m < M; ++m)
+            for (int64_t j = 0; j < widths[h]; ++j)
+                dst[(int64_t)m * ld_dst + off + j] =
+                    src ? src[(int64_t)m * sw + (j < sw ? j : sw - 1)] : (uint16_t)ORC_NAN_BF16;
+        off += widths[h];
+    }
+}
+
+/* ---------------------------------------------------------------- argmax -- */
+
+/* For each row m of bf16 values v[m][0..n): the largest finite value with the
+ * lowest index among equals, reported with global id id_base + j.  Any NaN,
+ * +Inf or -Inf flags the row.  Word layout (u64):
+ *   unflagged: high 32 = id, low 32 = the fp32 bits of the winning bf16 value
+ *   flagged:   high 32 = 0x80000000 | (id_base + first non-finite j),
+ *              low 32  = 0x7FC00000 (the NaN the pages report)
+ * Returns -1 for n < 1. */
+int orc_argmax_rows(const uint16_t *v, int M, int64_t n, int64_t ld, uint32_t id_base,
+                    uint64_t *words)
+{
+    if (n < 1 || M < 0 || ld < n)
+        return -1;
+    for (int m = 0; m < M; ++m) {
+        const uint16_t *r = v + (int64_t)m * ld;
+        int flagged = 0;
+        int64_t first_nf = 0, best = -1;
+        double bestv = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            double x = orc_bf16_to_f64(r[j]);
+            if (!isfinite(x)) {
+#if ORC_PLANT != 5
+                if (!flagged) {
+                    flagged = 1;
+                    first_nf = j;
+                }
+#endif
+                continue;
+            }
+#if ORC_PLANT == 3
+            if (best < 0 || x >= bestv) {
+#else
+            if (best < 0 || x > bestv) {
+#endif
+                best = j;
+                bestv = x;
+            }
+        }
+        if (flagged) {
+            uint32_t idw = ORC_FLAG | (id_base + (uint32_t)first_nf);
+            words[m] = ((uint64_t)idw << 32) | 0x7FC00000u;
+        } else if (best < 0) {
+            /* every value was non-finite but flagging is planted away */
+            words[m] = ((uint64_t)id_base << 32) | 0x7FC00000u;
+        } else {
+            uint32_t bits = (uint32_t)r[best] << 16;
+            words[m] = ((uint64_t)(id_base + (uint32_t)best) << 32) | bits;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ pick -- */
+
+static double orc_word_value(uint64_t w)
+{
+    uint32_t bits = (uint32_t)(w & 0xFFFFFFFFu);
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* words is [nparts][M].  For each row: if any part's id word has the flag bit,
+ * the pick is 0xFFFFFFFF; otherwise the id of the larger value, the lower id
+ * on equal values (+0 and -0 are equal). */
+void orc_pick(const uint64_t *words, int nparts, int M, uint32_t *ids)
+{
+    for (int m = 0; m < M; ++m) {
+        int flagged = 0;
+        for (int p = 0; p < nparts; ++p) {
+            uint32_t idw = (uint32_t)(words[(int64_t)p * M + m] >> 32);
+#if ORC_PLANT == 6
+            (void)idw;
+#else
+            if (idw & ORC_FLAG)
+                flagged = 1;
+#endif
+        }
+        if (flagged) {
+            ids[m] = ORC_SENTINEL;
+            continue;
+        }
+        uint32_t best_id = 0;
+        double best_v = 0.0;
+        for (int p = 0; p < nparts; ++p) {
+            uint64_t w = words[(int64_t)p * M + m];
+            uint32_t id = (uint32_t)(w >> 32);
+            double v = orc_word_value(w);
+#if ORC_PLANT == 4
+            if (p == 0 || v > best_v || (v == best_v && id > best_id)) {
+#else
+            if (p == 0 || v > best_v || (v == best_v && id < best_id)) {
+#endif
+                best_id = id;
+                best_v = v;
+            }
+        }
+        ids[m] = best_id;
+    }
+}
+
+/* ------------------------------------------------------------ top-two gap -- */
+
+/* gap[m] = best - (largest value at any other index), on unrounded double
+ * logits [M][n]; +Inf when n == 1.  The end-to-end id check only trusts ids
+ * whose gap exceeds the stated margin. */
+void orc_top2_gap(const double *logits, int M, int64_t n, double *gap)
+{
+    for (int m = 0; m < M; ++m) {
+        const double *r = logits + (int64_t)m * n;
+        int64_t best = 0;
+        for (int64_t j = 1; j < n; ++j)
+            if (r[j] > r[best])
+                best = j;
+        double second = -INFINITY;
+        for (int64_t j = 0; j < n; ++j)
+            if (j != best && r[j] > second)
+                second = r[j];
+        gap[m] = (n == 1) ? INFINITY : r[best] - second;
+    }
+}
