@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""bench.py -- one decode step of the row-split int4 hot path, timed on B200s.
+
+A step is one pass of every step of the path at M=1 over seeded synthetic
+inputs already resident in HBM, with the pages' two-rank split emulated as
+two row halves on one GPU (TensorFold PR #1433, step-1 and step-2 bodies):
+
+  gate+up  K=5,120 -> 2 x 17,408 rows, each half owning 8,704 rows of each
+           member, g * SiLU(u) fused, 2 calls          (tf_qmm_rows, GLU)
+  gather   the two 8,704-wide activated halves         (tf_gather_rows)
+  down     K=17,408 -> 5,120 rows as 2 x 2,560          (tf_qmm_rows)
+  gather   the two 2,560-wide halves                    (tf_gather_rows)
+  lm_head  K=5,120 -> 248,320 rows as 2 x 124,160       (tf_qmm_rows)
+  argmax   per half, global ids                         (tf_argmax_rows)
+  pick     the better half-winner                       (tf_pick)
+
+The metric is the int4 dequant-GEMV HBM throughput (GB/s of algorithmic
+bytes: 0.5625 B per weight plus activations in and out), with the
+lm_head+argmax+pick time per token beside it.  The weights of one step
+(866 MB) exceed the 126 MB L2, so every step reads them from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tf|reference]
+  python bench.py --sweep        # M in {1..128} x the four shapes, per-point lines
+
+For N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica of the step: the path has no exchange that crosses a device here, so
+`value` is the sum of all ranks' bytes over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "int4 dequant-GEMV HBM GB/s (% B200 peak) at M=1; lm_head+argmax µs/token"
+WORKLOAD = ("decode step M=1, two row halves on one GPU: gate_up 5120x34816 int4 g64 (GLU fused) + gather + "
+            "down 17408x5120 + gather + lm_head 5120x248320 + per-half argmax + pick")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------- helpers
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def qmm_bytes(K, rows, M=1, out_cols=None):
+    """Algorithmic bytes of one qmm call: 0.5625 B per weight + x read + y written."""
+    out_cols = rows if out_cols is None else out_cols
+    return int(0.5625 * K * rows) + 2 * M * K + 2 * M * out_cols
+
+
+def step_bytes():
+    H, F, V = 5120, 17408, 248320
+    b = {
+        "gate_up": 2 * qmm_bytes(H, F, out_cols=F // 2),      # each half: F rows (8,704 gate + 8,704 up)
+        "gather_act": 2 * (2 * F),                            # read both halves, write the frame
+        "down": 2 * qmm_bytes(F, H // 2),
+        "gather_y": 2 * (2 * H),
+        "lm_head": 2 * qmm_bytes(H, V // 2),
+        "argmax": 2 * V + 2 * 8,
+        "pick": 2 * 8 + 4,
+    }
+    b["total"] = sum(b.values())
+    return b
+
+
+def traffic_from_profiles(kernel_src):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    only while the kernel's source is the one the counters were taken on."""
+    path = os.path.join(ROOT, "profiles", "qmm_m1_lm_head_half.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
+    s = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    if not m or not s:
+        return None
+    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return int(m.group(1)) if cur == s.group(1) else None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read only) while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, index, period=0.01):
+        self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
+        self.period, self.index = period, index
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- the step
+class DecodeStep:
+    """Device buffers and weights of one decode step; run() enqueues it."""
+
+    def __init__(self, tf, synth, seed=0, host_weights=None):
+        import torch
+        self.tf, self.torch = tf, torch
+        H, F, V = synth.HIDDEN, synth.FFN, synth.VOCAB
+        self.H, self.F, self.V = H, F, V
+        hw = host_weights or make_host_weights(synth, seed)
+        self.host = hw
+        self.Wgu = synth.weights_to_device(hw["gate_up"])
+        self.Wd = synth.weights_to_device(hw["down"])
+        self.Wlm = synth.weights_to_device(hw["lm_head"])
+        bf = dict(dtype=torch.bfloat16, device="cuda")
+        self.x_mlp = synth.to_device(hw["x_mlp"])
+        self.x_head = synth.to_device(hw["x_head"])
+        self.act_h = [torch.empty(1, F // 2, **bf) for _ in range(2)]
+        self.act = torch.empty(1, F, **bf)
+        self.y_h = [torch.empty(1, H // 2, **bf) for _ in range(2)]
+        self.y = torch.empty(1, H, **bf)
+        self.logits = [torch.empty(1, V // 2, **bf) for _ in range(2)]
+        self.words = torch.empty(2, 1, dtype=torch.int64, device="cuda")
+        self.ids = torch.empty(1, dtype=torch.int32, device="cuda")
+        self.scratch = torch.empty(tf.tf_argmax_scratch_bytes(1, V // 2), dtype=torch.uint8, device="cuda")
+        self.member = [tf.tf_member_segs(F, 2, h) for h in range(2)]
+        self.down_rows = [tf.tf_split_rows(H, 2, h) for h in range(2)]
+        self.head_rows = [tf.tf_split_rows(V, 2, h) for h in range(2)]
+        self.window = synth.WINDOW_BYTES
+        self.launches_per_step = 2 + 1 + 2 + 1 + 2 + 2 * 2 + 1
+
+    def run(self, stream, lm_events=None, head_events=None):
+        tf = self.tf
+        for h in range(2):
+            tf.tf_qmm_rows(self.x_mlp, *self.Wgu, self.member[h], self.act_h[h], epi=tf.TF_EPI_GLU, stream=stream)
+        tf.tf_gather_rows(self.act, self.act_h, [self.F // 2] * 2, window_bytes=self.window, stream=stream)
+        for h in range(2):
+            tf.tf_qmm_rows(self.act, *self.Wd, [self.down_rows[h]], self.y_h[h], stream=stream)
+        tf.tf_gather_rows(self.y, self.y_h, [self.H // 2] * 2, window_bytes=self.window, stream=stream)
+        if head_events is not None:
+            head_events[0].record(stream)
+        for h in range(2):
+            if lm_events is not None:
+                lm_events[h][0].record(stream)
+            tf.tf_qmm_rows(self.x_head, *self.Wlm, [self.head_rows[h]], self.logits[h], stream=stream)
+            if lm_events is not None:
+                lm_events[h][1].record(stream)
+        for h in range(2):
+            tf.tf_argmax_rows(self.logits[h], self.head_rows[h][0], self.words[h], self.scratch, stream=stream)
+        tf.tf_pick(self.words, self.ids, stream=stream)
+        if head_events is not None:
+            head_events[1].record(stream)
+
+
+def make_host_weights(synth, seed=0):
+    H, F, V = synth.HIDDEN, synth.FFN, synth.VOCAB
+    return {
+        "gate_up": synth.make_weights(2 * F, H, seed=seed, tag=synth.TAG_W),
+        "down": synth.make_weights(H, F, seed=seed, tag=synth.TAG_W2),
+        "lm_head": synth.make_weights(V, H, seed=seed, tag=synth.TAG_HEAD),
+        "x_mlp": synth.make_x(1, H, seed=seed),
+        "x_head": synth.make_x(1, H, seed=seed, tag=5),
+    }
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(hw, frac, nthreads):
+    """Run the oracle on the first `frac` of every matrix's rows of the step
+    (M=1), plus argmax/pick over that many logits; return (seconds, bytes)."""
+    import numpy as np
+    import oracle
+    orc = oracle.load()
+    H, F, V = 5120, 17408, 248320
+    nF = max(8, int(F * frac)) // 2 * 2
+    nH = max(2, int(H * frac)) // 2 * 2
+    nV = max(16, int(V * frac)) // 2 * 2
+    t0 = time.perf_counter()
+    gu = hw["gate_up"].astuple()
+    g = orc.qmm_rows(hw["x_mlp"], *gu, np.arange(nF), nthreads=nthreads)
+    u = orc.qmm_rows(hw["x_mlp"], *gu, np.arange(F, F + nF), nthreads=nthreads)
+    a = orc.glu(g, u)
+    act = np.zeros((1, F), dtype=np.uint16)
+    act[:, :nF] = a
+    orc.qmm_rows(act, *hw["down"].astuple(), np.arange(nH), nthreads=nthreads)
+    lg = orc.qmm_rows(hw["x_head"], *hw["lm_head"].astuple(), np.arange(nV), nthreads=nthreads)
+    h = nV // 2
+    orc.head_split([lg[:, :h], lg[:, h:]], [0, h])
+    dt = time.perf_counter() - t0
+    nbytes = (qmm_bytes(H, 2 * nF, out_cols=nF) + qmm_bytes(F, nH) + qmm_bytes(H, nV) + 2 * nV)
+    return dt, nbytes, f"first {frac:.4%} of every matrix's rows (gate_up {2 * nF}, down {nH}, lm_head {nV} rows) at M=1"
+
+
+def calibrated_oracle(hw, target_s, nthreads):
+    frac = 1.0 / 512
+    dt, nb, _ = oracle_sample(hw, frac, nthreads)
+    frac = min(1.0, frac * max(1.0, target_s / max(dt, 1e-4)))
+    return frac
+
+
+def cpu_baseline(hw, target_s=12.0):
+    nthreads = os.cpu_count() or 1
+    frac = calibrated_oracle(hw, target_s, nthreads)
+    dt, nb, desc = oracle_sample(hw, frac, nthreads)
+    return {"value": round(nb / dt / 1e9, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+            "sample": desc + f", {dt:.1f} s, C fp64 oracle with OpenMP over rows"}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    hw = make_host_weights(synth, args.seed)
+    nthreads = os.cpu_count() or 1
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    frac = calibrated_oracle(hw, budget, nthreads)
+    for _ in range(args.warmup):
+        oracle_sample(hw, frac, nthreads)
+    tot_t, tot_b, desc = 0.0, 0, ""
+    for _ in range(args.steps):
+        dt, nb, desc = oracle_sample(hw, frac, nthreads)
+        tot_t += dt
+        tot_b += nb
+    value = tot_b / tot_t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_per_step": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- sweep
+def run_sweep(args):
+    raise SystemExit("--sweep: not available yet")
+
+
+# --------------------------------------------------------------------------- main arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["tf", "reference"], default="tf")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="per-point sweep over M and the four shapes")
+    ap.add_argument("--reps", type=int, default=1000)
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    import row_split_int4_b200 as tf
+    import synth
+
+    hw = make_host_weights(synth, args.seed)
+    step = DecodeStep(tf, synth, host_weights=hw)
+    stream = torch.cuda.current_stream()
+    nb = step_bytes()
+
+    for _ in range(args.warmup):
+        step.run(stream)
+    barrier()
+
+    K = args.steps
+    lm_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+             for _ in range(2)]
+    hd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    with sampler:
+        t0.record(stream)
+        for i in range(K):
+            step.run(stream, lm_events=[lm_ev[0][i], lm_ev[1][i]], head_events=hd_ev[i])
+        t1.record(stream)
+        barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    lm_ms = [a.elapsed_time(b) for h in range(2) for (a, b) in lm_ev[h]]
+    head_ms = [a.elapsed_time(b) for (a, b) in hd_ev]
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        xm_h = torch.empty_like(step.x_mlp, device="cpu").pin_memory()
+        xh_h = torch.empty_like(step.x_head, device="cpu").pin_memory()
+        xm_h.copy_(step.x_mlp)
+        xh_h.copy_(step.x_head)
+        y_h = torch.empty_like(step.y, device="cpu").pin_memory()
+        id_h = torch.empty_like(step.ids, device="cpu").pin_memory()
+        Ke = max(3, min(K, 1000))
+
+        def e2e_step():
+            step.x_mlp.copy_(xm_h, non_blocking=True)
+            step.x_head.copy_(xh_h, non_blocking=True)
+            step.run(stream)
+            y_h.copy_(step.y, non_blocking=True)
+            id_h.copy_(step.ids, non_blocking=True)
+            stream.synchronize()
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / Ke
+        e2e = {"e2e_ms": e2e_ms, "h2d": step.x_mlp.numel() * 2 + step.x_head.numel() * 2,
+               "d2h": step.y.numel() * 2 + step.ids.numel() * 4}
+
+    # max over ranks
+    vals = torch.tensor([elapsed_ms, e2e["e2e_ms"] if e2e else 0.0], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = float(vals[0]), float(vals[1])
+
+    if rank == 0:
+        ms_step = elapsed_ms / K
+        value = nb["total"] * world * K / (elapsed_ms / 1e3) / 1e9
+        peak, peak_kind = measured_peak()
+        lm_bytes = qmm_bytes(5120, 248320 // 2)
+        lm_avg_ms = statistics.fmean(lm_ms)
+        achieved = lm_bytes / (lm_avg_ms / 1e3) / 1e9
+        src = os.path.join(ROOT, "row_split_int4_b200", "csrc", "qmm_gemv.cu")
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": 1, "bytes_per_step": nb["total"],
+                       "l2": "no flush: inputs larger than L2 (866 MB of weights per step vs 126 MB L2)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "one GPU, two row halves"},
+            "lm_head_argmax_us_per_token": round(statistics.fmean(head_ms) * 1e3, 2),
+            "tokens_per_s_equiv": round(1e3 / ms_step, 1),
+            "roofline": {"bound": "hbm", "kernel": "qmm_m1_kernel (lm_head half, 124,160 x 5,120)",
+                         "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic_from_profiles(src),
+                         "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_avg_ms * 1e3, 3)},
+            "gpu_launches": step.launches_per_step * K,
+            "clocks": sampler.summary(),
+        }
+        if e2e:
+            line["e2e"] = {"value": round(nb["total"] * world / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                           "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                           "ms_per_step": round(e2e_ms, 5)}
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(hw)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,228 @@
+/*
+ * tf.h -- C ABI of libtf.so, the row-split int4 hot path on one NVIDIA B200.
+ *
+ * The library computes, on the GPU, the steps the TensorFold pair seam is made
+ * of (TensorFold PR #1433, "Step 1 of 6" body and step-2 "What this changes"):
+ * a 4-bit affine quantized projection over a slice of output rows, each row
+ * reduced over the whole K by whoever owns it; a pure copy that joins the
+ * slices; the head's argmax over each half of the vocabulary; and the pick
+ * between the halves.  The two ranks of the pages are emulated as two row
+ * ranges of one matrix on one GPU: no collective, no second device.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers named x, wq, scales, biases, y, dst, parts[], logits, words,
+ *    ids and scratch are DEVICE pointers (cudaMalloc'd or torch tensors on
+ *    the current device).  Arrays of pointers and sizes (segs, parts, widths)
+ *    are HOST arrays, read before the call returns.
+ *  - bf16 values are passed as their 16-bit patterns (bf16 = top half of an
+ *    IEEE fp32), row-major with the stated leading dimension in elements.
+ *  - The caller owns every buffer.  The library allocates nothing, keeps no
+ *    pointer after the call returns and never synchronises the stream: work
+ *    is enqueued on `stream` (NULL = the legacy default stream) and results
+ *    are valid once that stream reaches them.
+ *  - Every argument is validated on the host BEFORE anything is enqueued; a
+ *    rejected call moves no data ("refuse by name before any state moves",
+ *    TensorFold PR #1434 review thread).  The one exception is TF_E_BROKEN,
+ *    which is a result, not a refusal (see tf_gather_rows).
+ *  - No entry point exits, aborts, traps or prints.  A failed launch returns
+ *    TF_E_CUDA (the CUDA error is left for cudaGetLastError to report).
+ *  - Outputs must not overlap inputs.
+ */
+#ifndef TF_H
+#define TF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that callers need no CUDA header. */
+typedef struct CUstream_st *tf_stream;
+
+typedef enum {
+    TF_OK = 0,
+    TF_E_ARG = 1,     /* a NULL pointer, a count or size out of its stated range */
+    TF_E_RANGE = 2,   /* a row segment outside [0, N_whole), overlapping segments, or ids past 2^31 */
+    TF_E_ALIGN = 3,   /* a pointer or leading dimension without the stated alignment */
+    TF_E_WINDOW = 4,  /* a part of a gather is larger than the exchange window */
+    TF_E_BROKEN = 5,  /* a gather part was missing: its columns were filled with 0x7FC0 */
+    TF_E_CUDA = 6,    /* a kernel launch failed */
+    TF_E_UNIMPL = 7   /* a valid request this build does not implement */
+} tf_status;
+
+/* Bit 31 of an argmax id word: the row held a NaN or +-Inf
+ * (TensorFold PR #1433 step-1 body: "NaN bits with bit 31 set in its id word"). */
+#define TF_PAIR_FLAG 0x80000000u
+/* tf_pick's result for a flagged row; never a token id
+ * (TensorFold PR #1433 step-2 body: the session reads maxInt(u32) as error.PairFailed). */
+#define TF_PICK_FAILED 0xFFFFFFFFu
+/* The bf16 NaN a missing gather part reads as (TensorFold PR #1433 step-1 body). */
+#define TF_NAN_BF16 0x7FC0u
+/* Rows one qmm call may carry: chunk(requested) = min(requested, 128)
+ * (TensorFold PR #1434, step-3 body: batch_rows = 128). */
+#define TF_BATCH_ROWS 128
+/* K elements sharing one bf16 scale and one bf16 bias (TensorFold PR #1437 Receipt:
+ * "4-bit affine with group 64"). */
+#define TF_GROUP 64
+#define TF_MAX_K 65536
+#define TF_MAX_SEGS 8
+#define TF_MAX_PARTS 8
+/* Pass as window_bytes to skip the gather's window check. */
+#define TF_NO_WINDOW ((size_t)-1)
+
+/* A range of rows of the WHOLE checkpoint matrix: [row0, row0 + nrows). */
+typedef struct {
+    int32_t row0;
+    int32_t nrows;
+} tf_seg;
+
+typedef enum {
+    TF_EPI_NONE = 0, /* y holds the bf16 qmm outputs of every listed row */
+    TF_EPI_GLU = 1   /* two equal segments (gate rows, up rows): y[i] = bf16(g_i * SiLU(u_i)) */
+} tf_epi;
+
+/*
+ * tf_qmm_rows -- 4-bit affine quantized matrix-vector / matrix product over a
+ * slice of output rows, reduced over the full K in fp32.
+ *
+ * Defines (TensorFold PR #1433 step-1 body: "rank r owns 2,560 of the 5,120
+ * output columns ..., reduces over the full K on its own rank"; PR #1437
+ * Receipt: 4-bit affine, group 64):
+ *     w[n,k]  = s[n, k/64] * q[n,k] + b[n, k/64]
+ *     out[m,n] = bf16_RNE( sum_{k<K} x[m,k] * w[n,k] )   (fp32 accumulation)
+ * for every row n of the segments, in segment order.  The summation order
+ * depends on K alone -- never on the segments, their order, N_whole or M's
+ * position in a chunk -- so a row computed in a slice has the same bits as the
+ * same row computed in the whole matrix (PR #1433 review: "a different sk is
+ * a different fp32 order").
+ *
+ *   x       bf16 [M][ldx] activations.  16-byte aligned, ldx % 8 == 0, ldx >= K.
+ *   M       rows of x, 0 <= M <= TF_BATCH_ROWS (M == 0: nothing is enqueued).
+ *           Callers split larger requests into chunks of TF_BATCH_ROWS.
+ *   K       reduction length, 64 <= K <= TF_MAX_K, K % 64 == 0.
+ *   wq      uint8 [N_whole][K/2] packed codes of the whole matrix; element k of
+ *           a row is byte k/2, low nibble for even k, high nibble for odd k;
+ *           q is unsigned 0..15.  16-byte aligned.
+ *   scales  bf16 [N_whole][K/64]; biases bf16 [N_whole][K/64].  2-byte aligned.
+ *   N_whole rows of the whole matrix (>= 1).
+ *   segs    host array of nseg row ranges of the whole matrix, 1 <= nseg <= TF_MAX_SEGS,
+ *           inside [0, N_whole) and pairwise disjoint (TF_E_RANGE otherwise).
+ *   epi     TF_EPI_NONE: y[m][c] for c < sum(nrows) is the c-th listed row.
+ *           TF_EPI_GLU: nseg == 2 with equal nrows F; g and u are the bf16
+ *           outputs of row segs[0].row0+i and segs[1].row0+i, and
+ *           y[m][i] = bf16_RNE(g * SiLU(u)), SiLU(u) = u / (1 + exp(-u)), in fp32.
+ *   y       bf16 [M][ldy], ldy >= the number of output columns.  2-byte aligned.
+ * Errors: TF_E_ARG, TF_E_RANGE, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+tf_status tf_qmm_rows(const void *x, int M, int K, int ldx,
+                      const uint8_t *wq, const void *scales, const void *biases, int N_whole,
+                      const tf_seg *segs, int nseg, tf_epi epi,
+                      void *y, int ldy, tf_stream stream);
+
+/*
+ * tf_gather_rows -- join row slices into the whole frame by copying whole bf16
+ * rows; no arithmetic (TensorFold PR #1433 step-1 body: pair_gather copies
+ * whole rows in bf16 without doing any arithmetic; step-2 body: gather copies
+ * each rank's half to its own offset).
+ *
+ *     dst[m][off_h + j] = parts[h][m][j],   off_h = widths[0] + ... + widths[h-1]
+ *
+ *   dst     bf16 [M][ld_dst], ld_dst >= sum(widths).
+ *   parts   host array of nparts device pointers, part h dense bf16 [M][widths[h]];
+ *           1 <= nparts <= TF_MAX_PARTS.  A NULL part is a broken link.
+ *   widths  host array, widths[h] >= 0.
+ *   window_bytes  the exchange window: every part must satisfy
+ *           M * widths[h] * 2 <= window_bytes, else TF_E_WINDOW and nothing is
+ *           enqueued (PR #1434: seamBytes(rows) = rows * 8,704 * 2 must fit
+ *           pairBytes; the cap exists so that the widest seam never exceeds it).
+ *           TF_NO_WINDOW skips the check.
+ * Result: TF_OK; or TF_E_BROKEN when a part was NULL -- its columns are filled
+ * with TF_NAN_BF16 (0x7FC0), the other parts are copied, and everything is
+ * enqueued before the call returns (PR #1433: a broken link surfaces as bf16 NaN).
+ * Errors: TF_E_ARG, TF_E_WINDOW (before any launch), TF_E_CUDA.
+ */
+tf_status tf_gather_rows(void *dst, int ld_dst, const void *const *parts, const int *widths,
+                         int nparts, int M, size_t window_bytes, tf_stream stream);
+
+/*
+ * tf_argmax_rows -- argmax over one slice of the vocabulary for each row
+ * (TensorFold PR #1433 step-1 body: pair_argmax; step-2 body: argmax over each
+ * rank's 124,160-logit half).
+ *
+ * For each row m of logits[m][0..n): the largest finite value, the LOWEST id
+ * among equal values (+0 and -0 are equal).  Ids are global: id_base + j.  A
+ * row holding any NaN, +Inf or -Inf is flagged.  One 64-bit word per row:
+ *     unflagged: bits 63..32 = id, bits 31..0 = fp32 bits of the winning bf16
+ *                (its bf16 pattern << 16, the sign of a winning -0 kept)
+ *     flagged:   bits 63..32 = TF_PAIR_FLAG | (id_base + first non-finite j),
+ *                bits 31..0  = 0x7FC00000
+ *
+ *   logits  bf16 [M][ld], ld >= n, 2-byte aligned (16-byte aligned with
+ *           ld % 8 == 0 takes the vector path; both give the same result).
+ *   M       0 <= M <= 65535;  n >= 1;  id_base + n <= 2^31 (TF_E_RANGE).
+ *   words   uint64 [M].
+ *   scratch device buffer of at least tf_argmax_scratch_bytes(M, n) bytes,
+ *           8-byte aligned, owned by the caller; its contents on entry do not
+ *           matter and on return are unspecified.  Two calls in flight at
+ *           the same time need two scratch buffers.
+ * Errors: TF_E_ARG, TF_E_RANGE, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+size_t tf_argmax_scratch_bytes(int M, int n);
+tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_base,
+                         uint64_t *words, void *scratch, size_t scratch_bytes, tf_stream stream);
+
+/*
+ * tf_pick -- the better of the per-slice winners (TensorFold PR #1433 step-1
+ * body: pair_pick; the sixth control's test ((am | ap) & PAIR_FLAG) != 0u).
+ *
+ * words is uint64 [nparts][M] (word of part p for row m at p*M + m), as
+ * written by tf_argmax_rows.  For each row: if ANY part's id word has
+ * TF_PAIR_FLAG, ids[m] = TF_PICK_FAILED; otherwise the id of the larger value,
+ * and on equal values the lower id.  nparts == 1 applies the same flag rule to
+ * a whole-vocabulary word.  1 <= nparts <= TF_MAX_PARTS, 0 <= M <= 65535.
+ *   ids     uint32 [M].
+ * Errors: TF_E_ARG (before any launch), TF_E_CUDA.
+ */
+tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_stream stream);
+
+/*
+ * Host arithmetic of the row split (TensorFold PR #1433 step-2 body: the split
+ * is by output rows, rank 0's spans start at 0; 2,560 of 5,120, 8,704 of
+ * 17,408, 124,160 of 248,320; "the fused gate-up keeps the member split").
+ *   tf_split_rows   part h of nparts owns rows [h*N/nparts, (h+1)*N/nparts) of an
+ *                   N-row matrix; *seg receives them.  TF_E_ARG unless
+ *                   1 <= nparts <= TF_MAX_PARTS, 0 <= h < nparts, N >= 0 and
+ *                   N % nparts == 0 (an uneven split is refused, not rounded).
+ *   tf_member_segs  for a fused stack [gate(F rows); up(F rows)] (2F rows in all),
+ *                   part h owns gate rows [h*F/nparts, +F/nparts) and the same rows
+ *                   of up: segs[0] = gate range, segs[1] = up range (offset by F).
+ *                   Same errors as tf_split_rows, with F in place of N.
+ * Pure host functions; they touch no device.
+ */
+tf_status tf_split_rows(int N, int nparts, int h, tf_seg *seg);
+tf_status tf_member_segs(int F, int nparts, int h, tf_seg segs[2]);
+
+/*
+ * Host arithmetic of the seam window (TensorFold PR #1434, step-3 body):
+ *   tf_chunk_rows(requested)      = min(requested, TF_BATCH_ROWS)   (requested >= 0)
+ *   tf_seam_bytes(rows, width)    = rows * width * 2                 (bf16 bytes of one part)
+ * Both are pure functions; they touch no device.
+ */
+int tf_chunk_rows(int requested);
+size_t tf_seam_bytes(int rows, int width);
+
+/* Static name of a status ("TF_OK", "TF_E_ARG", ...); "TF_E_?" for an unknown value. */
+const char *tf_status_str(tf_status s);
+
+/* ABI version of this header; bumped when a signature changes. */
+#define TF_ABI_VERSION 1
+int tf_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TF_H */

@@ -1,0 +1,199 @@
+// seam.cu -- the kernels that join row slices and decide the head's token:
+// gather (a pure copy of whole bf16 rows), the per-slice argmax and the pick
+// (TensorFold PR #1433, step-1 body: pair_gather, pair_argmax, pair_pick
+// move bf16 frames and compare values only).
+#include "tf_common.cuh"
+#include "tf_kernels.h"
+
+namespace tf {
+
+// ---------------------------------------------------------------- gather --
+// One thread per 8 bf16 (16 bytes) of the output; every part's width and
+// offset and the row pitches are multiples of 8, the pointers 16-byte aligned.
+__global__ void gather_vec_kernel(GatherArgs a) {
+    const int total = a.off[a.nparts];
+    const int per_row = total / 8;
+    const long long n = (long long)a.M * per_row;
+    const uint4 nan8 = make_uint4(TF_NAN_BF16 * 0x10001u, TF_NAN_BF16 * 0x10001u, TF_NAN_BF16 * 0x10001u,
+                                  TF_NAN_BF16 * 0x10001u);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(i / per_row);
+        const int col = (int)(i % per_row) * 8;
+        int h = 0;
+#pragma unroll
+        for (int p = 1; p < TF_MAX_PARTS; ++p)
+            if (p < a.nparts && col >= a.off[p]) h = p;
+        const int j = col - a.off[h];
+        uint4 v = nan8;
+        if (a.part[h]) v = *reinterpret_cast<const uint4 *>(a.part[h] + (long long)m * a.width[h] + j);
+        *reinterpret_cast<uint4 *>(a.dst + (long long)m * a.ld_dst + col) = v;
+    }
+}
+
+// Element-wise form for pitches or widths that are not multiples of 8.
+__global__ void gather_scalar_kernel(GatherArgs a) {
+    const int total = a.off[a.nparts];
+    const long long n = (long long)a.M * total;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(i / total);
+        const int col = (int)(i % total);
+        int h = 0;
+#pragma unroll
+        for (int p = 1; p < TF_MAX_PARTS; ++p)
+            if (p < a.nparts && col >= a.off[p]) h = p;
+        const int j = col - a.off[h];
+        a.dst[(long long)m * a.ld_dst + col] =
+            a.part[h] ? a.part[h][(long long)m * a.width[h] + j] : (uint16_t)TF_NAN_BF16;
+    }
+}
+
+cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream) {
+    const long long total = (long long)a.M * a.off[a.nparts] / (vec ? 8 : 1);
+    if (total == 0) return cudaSuccess;
+    long long blocks = (total + 255) / 256;
+    if (blocks > kNumSMs * 16) blocks = kNumSMs * 16;
+    if (vec)
+        gather_vec_kernel<<<(int)blocks, 256, 0, stream>>>(a);
+    else
+        gather_scalar_kernel<<<(int)blocks, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- argmax --
+// A candidate is one 64-bit key whose unsigned order is the selection order:
+//   bit 63      non-finite flag (flagged beats every finite value)
+//   bits 62..31 16-bit order-preserving image of the bf16 value (finite only;
+//               -0 is mapped to +0 so that the two tie)
+//   bits 30..0  0x7FFFFFFF - id (the lower id wins among equals)
+// max() over keys is associative and commutative, so the block and grid
+// reduction trees cannot change the result.  0 is below every real key.
+__device__ __forceinline__ uint64_t cand_key(uint32_t h, uint32_t id) {
+    const uint64_t idpart = (uint64_t)(0x7FFFFFFFu - id);
+    if ((h & 0x7F80u) == 0x7F80u) return (1ull << 63) | idpart;   // NaN or +-Inf
+    if (h == 0x8000u) h = 0u;
+    const uint32_t mono = (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u);
+    return ((uint64_t)mono << 31) | idpart;
+}
+
+__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = umax64(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+constexpr int kArgmaxThreads = 256;
+
+__global__ void __launch_bounds__(kArgmaxThreads) argmax_partial_kernel(ArgmaxArgs a) {
+    const int m = blockIdx.y;
+    const int b = blockIdx.x;
+    const uint16_t *row = a.logits + (long long)m * a.ld;
+    const int j0 = b * a.span;
+    const int j1 = min(a.n, j0 + a.span);
+    uint64_t best = 0;
+    if (a.vec) {
+        const int jv_end = j0 + ((j1 - j0) / 8) * 8;
+        for (int j = j0 + threadIdx.x * 8; j < jv_end; j += kArgmaxThreads * 8) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + j);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                best = umax64(best, cand_key(w[e] & 0xFFFFu, a.id_base + j + 2 * e));
+                best = umax64(best, cand_key(w[e] >> 16, a.id_base + j + 2 * e + 1));
+            }
+        }
+        for (int j = jv_end + threadIdx.x; j < j1; j += kArgmaxThreads) best = umax64(best, cand_key(row[j], a.id_base + j));
+    } else {
+        for (int j = j0 + threadIdx.x; j < j1; j += kArgmaxThreads) best = umax64(best, cand_key(row[j], a.id_base + j));
+    }
+    best = warp_max64(best);
+    __shared__ uint64_t red[kArgmaxThreads / 32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = best;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        uint64_t v = threadIdx.x < kArgmaxThreads / 32 ? red[threadIdx.x] : 0ull;
+        v = warp_max64(v);
+        if (threadIdx.x == 0) a.partial[(long long)m * a.blocks_per_row + b] = v;
+    }
+}
+
+// One warp per row: max over the row's partial keys, then the word.  The
+// winning value is read back from the logits so that a winning -0 keeps its sign.
+__global__ void argmax_final_kernel(ArgmaxArgs a) {
+    const int m = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (m >= a.M) return;
+    const int lane = threadIdx.x & 31;
+    uint64_t best = 0;
+    for (int b = lane; b < a.blocks_per_row; b += 32) best = umax64(best, a.partial[(long long)m * a.blocks_per_row + b]);
+    best = warp_max64(best);
+    if (lane == 0) {
+        const uint32_t id = 0x7FFFFFFFu - (uint32_t)(best & 0x7FFFFFFFull);
+        uint64_t word;
+        if (best == 0) {
+            // unreachable for n >= 1 (every element yields a nonzero key); kept so that
+            // no input can make the read below leave the row
+            word = ((uint64_t)(TF_PAIR_FLAG | a.id_base) << 32) | 0x7FC00000ull;
+        } else if (best >> 63) {
+            word = ((uint64_t)(TF_PAIR_FLAG | id) << 32) | 0x7FC00000ull;
+        } else {
+            const uint32_t h = a.logits[(long long)m * a.ld + (id - a.id_base)];
+            word = ((uint64_t)id << 32) | ((uint64_t)h << 16);
+        }
+        a.words[m] = word;
+    }
+}
+
+// Blocks per row: enough CTAs to cover the GPU a few times over for small M,
+// at least 2048 elements per block.  The scratch size is derived from it.
+int argmax_blocks_per_row(int M, int n) {
+    const int by_size = (n + 2047) / 2048;
+    int by_grid = (4 * kNumSMs + (M > 0 ? M : 1) - 1) / (M > 0 ? M : 1);
+    if (by_grid < 1) by_grid = 1;
+    int b = by_size < by_grid ? by_size : by_grid;
+    if (b < 1) b = 1;
+    if (b > 1024) b = 1024;
+    return b;
+}
+
+cudaError_t launch_argmax(ArgmaxArgs a, cudaStream_t stream) {
+    a.blocks_per_row = argmax_blocks_per_row(a.M, a.n);
+    int span = (a.n + a.blocks_per_row - 1) / a.blocks_per_row;
+    span = (span + 7) / 8 * 8;
+    a.span = span;
+    dim3 grid(a.blocks_per_row, a.M);
+    argmax_partial_kernel<<<grid, kArgmaxThreads, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    argmax_final_kernel<<<(a.M + 7) / 8, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ pick --
+// One thread per row: any flagged id word -> the sentinel; otherwise the larger
+// value, the lower id on equal values (fp32 compare: +0 == -0).
+__global__ void pick_kernel(const uint64_t *words, int nparts, int M, uint32_t *ids) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M) return;
+    bool flagged = false;
+    uint32_t best_id = 0;
+    float best_v = 0.0f;
+    for (int p = 0; p < nparts; ++p) {
+        const uint64_t w = words[(long long)p * M + m];
+        const uint32_t id = (uint32_t)(w >> 32);
+        const float v = __uint_as_float((uint32_t)w);
+        if (id & TF_PAIR_FLAG) flagged = true;
+        if (p == 0 || v > best_v || (v == best_v && id < best_id)) {
+            best_id = id;
+            best_v = v;
+        }
+    }
+    ids[m] = flagged ? TF_PICK_FAILED : best_id;
+}
+
+cudaError_t launch_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, cudaStream_t stream) {
+    pick_kernel<<<(M + 127) / 128, 128, 0, stream>>>(words, nparts, M, ids);
+    return cudaGetLastError();
+}
+
+}  // namespace tf

@@ -1,0 +1,182 @@
+// tf_abi.cu -- the extern "C" entry points of libtf.so (declared in include/tf.h).
+//
+// Each entry point validates every argument on the host and refuses a bad
+// call by status before anything is enqueued (TensorFold PR #1434 review
+// thread: refuse by name before the backend moves any state; fail closed).
+#include <climits>
+#include <cstring>
+
+#include "tf_common.cuh"
+#include "tf_kernels.h"
+
+
+using namespace tf;
+
+extern "C" {
+
+const char *tf_status_str(tf_status s) {
+    switch (s) {
+    case TF_OK: return "TF_OK";
+    case TF_E_ARG: return "TF_E_ARG";
+    case TF_E_RANGE: return "TF_E_RANGE";
+    case TF_E_ALIGN: return "TF_E_ALIGN";
+    case TF_E_WINDOW: return "TF_E_WINDOW";
+    case TF_E_BROKEN: return "TF_E_BROKEN";
+    case TF_E_CUDA: return "TF_E_CUDA";
+    case TF_E_UNIMPL: return "TF_E_UNIMPL";
+    }
+    return "TF_E_?";
+}
+
+int tf_abi_version(void) { return TF_ABI_VERSION; }
+
+tf_status tf_split_rows(int N, int nparts, int h, tf_seg *seg) {
+    if (seg == nullptr || nparts < 1 || nparts > TF_MAX_PARTS || h < 0 || h >= nparts || N < 0 || N % nparts != 0)
+        return TF_E_ARG;
+    const int w = N / nparts;
+    seg->row0 = h * w;
+    seg->nrows = w;
+    return TF_OK;
+}
+
+tf_status tf_member_segs(int F, int nparts, int h, tf_seg segs[2]) {
+    if (segs == nullptr || F > INT_MAX / 2) return TF_E_ARG;
+    tf_seg g;
+    const tf_status st = tf_split_rows(F, nparts, h, &g);
+    if (st != TF_OK) return st;
+    segs[0] = g;
+    segs[1].row0 = F + g.row0;
+    segs[1].nrows = g.nrows;
+    return TF_OK;
+}
+
+int tf_chunk_rows(int requested) {
+    if (requested < 0) return 0;
+    return requested < TF_BATCH_ROWS ? requested : TF_BATCH_ROWS;
+}
+
+size_t tf_seam_bytes(int rows, int width) {
+    if (rows <= 0 || width <= 0) return 0;
+    return (size_t)rows * (size_t)width * 2u;
+}
+
+tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
+                      const void *biases, int N_whole, const tf_seg *segs, int nseg, tf_epi epi, void *y,
+                      int ldy, tf_stream stream) {
+    if (M < 0 || M > TF_BATCH_ROWS) return TF_E_ARG;
+    if (K < TF_GROUP || K > TF_MAX_K || K % TF_GROUP != 0) return TF_E_ARG;
+    if (N_whole < 1) return TF_E_ARG;
+    if (segs == nullptr || nseg < 1 || nseg > TF_MAX_SEGS) return TF_E_ARG;
+    if (epi != TF_EPI_NONE && epi != TF_EPI_GLU) return TF_E_ARG;
+    if (epi == TF_EPI_GLU && (nseg != 2 || segs[0].nrows != segs[1].nrows)) return TF_E_ARG;
+
+    SegTable t;
+    std::memset(&t, 0, sizeof t);
+    long long cols = 0;
+    for (int i = 0; i < nseg; ++i) {
+        const long long r0 = segs[i].row0, nr = segs[i].nrows;
+        if (r0 < 0 || nr < 0 || r0 + nr > N_whole) return TF_E_RANGE;
+        for (int j = 0; j < i; ++j) {
+            const long long a0 = segs[j].row0, an = segs[j].nrows;
+            if (nr > 0 && an > 0 && r0 < a0 + an && a0 < r0 + nr) return TF_E_RANGE;
+        }
+        t.row0[i] = (int)r0;
+        t.nrows[i] = (int)nr;
+        t.col0[i] = (int)cols;
+        cols += nr;
+    }
+    t.nseg = nseg;
+    t.ncols = (epi == TF_EPI_GLU) ? segs[0].nrows : (int)cols;
+    if (cols > INT_MAX) return TF_E_RANGE;
+    if (ldx < K || ldy < t.ncols) return TF_E_ARG;
+    if (M == 0 || t.ncols == 0) return TF_OK;
+    if (!x || !wq || !scales || !biases || !y) return TF_E_ARG;
+    if (!aligned(x, 16) || ldx % 8 != 0 || !aligned(wq, 16) || !aligned(scales, 2) || !aligned(biases, 2) ||
+        !aligned(y, 2))
+        return TF_E_ALIGN;
+
+    QmmArgs a;
+    a.x = static_cast<const uint16_t *>(x);
+    a.M = M;
+    a.K = K;
+    a.ldx = ldx;
+    a.wq = wq;
+    a.scales = static_cast<const uint16_t *>(scales);
+    a.biases = static_cast<const uint16_t *>(biases);
+    a.seg = t;
+    a.glu = epi == TF_EPI_GLU;
+    a.y = static_cast<uint16_t *>(y);
+    a.ldy = ldy;
+    return launch_qmm(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_E_CUDA;
+}
+
+tf_status tf_gather_rows(void *dst, int ld_dst, const void *const *parts, const int *widths, int nparts, int M,
+                         size_t window_bytes, tf_stream stream) {
+    if (nparts < 1 || nparts > TF_MAX_PARTS || parts == nullptr || widths == nullptr || M < 0) return TF_E_ARG;
+    GatherArgs g;
+    std::memset(&g, 0, sizeof g);
+    long long total = 0;
+    bool broken = false;
+    bool vec = aligned(dst, 16) && (ld_dst % 8 == 0);
+    for (int h = 0; h < nparts; ++h) {
+        if (widths[h] < 0) return TF_E_ARG;
+        g.off[h] = (int)total;
+        total += widths[h];
+        if (total > INT_MAX) return TF_E_ARG;
+        g.part[h] = static_cast<const uint16_t *>(parts[h]);
+        g.width[h] = widths[h];
+        if (!parts[h]) broken = true;
+        if (widths[h] % 8 != 0 || (parts[h] && !aligned(parts[h], 16))) vec = false;
+        if (parts[h] && !aligned(parts[h], 2)) return TF_E_ALIGN;
+    }
+    g.off[nparts] = (int)total;
+    if (ld_dst < total) return TF_E_ARG;
+    for (int h = 0; h < nparts; ++h)
+        if (window_bytes != TF_NO_WINDOW && (size_t)M * (size_t)widths[h] * 2u > window_bytes) return TF_E_WINDOW;
+    if (M == 0 || total == 0) return broken ? TF_E_BROKEN : TF_OK;
+    if (!dst) return TF_E_ARG;
+    if (!aligned(dst, 2)) return TF_E_ALIGN;
+    g.dst = static_cast<uint16_t *>(dst);
+    g.ld_dst = ld_dst;
+    g.nparts = nparts;
+    g.M = M;
+    if (launch_gather(g, vec, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TF_E_CUDA;
+    return broken ? TF_E_BROKEN : TF_OK;
+}
+
+size_t tf_argmax_scratch_bytes(int M, int n) {
+    if (M <= 0 || n <= 0) return 0;
+    return (size_t)M * (size_t)argmax_blocks_per_row(M, n) * sizeof(uint64_t);
+}
+
+tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_base, uint64_t *words, void *scratch,
+                         size_t scratch_bytes, tf_stream stream) {
+    if (M < 0 || M > 65535 || n < 1 || ld < n) return TF_E_ARG;
+    if ((unsigned long long)id_base + (unsigned long long)n > 0x80000000ull) return TF_E_RANGE;
+    if (M == 0) return TF_OK;
+    if (!logits || !words || !scratch) return TF_E_ARG;
+    if (scratch_bytes < tf_argmax_scratch_bytes(M, n)) return TF_E_ARG;
+    if (!aligned(logits, 2) || !aligned(words, 8) || !aligned(scratch, 8)) return TF_E_ALIGN;
+    ArgmaxArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.logits = static_cast<const uint16_t *>(logits);
+    a.ld = ld;
+    a.n = n;
+    a.id_base = id_base;
+    a.M = M;
+    a.partial = static_cast<uint64_t *>(scratch);
+    a.words = words;
+    a.vec = aligned(logits, 16) && (ld % 8 == 0);
+    return launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_E_CUDA;
+}
+
+tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_stream stream) {
+    if (nparts < 1 || nparts > TF_MAX_PARTS || M < 0 || M > 65535) return TF_E_ARG;
+    if (M == 0) return TF_OK;
+    if (!words || !ids) return TF_E_ARG;
+    if (!aligned(words, 8) || !aligned(ids, 4)) return TF_E_ALIGN;
+    return launch_pick(words, nparts, M, ids, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK
+                                                                                                     : TF_E_CUDA;
+}
+
+}  // extern "C"

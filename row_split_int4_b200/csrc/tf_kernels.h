@@ -1,0 +1,64 @@
+// tf_kernels.h -- launch arguments and host launchers shared by the
+// translation units of libtf.so (internal; the public ABI is include/tf.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/tf.h"
+
+namespace tf {
+
+// Output columns of one qmm call: segment i covers columns [col0[i], col0[i] + nrows[i])
+// and whole-matrix rows [row0[i], row0[i] + nrows[i]).
+struct SegTable {
+    int row0[TF_MAX_SEGS];
+    int nrows[TF_MAX_SEGS];
+    int col0[TF_MAX_SEGS];
+    int nseg;
+    int ncols;   // sum of nrows (TF_EPI_NONE) or the common nrows (TF_EPI_GLU)
+};
+
+struct QmmArgs {
+    const uint16_t *x;
+    int M, K, ldx;
+    const uint8_t *wq;
+    const uint16_t *scales;
+    const uint16_t *biases;
+    SegTable seg;
+    int glu;
+    uint16_t *y;
+    int ldy;
+};
+
+struct GatherArgs {
+    uint16_t *dst;
+    long long ld_dst;
+    const uint16_t *part[TF_MAX_PARTS];
+    int width[TF_MAX_PARTS];
+    int off[TF_MAX_PARTS + 1];
+    int nparts;
+    int M;
+};
+
+struct ArgmaxArgs {
+    const uint16_t *logits;
+    long long ld;
+    int n;
+    uint32_t id_base;
+    int M;
+    int blocks_per_row;
+    int span;              // elements per block (multiple of 8)
+    uint64_t *partial;     // [M][blocks_per_row] keys
+    uint64_t *words;       // [M]
+    int vec;               // 16-byte loads allowed
+};
+
+cudaError_t launch_qmm(const QmmArgs &a, cudaStream_t stream);
+cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream);
+cudaError_t launch_argmax(ArgmaxArgs a, cudaStream_t stream);
+cudaError_t launch_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, cudaStream_t stream);
+int argmax_blocks_per_row(int M, int n);
+int num_sms();
+
+}  // namespace tf
