@@ -20,84 +20,12 @@
 // in a segment, or on the grid, so split == whole holds bit for bit.
 #include "tf_common.cuh"
 #include "tf_kernels.h"
+#include "qmm_common.cuh"
 
 namespace tf {
 
-constexpr int kChunk = 1024;             // k per warp-wide 16-byte load of packed codes
 constexpr int kWarps = 8;                // warps per CTA
 constexpr int kSlots = 4;                // weight rows a warp carries at once
-
-// Whole-matrix row of output column `col` (NONE), or of member `which`
-// (0 = gate, 1 = up) of column `col` (GLU).
-__device__ __forceinline__ int seg_row(const SegTable &t, int col, int glu, int which) {
-    if (glu) return t.row0[which] + col;
-    int r = -1;
-#pragma unroll
-    for (int s = 0; s < TF_MAX_SEGS; ++s)
-        if (s < t.nseg && col >= t.col0[s] && col < t.col0[s] + t.nrows[s]) r = t.row0[s] + (col - t.col0[s]);
-    return r;
-}
-
-// 8 codes of one 32-bit word -> fp32, exactly.  Each nibble is masked in place
-// and OR-ed with the exponent that makes its bit position worth 1, so the
-// float holds 2^E + q; subtracting 2^E leaves q.  Positions 0..4 are read
-// from w, positions 5..7 from w >> 12.
-struct Codes8 {
-    float f[8];
-};
-__device__ __forceinline__ Codes8 decode8(uint32_t w) {
-    const uint32_t h = w >> 12;
-    Codes8 c;
-    c.f[0] = __uint_as_float((w & 0x0000000Fu) | 0x4B000000u) - 8388608.0f;  // 2^23
-    c.f[1] = __uint_as_float((w & 0x000000F0u) | 0x49000000u) - 524288.0f;   // 2^19
-    c.f[2] = __uint_as_float((w & 0x00000F00u) | 0x47000000u) - 32768.0f;    // 2^15
-    c.f[3] = __uint_as_float((w & 0x0000F000u) | 0x45000000u) - 2048.0f;     // 2^11
-    c.f[4] = __uint_as_float((w & 0x000F0000u) | 0x43000000u) - 128.0f;      // 2^7
-    c.f[5] = __uint_as_float((h & 0x00000F00u) | 0x47000000u) - 32768.0f;
-    c.f[6] = __uint_as_float((h & 0x0000F000u) | 0x45000000u) - 2048.0f;
-    c.f[7] = __uint_as_float((h & 0x000F0000u) | 0x43000000u) - 128.0f;
-    return c;
-}
-
-// P = sum_{i<32} q_i x_i for one lane-chunk, two accumulators (even/odd i).
-// xv[j] holds x for the lane's elements 4j..4j+3.
-__device__ __forceinline__ float lane_chunk_dot(const uint4 &q, const float4 *xv) {
-    float pe = 0.0f, po = 0.0f;
-    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        Codes8 c = decode8(words[w]);
-        const float4 a = xv[2 * w], b = xv[2 * w + 1];
-        pe = fmaf(c.f[0], a.x, pe);
-        po = fmaf(c.f[1], a.y, po);
-        pe = fmaf(c.f[2], a.z, pe);
-        po = fmaf(c.f[3], a.w, po);
-        pe = fmaf(c.f[4], b.x, pe);
-        po = fmaf(c.f[5], b.y, po);
-        pe = fmaf(c.f[6], b.z, pe);
-        po = fmaf(c.f[7], b.w, po);
-    }
-    return pe + po;
-}
-
-// X = ascending fp32 sum of the lane's 32 x values.
-__device__ __forceinline__ float lane_chunk_xsum(const float4 *xv) {
-    float s = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        s += xv[j].x;
-        s += xv[j].y;
-        s += xv[j].z;
-        s += xv[j].w;
-    }
-    return s;
-}
-
-__device__ __forceinline__ float warp_sum_to_lane0(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xFFFFFFFFu, v, o);
-    return v;
-}
 
 // Read-once weight stream: bypass L1.
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
@@ -386,6 +314,7 @@ constexpr size_t kM1SmemMax = 200 * 1024;
 
 cudaError_t launch_qmm(const QmmArgs &a, cudaStream_t stream) {
     const int ncols = a.seg.ncols;
+    if (qmm_m1_stream_eligible(a)) return launch_qmm_m1_stream(a, stream);
     if (a.M == 1 && qmm_m1_smem_bytes(a.K) <= kM1SmemMax) {
         const size_t smem = qmm_m1_smem_bytes(a.K);
         const int dev = current_device();
