@@ -26,7 +26,7 @@
  *            ties (PR #1433 step-1 body; step-2 body: the pick is the better of
  *            the two half-vocab winners).
  *
- * Readings taken where the pages are silent (all listed in the design doc):
+ * Readings taken where the pages are silent:
  *   nibble order  element k lives in byte k/2 of its row, low nibble for even k;
  *   q             unsigned 0..15, no separate zero point (the bias carries it);
  *   rounding      round-to-nearest-even straight from double to bf16, NaN -> 0x7FC0;
