@@ -121,7 +121,7 @@ void orc_bf16_rne_array(const double *v, uint16_t *out, int64_t n)
 
 /* --------------------------------------------------------------- dequant -- */
 
-/* q of element k of one packed row (C1 reading: byte k/2, low nibble = even k). */
+/* q of element k of one packed row (byte k/2, low nibble for even k). */
 static unsigned orc_nibble(const uint8_t *row, int64_t k)
 {
     uint8_t byte = row[k >> 1];
