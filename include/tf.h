@@ -189,6 +189,33 @@ tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_b
 tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_stream stream);
 
 /*
+ * tf_argmax_rows_static -- tf_argmax_rows for callers that cannot allocate
+ * device memory.  The pages have no counterpart of this entry point; it exists
+ * for hosts that own every byte of device memory up front (a fixed arena that
+ * forbids any other cudaMalloc) and for latency paths where the implicit
+ * device synchronisation of cudaMalloc/cudaFree is not acceptable.
+ *
+ * Same arguments, result and errors as tf_argmax_rows, without the scratch
+ * arguments: the per-block partial results go to a device array built into
+ * libtf.so (TF_STATIC_SCRATCH_BYTES bytes, present on every GPU that loads the
+ * library, for as long as the process lives).  Nothing is allocated and no
+ * allocating routine is called.
+ *   - TF_E_ARG when tf_argmax_scratch_bytes(M, n) > TF_STATIC_SCRATCH_BYTES
+ *     (for example M = 8,193 rows of any length); nothing is enqueued.
+ *   - The first call on a device looks up that array's device address
+ *     (cudaGetSymbolAddress, with the device current) and keeps it; make that
+ *     first call before any stream capture.  A failed lookup returns TF_E_CUDA.
+ *   - Every call on a device uses the same array, and the array keeps what the
+ *     last call left there.  Each call writes every entry it later reads, so no
+ *     clearing is needed, but two calls whose kernels overlap on the GPU (other
+ *     streams, or other host threads) race on it: order them on one stream, or
+ *     use tf_argmax_rows with a scratch buffer per stream.
+ */
+#define TF_STATIC_SCRATCH_BYTES ((size_t)64 * 1024)
+tf_status tf_argmax_rows_static(const void *logits, int M, int n, int ld, uint32_t id_base, uint64_t *words,
+                                tf_stream stream);
+
+/*
  * Host arithmetic of the row split (TensorFold PR #1433 step-2 body: the split
  * is by output rows, rank 0's spans start at 0; 2,560 of 5,120, 8,704 of
  * 17,408, 124,160 of 248,320; "the fused gate-up keeps the member split").

@@ -34,11 +34,12 @@ TF_MAX_K = 65536
 TF_MAX_SEGS = 8
 TF_MAX_PARTS = 8
 TF_NO_WINDOW = ctypes.c_size_t(-1).value
+TF_STATIC_SCRATCH_BYTES = 64 * 1024
 TF_EPI_NONE, TF_EPI_GLU = 0, 1
 
 EXPORTS = ["tf_qmm_rows", "tf_gather_rows", "tf_argmax_scratch_bytes", "tf_argmax_rows", "tf_pick",
            "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str",
-           "tf_abi_version"]
+           "tf_abi_version", "tf_argmax_rows_static"]
 
 
 class tf_seg(ctypes.Structure):
@@ -54,6 +55,8 @@ lib.tf_argmax_scratch_bytes.restype = _sz
 lib.tf_argmax_scratch_bytes.argtypes = [_i, _i]
 lib.tf_argmax_rows.restype = _i
 lib.tf_argmax_rows.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _sz, _vp]
+lib.tf_argmax_rows_static.restype = _i
+lib.tf_argmax_rows_static.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp]
 lib.tf_pick.restype = _i
 lib.tf_pick.argtypes = [_vp, _i, _i, _vp, _vp]
 lib.tf_split_rows.restype = _i
@@ -164,6 +167,17 @@ def tf_argmax_rows(logits: torch.Tensor, id_base: int, words: torch.Tensor, scra
     st = lib.tf_argmax_rows(_ptr(logits), M, n, _ld(logits), int(id_base), _ptr(words), _ptr(scratch),
                             scratch.numel(), _stream(stream))
     return _ret(st, "tf_argmax_rows", check)
+
+
+def tf_argmax_rows_static(logits: torch.Tensor, id_base: int, words: torch.Tensor, stream=None,
+                          check: bool = True) -> int:
+    """tf_argmax_rows without a scratch buffer, for callers that cannot allocate
+    device memory: the library's own TF_STATIC_SCRATCH_BYTES device array holds
+    the partial results.  Calls that overlap on the GPU must not share it."""
+    assert logits.dtype == torch.bfloat16 and words.dtype == torch.int64
+    M, n = logits.shape
+    st = lib.tf_argmax_rows_static(_ptr(logits), M, n, _ld(logits), int(id_base), _ptr(words), _stream(stream))
+    return _ret(st, "tf_argmax_rows_static", check)
 
 
 def tf_pick(words: torch.Tensor, ids: torch.Tensor, stream=None, check: bool = True) -> int:
