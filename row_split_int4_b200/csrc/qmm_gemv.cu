@@ -315,6 +315,7 @@ constexpr size_t kM1SmemMax = 200 * 1024;
 cudaError_t launch_qmm(const QmmArgs &a, cudaStream_t stream) {
     const int ncols = a.seg.ncols;
     if (qmm_m1_stream_eligible(a)) return launch_qmm_m1_stream(a, stream);
+    if (qmm_tc_eligible(a)) return launch_qmm_tc(a, stream);
     if (a.M == 1 && qmm_m1_smem_bytes(a.K) <= kM1SmemMax) {
         const size_t smem = qmm_m1_smem_bytes(a.K);
         const int dev = current_device();

@@ -107,6 +107,7 @@ tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, c
     a.glu = epi == TF_EPI_GLU;
     a.y = static_cast<uint16_t *>(y);
     a.ldy = ldy;
+    a.n_whole = N_whole;
     return launch_qmm(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_E_CUDA;
 }
 

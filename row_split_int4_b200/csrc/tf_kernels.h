@@ -29,6 +29,7 @@ struct QmmArgs {
     int glu;
     uint16_t *y;
     int ldy;
+    int n_whole;   // rows of the whole matrix (the call may cover only some of them)
 };
 
 struct GatherArgs {
@@ -59,6 +60,8 @@ cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream);
 cudaError_t launch_argmax(ArgmaxArgs a, cudaStream_t stream);
 cudaError_t launch_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, cudaStream_t stream);
 bool qmm_m1_stream_eligible(const QmmArgs &a);
+bool qmm_tc_eligible(const QmmArgs &a);
+cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream);
 cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream);
 int argmax_blocks_per_row(int M, int n);
 int num_sms();
