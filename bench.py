@@ -58,6 +58,32 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s of this machine's B200s (burst, for a kernel timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def max_over_ranks(values, world, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank times: the slowest rank decides a
+    whole-job figure.  With one rank the values come back unchanged."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_value(bytes_per_step, world, steps, elapsed_ms):
+    """Whole-job GB/s of `world` independent replicas, each moving
+    `bytes_per_step` per step, over the slowest rank's time."""
+    return bytes_per_step * world * steps / (elapsed_ms / 1e3) / 1e9
+
+
 def qmm_bytes(K, rows, M=1, out_cols=None):
     """Algorithmic bytes of one qmm call: 0.5625 B per weight + x read + y written."""
     out_cols = rows if out_cols is None else out_cols
@@ -326,8 +352,92 @@ def run_kernel(args):
 
 
 # --------------------------------------------------------------------------- sweep
+SWEEP_M = (1, 2, 4, 8, 16, 32, 64, 128)
+SWEEP_SHAPES = {   # name: (whole rows, K, epilogue); every point runs the two row halves
+    "attn_out": (5120, 5120, 0),
+    "gate_up": (34816, 5120, 1),
+    "down": (5120, 17408, 0),
+    "lm_head": (248320, 5120, 0),
+}
+L2_BYTES = 126 * 1024 * 1024
+
+
 def run_sweep(args):
-    raise SystemExit("--sweep: not available yet")
+    """M in {1..128} over the four shapes, each point the two row halves of the
+    shape (plus both argmaxes and the pick for lm_head), --reps back-to-back
+    repetitions timed with CUDA events.  The weights stay in HBM; each shape is
+    replicated into enough separate buffers to span 3 x L2 and the repetitions
+    rotate through them, so a repetition never finds its weights in L2, and a
+    512 MB write flushes L2 between shapes.  One JSON line per point."""
+    import torch
+    import row_split_int4_b200 as tf
+    import synth
+    torch.cuda.set_device(0)
+    peak_hbm, hbm_kind = measured_peak()
+    peak_tc, tc_kind = measured_tensor_peak()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    shapes = [s for s in SWEEP_SHAPES if not args.shapes or s in args.shapes.split(",")]
+    Ms = [int(m) for m in args.sweep_m.split(",")] if args.sweep_m else list(SWEEP_M)
+    for name in shapes:
+        N, K, epi = SWEEP_SHAPES[name]
+        tag = {"attn_out": synth.TAG_ATTN, "gate_up": synth.TAG_W, "down": synth.TAG_W2, "lm_head": synth.TAG_HEAD}[name]
+        w = synth.weights_to_device(synth.make_weights(N, K, seed=args.seed, tag=tag))
+        wbytes = sum(t.numel() * t.element_size() for t in w)
+        nrep = max(1, -(-3 * L2_BYTES // wbytes))
+        replicas = [w] + [tuple(t.clone() for t in w) for _ in range(nrep - 1)]
+        x = synth.to_device(synth.make_x(max(Ms), K, seed=args.seed, tag=synth.TAG_X))
+        if epi:
+            segs = [tf.tf_member_segs(N // 2, 2, h) for h in range(2)]
+            cols = N // 4
+        else:
+            segs = [[tf.tf_split_rows(N, 2, h)] for h in range(2)]
+            cols = N // 2
+        y = [torch.empty(max(Ms), cols, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        head = name == "lm_head"
+        if head:
+            ids = torch.empty(max(Ms), dtype=torch.int32, device="cuda")
+            scratch = torch.empty(tf.tf_argmax_scratch_bytes(max(Ms), cols), dtype=torch.uint8, device="cuda")
+        for M in Ms:
+            if head:
+                words = torch.empty(2, M, dtype=torch.int64, device="cuda")   # [half][M], contiguous
+
+            def rep(r):
+                wr = replicas[r % nrep]
+                for h in range(2):
+                    tf.tf_qmm_rows(x[:M], *wr, segs[h], y[h][:M], epi=epi, stream=stream)
+                if head:
+                    for h in range(2):
+                        tf.tf_argmax_rows(y[h][:M], segs[h][0][0], words[h], scratch, stream=stream)
+                    tf.tf_pick(words, ids[:M], stream=stream)
+            flush.zero_()
+            for r in range(max(3, args.warmup)):
+                rep(r)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            sampler = ClockSampler(0)
+            with sampler:
+                e0.record(stream)
+                for r in range(args.reps):
+                    rep(r)
+                e1.record(stream)
+                torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / args.reps
+            nbytes = 2 * qmm_bytes(K, N // 2, M=M, out_cols=cols) + (2 * M * N + 2 * 8 * M + 4 * M if head else 0)
+            flops = 2.0 * M * K * N
+            t_hbm, t_tc = nbytes / (peak_hbm * 1e3), flops / (peak_tc * 1e6)   # microseconds
+            bound = "hbm" if t_hbm >= t_tc else "tensor"
+            print(json.dumps({
+                "sweep": name, "M": M, "K": K, "rows": N, "reps": args.reps, "us_per_rep": round(us, 3),
+                "GB/s": round(nbytes / us / 1e3, 1), "TFLOP/s": round(flops / us / 1e6, 2),
+                "hbm_frac": round(nbytes / us / 1e3 / peak_hbm, 4), "tensor_frac": round(flops / us / 1e6 / peak_tc, 4),
+                "bound": bound, "roofline_frac": round(max(t_hbm, t_tc) / us, 4),
+                "peaks": {"hbm_gbs": peak_hbm, "bf16_tflops": peak_tc, "kind": f"{hbm_kind}/{tc_kind}"},
+                "weight_replicas": nrep, "l2": "replicas span 3 x L2; L2 flushed between points",
+                "clocks": sampler.summary()}), flush=True)
+        del replicas, w, x, y
+        torch.cuda.empty_cache()
+    return 0
 
 
 # --------------------------------------------------------------------------- main arm
@@ -344,6 +454,8 @@ def main():
     ap.add_argument("--reps", type=int, default=1000)
     ap.add_argument("--kernel", choices=sorted(KERNELS), help="time one qmm call of the step (profiling driver)")
     ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--shapes", default="", help="sweep: comma-separated subset of " + ",".join(SWEEP_SHAPES))
+    ap.add_argument("--sweep-m", default="", help="sweep: comma-separated M values")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     if args.impl == "reference":
@@ -431,14 +543,11 @@ def main():
                "d2h": step.y.numel() * 2 + step.ids.numel() * 4}
 
     # max over ranks
-    vals = torch.tensor([elapsed_ms, e2e["e2e_ms"] if e2e else 0.0], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(vals[0]), float(vals[1])
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e["e2e_ms"] if e2e else 0.0], world, dist, device="cuda")
 
     if rank == 0:
         ms_step = elapsed_ms / K
-        value = nb["total"] * world * K / (elapsed_ms / 1e3) / 1e9
+        value = job_value(nb["total"], world, K, elapsed_ms)
         peak, peak_kind = measured_peak()
         lm_bytes = qmm_bytes(5120, 248320 // 2)
         lm_avg_ms = statistics.fmean(lm_ms)
@@ -461,7 +570,7 @@ def main():
             "clocks": sampler.summary(),
         }
         if e2e:
-            line["e2e"] = {"value": round(nb["total"] * world / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            line["e2e"] = {"value": round(job_value(nb["total"], world, 1, e2e_ms), 2), "unit": "GB/s",
                            "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                            "ms_per_step": round(e2e_ms, 5)}
         if not args.no_cpu_baseline and world == 1:

@@ -244,6 +244,12 @@ size_t tf_seam_bytes(int rows, int width);
 /* Static name of a status ("TF_OK", "TF_E_ARG", ...); "TF_E_?" for an unknown value. */
 const char *tf_status_str(tf_status s);
 
+/* The CUDA runtime's message for the error behind the last TF_E_CUDA that a
+ * tf_* call returned on the calling host thread ("no error" before any).  The
+ * string has static storage; the call never fails and never returns NULL.
+ * Not an operation of the pages: it only makes TF_E_CUDA diagnosable. */
+const char *tf_last_cuda_error(void);
+
 /* ABI version of this header; bumped when a signature changes. */
 #define TF_ABI_VERSION 1
 int tf_abi_version(void);

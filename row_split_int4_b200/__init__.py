@@ -38,7 +38,7 @@ TF_STATIC_SCRATCH_BYTES = 64 * 1024
 TF_EPI_NONE, TF_EPI_GLU = 0, 1
 
 EXPORTS = ["tf_qmm_rows", "tf_gather_rows", "tf_argmax_scratch_bytes", "tf_argmax_rows", "tf_pick",
-           "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str",
+           "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str", "tf_last_cuda_error",
            "tf_abi_version", "tf_argmax_rows_static"]
 
 
@@ -69,6 +69,8 @@ lib.tf_seam_bytes.restype = _sz
 lib.tf_seam_bytes.argtypes = [_i, _i]
 lib.tf_status_str.restype = ctypes.c_char_p
 lib.tf_status_str.argtypes = [_i]
+lib.tf_last_cuda_error.restype = ctypes.c_char_p
+lib.tf_last_cuda_error.argtypes = []
 lib.tf_abi_version.restype = _i
 lib.tf_abi_version.argtypes = []
 
@@ -76,11 +78,19 @@ lib.tf_abi_version.argtypes = []
 class TFError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {tf_status_str(status)}")
+        msg = f"{where}: {tf_status_str(status)}"
+        if status == TF_E_CUDA:
+            msg += f" ({tf_last_cuda_error()})"
+        super().__init__(msg)
 
 
 def tf_status_str(status: int) -> str:
     return lib.tf_status_str(int(status)).decode()
+
+
+def tf_last_cuda_error() -> str:
+    """The CUDA runtime's message behind the last TF_E_CUDA on this thread."""
+    return lib.tf_last_cuda_error().decode()
 
 
 def tf_split_rows(N: int, nparts: int, h: int) -> Tuple[int, int]:

@@ -45,7 +45,7 @@ extern "C" tf_status tf_argmax_rows_static(const void *logits, int M, int n, int
     if (tf_argmax_scratch_bytes(M, n) > TF_STATIC_SCRATCH_BYTES) return TF_E_ARG;
     if (!aligned(logits, 2) || !aligned(words, 8)) return TF_E_ALIGN;
     void *scratch = nullptr;
-    if (static_scratch(&scratch) != cudaSuccess) return TF_E_CUDA;
+    if (cuda_status(static_scratch(&scratch)) != TF_OK) return TF_E_CUDA;
     ArgmaxArgs a;
     std::memset(&a, 0, sizeof a);
     a.logits = static_cast<const uint16_t *>(logits);
@@ -56,5 +56,5 @@ extern "C" tf_status tf_argmax_rows_static(const void *logits, int M, int n, int
     a.partial = static_cast<uint64_t *>(scratch);
     a.words = words;
     a.vec = aligned(logits, 16) && (ld % 8 == 0);
-    return launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_E_CUDA;
+    return cuda_status(launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)));
 }

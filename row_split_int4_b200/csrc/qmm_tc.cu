@@ -1,39 +1,50 @@
 // qmm_tc.cu -- prompt-chunk qmm (M = 2..128 activation rows) on the 5th-generation
-// tensor cores: tcgen05.mma with the weights dequantised into tensor memory (the
-// A operand), the activations in shared memory (the B operand) and the fp32
-// accumulator in tensor memory.
+// tensor cores.
 //
-// A tile is 128 weight rows (the MMA's M) against all M activation rows of the
-// call (the MMA's N, rounded up to a multiple of 16; the extra rows are zero).
-// A tile never straddles two segments of the call; with TF_EPI_GLU its rows
-// 0-63 are gate rows and 64-127 the up rows of the same outputs.
+// The weights enter the tensor core as their 4-bit codes, held exactly in bf16
+// as 128 + q (128..143), so one group of 64 values gives
+// D_g = sum_{k in g} (128 + q_k) x_k per weight row and activation row, with the
+// fp32 sums in tensor memory.  The group's scale and bias are applied on the CUDA
+// cores:
+//     y += s_g * D_g + (b_g - 128 s_g) * X_g,        X_g = sum_{k in g} x_k,
+// which is sum_{k in g} x_k (s_g q_k + b_g) -- the affine format's dot product,
+// with no rounded copy of the weights anywhere (b_g - 128 s_g is exact in fp32).
+// Per output the fp32 sum runs over the groups in ascending order, an order fixed
+// by K alone.
 //
-// The K loop runs in stages of 64 values (one scale group):
-//   * warp 0, one thread: per stage one TMA copy of the activation tile [N x 64]
-//     (128-byte swizzle) and two of the tile's packed codes [2 x 64 rows x 32 B]
-//     into a four-deep ring in shared memory.  No multicast.
-//   * warps 2-5, one thread per weight row (= tensor-memory lane): take the
-//     row's 64 codes from the ring and its scale and bias (loaded eight groups
-//     at a time, one period ahead), form w = s*q + b in fp32, split it into two
-//     bf16, hi = RN(w) and lo = RN(w - hi), and store both into one of two
-//     A stages in tensor memory (tcgen05.st).  hi + lo carries w's 16
-//     significant bits, so the contraction sees the weights of the 4-bit format,
-//     not a rounded copy of them.
-//   * warp 1, one thread: tcgen05.mma kind::f16 with A in tensor memory, four
-//     K=16 steps per stage, each on hi and then on lo, into one accumulator;
-//     tcgen05.commit releases the ring slot and the A stage.
+// A tile is 128 weight rows (the MMA's M) against the call's M activation rows
+// (the MMA's N: 16, 32, 64 or 128, the rows past M zero).  A tile never
+// straddles two segments; with TF_EPI_GLU its rows 0-63 are gate rows and
+// 64-127 the up rows of the same outputs.  Two CTAs per SM for N <= 32 (each
+// with half of tensor memory), one CTA per SM above; 10 to 22 warps:
+//   * warp 0, one thread: per group one TMA copy of the activation tile
+//     [N x 64] (128-byte swizzle) and two of the tile's packed codes
+//     [2 x 64 rows x 32 B] into a ring of 8 to 16 slots in shared memory.  No
+//     multicast.
+//   * 4 or 8 decoder warps, one thread per weight row (= tensor-memory lane):
+//     the row's codes -> bf16 pairs, stored into an A stage in tensor memory
+//     (tcgen05.st), software-pipelined so that a store drains while the next
+//     group is decoded; four of them, one thread per activation row, also form
+//     X_g from the activation tile.
+//   * warp 1, one thread: tcgen05.mma kind::f16, A from tensor memory, B (the
+//     activations) from shared memory, four K=16 steps per group into one of
+//     several D buffers; tcgen05.commit releases the ring slot and the A stage and
+//     publishes the D buffer.
+//   * scale warps, per tensor-memory lane quarter one per 32 activation rows
+//     (4 to 16 warps): read D_g (tcgen05.ld), fold it and X_g into fp32
+//     accumulators held in registers, release the D buffer.
 //
-// Split K.  The stages are cut into `ks` slices, given to the `ks` CTAs of one
-// thread-block cluster; ks and the cut are functions of K and of the whole
-// matrix's row count only (never of M, of the segments, or of the device), so a
-// row's result does not depend on which call or which half computes it.  Each
-// CTA moves its accumulator to shared memory; after a cluster barrier CTA r
-// reads the partial sums of all CTAs of the cluster through distributed shared
-// memory for its share of the activation rows, adds them in rank order in fp32,
-// rounds to bf16 (and applies gate*SiLU(up) with TF_EPI_GLU), and writes y.
+// Split K.  The groups are cut into `ks` slices, one per CTA of a thread-block
+// cluster of `ks` CTAs; ks and the cut depend on K and the whole matrix's row
+// count only (never on M, the segments or the device), so a row's result does
+// not depend on which call or which half computes it.  Each CTA puts its
+// accumulators in shared memory; after a cluster barrier CTA r reads the partial
+// sums of the whole cluster through distributed shared memory for its share of
+// the activation rows, adds them in rank order in fp32, rounds to bf16 (and
+// forms gate*SiLU(up) with TF_EPI_GLU) and writes y.
 //
 // Every wait on an mbarrier is bounded; a wait that gives up marks the CTA
-// failed, and every output the cluster writes becomes NaN.  All threads still
+// failed and every output the cluster writes becomes NaN.  All threads still
 // reach both cluster barriers, and tensor memory is released before exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -44,27 +55,56 @@
 
 namespace tf {
 
-constexpr int kTcRows = 128;       // weight rows per tile (MMA M)
-constexpr int kTcK = 64;           // K per stage
-constexpr int kTcRing = 4;         // activation + code ring depth
-constexpr int kTcAStages = 2;      // A stages in tensor memory
-constexpr int kTcThreads = 192;    // 6 warps
-constexpr int kTcMaxN = 128;       // activation rows per call
-constexpr int kTcMaxSplit = 8;     // CTAs per cluster
-constexpr int kTcXBytes = kTcMaxN * kTcK * 2;       // 16 KB
-constexpr int kTcCBytes = kTcRows * kTcK / 2;       // 4 KB of codes
-constexpr int kTcSlot = kTcXBytes + kTcCBytes;      // 20 KB, a multiple of 1 KB
-constexpr int kTcRingBytes = kTcRing * kTcSlot;     // 80 KB; later the partial sums
-constexpr int kTcSmem = kTcRingBytes + 256 /* barriers, flag */ + 1024 /* alignment */;
-constexpr uint32_t kTcTmemCols = 256;              // accumulator 128 + 2 x (hi 32 + lo 32)
+constexpr int kTcRows = 128;                    // weight rows per tile (MMA M)
+constexpr int kTcK = 64;                        // K per group / pipeline stage
+constexpr int kTcXbSlots = 8;                   // X_g slots in shared memory
+// Per MMA N: CTAs per SM (two for N <= 32, each with half of tensor memory),
+// decoder and scale warps, and pipeline depths.  Ring slot: the activation tile
+// (N x 128 B) and the codes (4 KB).  Tensor memory: tc_dbufs(N) D buffers of N
+// columns from column 0, tc_astages(N) A stages of 32 columns at the top.
+__host__ __device__ constexpr int tc_ctas_per_sm(int n) { return n <= 32 ? 2 : 1; }
+__host__ __device__ constexpr uint32_t tc_tmem_cols(int n) { return n <= 32 ? 256u : 512u; }
+__host__ __device__ constexpr int tc_dec_warps(int n) { return n == 64 ? 8 : 4; }
+// Scale warps: per tensor-memory lane quarter one warp per 32 activation rows.
+__host__ __device__ constexpr int tc_scale_warps(int n) { return 4 * (n < 32 ? 1 : n / 32); }
+__host__ __device__ constexpr int tc_threads(int n) { return 32 * (2 + tc_dec_warps(n) + tc_scale_warps(n)); }
+__host__ __device__ constexpr int tc_slot_bytes(int n) { return n * kTcK * 2 + kTcRows * kTcK / 2; }
+__host__ __device__ constexpr int tc_ring(int n) { return n == 16 ? 16 : (n == 32 ? 12 : (n == 64 ? 12 : 8)); }
+__host__ __device__ constexpr int tc_astages(int n) { return n == 64 ? 8 : 4; }
+__host__ __device__ constexpr int tc_dbufs(int n) {
+    return (int)(tc_tmem_cols(n) - 32 * tc_astages(n)) / n < 8 ? (int)(tc_tmem_cols(n) - 32 * tc_astages(n)) / n : 8;
+}
+constexpr int kTcMaxN = 128;                    // activation rows per call
+constexpr int kTcMaxSplit = 8;                  // CTAs per cluster
+constexpr int kTcCBytes = kTcRows * kTcK / 2;   // 4 KB of codes per group
+constexpr int kTcXbBytes = kTcXbSlots * kTcMaxN * 4;
+constexpr int kTcBarBytes = 1024;               // mbarriers, TMEM address, failure flag
+__host__ __device__ constexpr int tc_num_bars(int n) {
+    return 3 * tc_ring(n) + 2 * tc_astages(n) + 2 * tc_dbufs(n) + 2 * kTcXbSlots;
+}
+// Shared memory per CTA.  A CTA that takes all 512 tensor-memory columns asks for
+// more than half of the SM's shared memory, so that a second CTA is never placed
+// beside it only to wait in tcgen05.alloc; with two CTAs per SM each fits in half.
+__host__ __device__ constexpr int tc_smem_need(int n) { return tc_ring(n) * tc_slot_bytes(n) + kTcXbBytes + kTcBarBytes + 1024; }
+__host__ __device__ constexpr int tc_smem_bytes(int n) {
+    return tc_ctas_per_sm(n) == 2 ? tc_smem_need(n) : (tc_smem_need(n) > 120 * 1024 ? tc_smem_need(n) : 120 * 1024);
+}
 constexpr long long kTcSpin = 1ll << 24;
-static_assert(kTcMaxN * kTcRows * 4 <= kTcRingBytes, "partial sums must fit in the ring");
+template <int N>
+struct TcChecks {
+    static_assert(tc_slot_bytes(N) % 1024 == 0, "ring slots keep the 1 KB alignment of the swizzled tile");
+    static_assert(N * kTcRows * 4 <= tc_ring(N) * tc_slot_bytes(N), "partial sums must fit in the ring");
+    static_assert(tc_num_bars(N) * 8 + 8 <= kTcBarBytes, "barrier area");
+    static_assert(tc_dbufs(N) >= 2 && tc_dbufs(N) * N + 32 * tc_astages(N) <= (int)tc_tmem_cols(N), "tensor memory map");
+    static_assert(tc_smem_bytes(N) <= 227 * 1024, "shared memory");
+    static_assert(tc_ctas_per_sm(N) == 1 || (tc_smem_bytes(N) + 1024) * 3 > 228 * 1024, "at most two CTAs per SM");
+    static_assert(tc_ctas_per_sm(N) == 2 || (tc_smem_bytes(N) + 1024) * 2 > 228 * 1024, "one CTA per SM");
+};
 
 // Plan of one launch, computed on the host.
 struct TcPlan {
     int ks;                        // CTAs per cluster (K slices)
-    int periods;                   // K / 512: eight stages each
-    int n_mma;                     // MMA N
+    int periods;                   // K / 512: eight groups each
     int ntiles;
     int tstart[TF_MAX_SEGS + 1];   // first tile of each segment (TF_EPI_NONE)
 };
@@ -158,15 +198,48 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t dtm, uint32_t atm, uint64_t b
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t *r) {
+
+template <int X>
+__device__ __forceinline__ void tc_ld(uint32_t taddr, uint32_t *r);
+template <>
+__device__ __forceinline__ void tc_ld<8>(uint32_t taddr, uint32_t *r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tc_ld<16>(uint32_t taddr, uint32_t *r) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
                    "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
                  : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-// 32 consecutive 32-bit columns of this thread's lane.
-__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t *v) {
+template <>
+__device__ __forceinline__ void tc_ld<32>(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// X consecutive 32-bit columns of this thread's lane.
+template <int X>
+__device__ __forceinline__ void tc_st(uint32_t taddr, const uint32_t *v);
+template <>
+__device__ __forceinline__ void tc_st<16>(uint32_t taddr, const uint32_t *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+template <>
+__device__ __forceinline__ void tc_st<32>(uint32_t taddr, const uint32_t *v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
         "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
@@ -177,23 +250,27 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t *v) {
         : "memory");
 }
 
-// Two fp32 -> packed bf16x2 (first argument in the low half), round to nearest even.
-__device__ __forceinline__ uint32_t tc_pack_bf16(float lo_half, float hi_half) {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi_half), "f"(lo_half));
-    return r;
+// Codes 2j and 2j+1 of a packed word as the bf16 pair (128 + q_2j, 128 + q_2j+1),
+// exactly (code 2j in the low half).  w holds code i at bits 4i, ws = w >> 4.
+// Byte j of w has code 2j in its low nibble, byte j of ws has code 2j+1 there;
+// prmt puts them at bits 0 and 16, the mask keeps the nibbles and ORs in the
+// bf16 exponent of 128.  The offset 128 is taken out with the bias term.
+template <int j>
+__device__ __forceinline__ uint32_t tc_code_pair(uint32_t w, uint32_t ws) {
+    constexpr uint32_t sel = j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12);
+    uint32_t p;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(p) : "r"(w), "r"(ws), "n"(sel));
+    return (p & 0x000F000Fu) | 0x43004300u;
 }
 
-// 8 codes of a word -> the hi and lo bf16 pairs of w = s*q + b (element 2p in
-// the low half of pair p).  hi = RN(w); w - hi is exact in fp32 and lo = RN(w - hi).
-__device__ __forceinline__ void tc_dequant8(uint32_t word, float s, float b, uint32_t *hi, uint32_t *lo) {
-    const Codes8 c = decode8(word);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const float w0 = fmaf(s, c.f[2 * p], b), w1 = fmaf(s, c.f[2 * p + 1], b);
-        hi[p] = tc_pack_bf16(w0, w1);
-        lo[p] = tc_pack_bf16(w0 - __uint_as_float(hi[p] << 16), w1 - __uint_as_float(hi[p] & 0xFFFF0000u));
-    }
+// acc + lo(w) + hi(w) for a bf16 pair w, each add fp32 += bf16 (Blackwell's
+// mixed-precision add: the bf16 operand is widened exactly, one rounding per add).
+__device__ __forceinline__ float tc_add_bf16x2(float acc, uint32_t w) {
+    float r;
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n add.rn.f32.bf16 %0, l, %2;\n add.rn.f32.bf16 %0, h, %0;\n}"
+        : "=f"(r)
+        : "r"(w), "f"(acc));
+    return r;
 }
 
 // bf16 number j (0..7) of a 16-byte vector, compile-time j.
@@ -203,28 +280,26 @@ __device__ __forceinline__ float tc_pick_bf16(const uint4 &v) {
     return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 
-// Dequantise one stage (group g) of this thread's row into A stage `acol` of its lane.
-template <int j>
-__device__ __forceinline__ void tc_stage_dequant(const uint4 &q0, const uint4 &q1, const uint4 &s8, const uint4 &b8,
-                                                 uint32_t taddr) {
-    const float sf = tc_pick_bf16<j>(s8), bf = tc_pick_bf16<j>(b8);
-    uint32_t hi[32], lo[32];
-    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-    for (int c = 0; c < 8; ++c) tc_dequant8(words[c], sf, bf, hi + 4 * c, lo + 4 * c);
-    tc_st32(taddr, hi);
-    tc_st32(taddr + 32, lo);
-}
-
-__global__ void __launch_bounds__(kTcThreads, 2)
+template <int N>
+__global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     qmm_tc_kernel(QmmArgs a, const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap, TcPlan plan) {
+    constexpr int SW = tc_scale_warps(N);     // scale warps
+    constexpr int NT = N / (SW / 4);          // activation rows per scale thread (16 or 32)
+    constexpr int CH = 16;                    // columns per tcgen05.ld
+    constexpr int R = tc_ring(N), NA = tc_astages(N), ND = tc_dbufs(N);
+    constexpr int SLOT = tc_slot_bytes(N), XBYTES = N * kTcK * 2, RING = R * SLOT;
+    constexpr uint32_t TCOLS = tc_tmem_cols(N);
+    constexpr uint32_t ACOL = TCOLS - 32 * NA;        // first A-stage column
+    constexpr int DW = tc_dec_warps(N);               // decoder warps
+    constexpr int VW = 32 * 4 / DW;                   // bf16 pairs per decoder thread and group: 32 or 16
+    (void)sizeof(TcChecks<N>);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *ring = smem;                                            // [slot][x | codes], later partial sums
-    float *part = reinterpret_cast<float *>(smem);                   // [n_mma][128] fp32
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcRingBytes);
-    // bars: full[R], xfree[R], cfree[R], afull[A], aempty[A], acc_full; then the TMEM address and the flag
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * kTcRing + 2 * kTcAStages + 1);
+    uint8_t *ring = smem;                                               // [slot][x | codes]
+    float *part = reinterpret_cast<float *>(smem);                      // at the end: [N][128] fp32
+    float *xbar = reinterpret_cast<float *>(smem + RING);       // [slot][128] fp32
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + RING + kTcXbBytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + tc_num_bars(N));
     volatile int *fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -232,14 +307,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int rank = (int)tc_cluster_rank();
     const int tile = blockIdx.x / ks;
     const int p0 = rank * plan.periods / ks, p1 = (rank + 1) * plan.periods / ks;
-    const int i0 = 8 * p0, nst = 8 * (p1 - p0);          // this CTA's stages [i0, i0 + nst)
+    const int i0 = 8 * p0, nst = 8 * (p1 - p0);          // this CTA's groups [i0, i0 + nst)
     const uint32_t bar_s = tc_smem(bars);
+    // barrier addresses: full[R] xfree[R] cfree[R] afull[A] aempty[A] dfull[D] dfree[D] xbfull[X] xbfree[X]
     auto full = [=](int s) { return bar_s + 8u * s; };
-    auto xfree = [=](int s) { return bar_s + 8u * (kTcRing + s); };
-    auto cfree = [=](int s) { return bar_s + 8u * (2 * kTcRing + s); };
-    auto afull = [=](int s) { return bar_s + 8u * (3 * kTcRing + s); };
-    auto aempty = [=](int s) { return bar_s + 8u * (3 * kTcRing + kTcAStages + s); };
-    const uint32_t acc_full = bar_s + 8u * (3 * kTcRing + 2 * kTcAStages);
+    auto xfree = [=](int s) { return bar_s + 8u * (R + s); };
+    auto cfree = [=](int s) { return bar_s + 8u * (2 * R + s); };
+    auto afull = [=](int s) { return bar_s + 8u * (3 * R + s); };
+    auto aempty = [=](int s) { return bar_s + 8u * (3 * R + NA + s); };
+    auto dfull = [=](int s) { return bar_s + 8u * (3 * R + 2 * NA + s); };
+    auto dfree = [=](int s) { return bar_s + 8u * (3 * R + 2 * NA + ND + s); };
+    auto xbfull = [=](int s) { return bar_s + 8u * (3 * R + 2 * NA + 2 * ND + s); };
+    auto xbfree = [=](int s) { return bar_s + 8u * (3 * R + 2 * NA + 2 * ND + kTcXbSlots + s); };
 
     // The tile's rows: box A (tile rows 0-63) and box B (64-127) of the whole
     // matrix, how many of each box are valid, and the output column of tile row 0.
@@ -270,22 +349,29 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcRing; ++s) {
+        for (int s = 0; s < R; ++s) {
             tc_mbar_init(full(s), 1);
             tc_mbar_init(xfree(s), 1);
-            tc_mbar_init(cfree(s), 4);
+            tc_mbar_init(cfree(s), DW);
         }
-        for (int s = 0; s < kTcAStages; ++s) {
-            tc_mbar_init(afull(s), 4);
+        for (int s = 0; s < NA; ++s) {
+            tc_mbar_init(afull(s), DW);
             tc_mbar_init(aempty(s), 1);
         }
-        tc_mbar_init(acc_full, 1);
+        for (int s = 0; s < ND; ++s) {
+            tc_mbar_init(dfull(s), 1);
+            tc_mbar_init(dfree(s), SW);
+        }
+        for (int s = 0; s < kTcXbSlots; ++s) {
+            tc_mbar_init(xbfull(s), 4);
+            tc_mbar_init(xbfree(s), SW);
+        }
         *fail = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem(tmem_slot)),
-                     "r"(kTcTmemCols)
+                     "r"(TCOLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -293,66 +379,165 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_mma = plan.n_mma;
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA
         if (lane == 0) {
-            const uint32_t bytes = (uint32_t)n_mma * kTcK * 2 + kTcCBytes;
+            const uint32_t bytes = (uint32_t)SLOT;
             int issued = 0;
             for (int li = 0; li < nst; ++li) {
-                const int s = li % kTcRing;
-                if (li >= kTcRing) {
-                    const uint32_t par = ((li / kTcRing) - 1) & 1;
+                const int s = li % R;
+                if (li >= R) {
+                    const uint32_t par = ((li / R) - 1) & 1;
                     if (!tc_wait(xfree(s), par, fail) || !tc_wait(cfree(s), par, fail)) { *fail = 1; break; }
                 }
                 if (*fail) break;
                 const int i = i0 + li;
-                const uint32_t slot = tc_smem(ring + s * kTcSlot);
+                const uint32_t slot = tc_smem(ring + s * SLOT);
                 tc_expect_tx(full(s), bytes);
                 tc_tma_2d(slot, &xmap, i * kTcK, 0, full(s));
-                tc_tma_2d(slot + kTcXBytes, &cmap, i * (kTcK / 2), rowA, full(s));
-                tc_tma_2d(slot + kTcXBytes + kTcCBytes / 2, &cmap, i * (kTcK / 2), rowB, full(s));
+                tc_tma_2d(slot + XBYTES, &cmap, i * (kTcK / 2), rowA, full(s));
+                tc_tma_2d(slot + XBYTES + kTcCBytes / 2, &cmap, i * (kTcK / 2), rowB, full(s));
                 issued = li + 1;
             }
             // every copy issued must land before the ring is reused or the CTA exits
-            for (int li = issued - kTcRing; li < issued; ++li)
-                if (li >= 0) tc_wait(full(li % kTcRing), (li / kTcRing) & 1, fail, 1 << 16);
+            for (int li = issued - R; li < issued; ++li)
+                if (li >= 0) tc_wait(full(li % R), (li / R) & 1, fail, 1 << 16);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
-            const uint32_t idesc = tc_idesc(n_mma);
+            const uint32_t idesc = tc_idesc(N);
             for (int li = 0; li < nst; ++li) {
-                const int s = li % kTcRing, sa = li % kTcAStages;
-                if (!tc_wait(full(s), (li / kTcRing) & 1, fail) || !tc_wait(afull(sa), (li / kTcAStages) & 1, fail)) {
+                const int s = li % R, sa = li % NA, sd = li % ND;
+                if (!tc_wait(full(s), (li / R) & 1, fail) || !tc_wait(afull(sa), (li / NA) & 1, fail) ||
+                    (li >= ND && !tc_wait(dfree(sd), ((li / ND) - 1) & 1, fail))) {
                     *fail = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t xb = tc_smem(ring + s * kTcSlot);
-                const uint32_t ahi = tmem + 128u + 64u * sa, alo = ahi + 32u;
+                const uint32_t xb = tc_smem(ring + s * SLOT);
+                const uint32_t dt = tmem + (uint32_t)(N * sd), at = tmem + ACOL + 32u * sa;
 #pragma unroll
-                for (int kk = 0; kk < kTcK / 16; ++kk) {
-                    const uint64_t db = tc_desc(xb + kk * 32);
-                    tc_mma_ts(tmem, ahi + 8 * kk, db, idesc, (li > 0 || kk > 0) ? 1u : 0u);
-                    tc_mma_ts(tmem, alo + 8 * kk, db, idesc, 1u);
-                }
+                for (int kk = 0; kk < kTcK / 16; ++kk) tc_mma_ts(dt, at + 8 * kk, tc_desc(xb + kk * 32), idesc, kk > 0 ? 1u : 0u);
                 tc_commit(xfree(s));
                 tc_commit(aempty(sa));
+                tc_commit(dfull(sd));
             }
-            tc_commit(acc_full);
         }
+    } else if (warp < 2 + DW) {
+        // ------------------------------------------- codes -> A stages, and X_g
+        // Software-pipelined: group li is decoded into registers while the
+        // tensor-memory store of group li-1 drains; an A stage is published
+        // (afull) only after tcgen05.wait::st.  With 8 decoder warps each
+        // thread takes half of its row's 64 codes.
+        const int q = warp & 3, dh = (warp - 2) >> 2;   // lane quarter; part of the group's codes
+        const int t = 32 * q + lane;                    // tile row == TMEM lane; also an activation row
+        const uint32_t a_lane = tmem + ((uint32_t)(32 * q) << 16) + ACOL + (uint32_t)(dh * VW);
+        const bool xrole = dh == 0;                     // these four warps also form X_g
+        uint32_t va[VW], vb[VW];
+        bool ok = true;
+        int stored = 0;
+#define TC_PRODUCE(LI, V)                                                                                           \
+    {                                                                                                               \
+        const int s_ = (LI) % R, xs_ = (LI) % kTcXbSlots;                                                           \
+        ok = tc_wait(full(s_), ((LI) / R) & 1, fail);                                                               \
+        if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                         \
+            *fail = 1;                                                                                              \
+            break;                                                                                                  \
+        }                                                                                                           \
+        const uint8_t *slot_ = ring + s_ * SLOT;                                                                    \
+        const uint4 *cp_ = reinterpret_cast<const uint4 *>(slot_ + XBYTES + 32 * t);                                \
+        uint32_t w_[VW / 4];                                                                                        \
+        if (VW == 32) { /* lanes 4-7 of each eight read the second half first: no bank conflict */                 \
+            const int sw_ = (lane >> 2) & 1;                                                                        \
+            const uint4 ca_ = cp_[sw_], cb_ = cp_[sw_ ^ 1];                                                         \
+            const uint4 c0_ = sw_ ? cb_ : ca_, c1_ = sw_ ? ca_ : cb_;                                               \
+            w_[0] = c0_.x; w_[1] = c0_.y; w_[2] = c0_.z; w_[3] = c0_.w;                                             \
+            w_[VW / 4 - 4] = c1_.x; w_[VW / 4 - 3] = c1_.y; w_[VW / 4 - 2] = c1_.z; w_[VW / 4 - 1] = c1_.w;         \
+        } else {                                                                                                    \
+            const uint4 c0_ = cp_[dh];                                                                              \
+            w_[0] = c0_.x; w_[1] = c0_.y; w_[2] = c0_.z; w_[3] = c0_.w;                                             \
+        }                                                                                                           \
+        float xsum_ = 0.0f;                                                                                         \
+        if (xrole && t < N) { /* X_g of activation row t: 64 values, k ascending (8 chunks of 8) */                \
+            const uint8_t *xrow_ = slot_ + t * 128;                                                                 \
+            _Pragma("unroll") for (int c = 0; c < 8; ++c) {                                                         \
+                const uint4 v_ = *reinterpret_cast<const uint4 *>(xrow_ + ((c ^ (t & 7)) << 4));                    \
+                const float cs_ = tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(0.0f, v_.x), v_.y), v_.z), v_.w); \
+                xsum_ = c == 0 ? cs_ : xsum_ + cs_;                                                                 \
+            }                                                                                                       \
+        }                                                                                                           \
+        __syncwarp();                                                                                               \
+        if (lane == 0) tc_arrive(cfree(s_));                                                                        \
+        if (xrole) {                                                                                                \
+            ok = (LI) < kTcXbSlots || tc_wait(xbfree(xs_), (((LI) / kTcXbSlots) - 1) & 1, fail);                    \
+            if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                     \
+                *fail = 1;                                                                                          \
+                break;                                                                                              \
+            }                                                                                                       \
+            if (t < N) xbar[xs_ * kTcMaxN + t] = xsum_;                                                             \
+            __syncwarp();                                                                                           \
+            if (lane == 0) tc_arrive(xbfull(xs_));                                                                  \
+        }                                                                                                           \
+        _Pragma("unroll") for (int c = 0; c < VW / 4; ++c) {                                                        \
+            const uint32_t ws_ = w_[c] >> 4;                                                                        \
+            V[4 * c + 0] = tc_code_pair<0>(w_[c], ws_);                                                             \
+            V[4 * c + 1] = tc_code_pair<1>(w_[c], ws_);                                                             \
+            V[4 * c + 2] = tc_code_pair<2>(w_[c], ws_);                                                             \
+            V[4 * c + 3] = tc_code_pair<3>(w_[c], ws_);                                                             \
+        }                                                                                                           \
+    }
+#define TC_PUBLISH(LI)                                                                                              \
+    {                                                                                                               \
+        tc_wait_st();                                                                                               \
+        tc_fence_before();                                                                                          \
+        __syncwarp();                                                                                               \
+        if (lane == 0) tc_arrive(afull((LI) % NA));                                                                 \
+    }
+#define TC_STORE(LI, V)                                                                                             \
+    {                                                                                                               \
+        const int sa_ = (LI) % NA;                                                                                  \
+        ok = (LI) < NA || tc_wait(aempty(sa_), (((LI) / NA) - 1) & 1, fail);                                        \
+        if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                         \
+            *fail = 1;                                                                                              \
+            break;                                                                                                  \
+        }                                                                                                           \
+        tc_fence_after();                                                                                           \
+        tc_st<VW>(a_lane + 32u * sa_, V);                                                                           \
+        stored = (LI) + 1;                                                                                          \
+    }
+        for (int li = 0; li < nst; li += 2) {   // nst is a multiple of 8
+            TC_PRODUCE(li, va)
+            if (li > 0) TC_PUBLISH(li - 1)
+            TC_STORE(li, va)
+            TC_PRODUCE(li + 1, vb)
+            TC_PUBLISH(li)
+            TC_STORE(li + 1, vb)
+        }
+        if (stored == nst && nst > 0) {
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc_arrive(afull((nst - 1) % NA));
+        }
+#undef TC_PRODUCE
+#undef TC_PUBLISH
+#undef TC_STORE
     } else {
-        // ---------------------------------------------------------------- dequant
-        const int q = warp & 3;                        // TMEM lane quarter of this warp
+        // ------------------------------------------------ y += s D_g + b X_g
+        const int q = warp & 3, h = (warp - 2 - DW) >> 2;   // lane quarter, block of NT rows
         const int t = 32 * q + lane;                   // tile row == TMEM lane
         const int G = a.K / kGroup;
         const bool valid = t < 64 ? t < validA : (t - 64) < validB;
         const int row = t < 64 ? rowA + t : rowB + (t - 64);
         const uint16_t *srow = valid ? a.scales + (size_t)row * G : nullptr;
         const uint16_t *brow = valid ? a.biases + (size_t)row * G : nullptr;
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + 128u;
+        const uint32_t d_lane = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * NT);
+        const float *xb_h = xbar + h * NT;
+        float acc[NT];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
         uint4 s8 = make_uint4(0, 0, 0, 0), b8 = s8, sn = s8, bn = s8;
         if (srow) {
             s8 = __ldg(reinterpret_cast<const uint4 *>(srow + 8 * p0));
@@ -364,57 +549,56 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 sn = __ldg(reinterpret_cast<const uint4 *>(srow + 8 * (p + 1)));
                 bn = __ldg(reinterpret_cast<const uint4 *>(brow + 8 * (p + 1)));
             }
-#define TC_STAGE(J)                                                                                                  \
-    {                                                                                                                \
-        const int s = li % kTcRing, sa = li % kTcAStages;                                                            \
-        bool ok = tc_wait(full(s), (li / kTcRing) & 1, fail);                                                        \
-        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;                                                                  \
-        if (ok) {                                                                                                    \
-            const uint4 *src = reinterpret_cast<const uint4 *>(ring + s * kTcSlot + kTcXBytes + 32 * t);             \
-            q0 = src[0];                                                                                             \
-            q1 = src[1];                                                                                             \
-        }                                                                                                            \
-        __syncwarp();                                                                                                \
-        if (lane == 0) tc_arrive(cfree(s));                                                                          \
-        if (ok && li >= kTcAStages) ok = tc_wait(aempty(sa), ((li / kTcAStages) - 1) & 1, fail);                     \
-        if (!ok) *fail = 1;                                                                                          \
-        if (__any_sync(0xFFFFFFFFu, !ok)) break;                                                                     \
-        tc_fence_after();                                                                                            \
-        tc_stage_dequant<J>(q0, q1, s8, b8, lane_base + 64u * sa);                                                     \
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");                                                \
-        tc_fence_before();                                                                                           \
-        __syncwarp();                                                                                                \
-        if (lane == 0) tc_arrive(afull(sa));                                                                         \
-        ++li;                                                                                                        \
+#define TC_GROUP(J)                                                                                                 \
+    {                                                                                                               \
+        const int sd = li % ND, xs = li % kTcXbSlots;                                                         \
+        const bool ok = tc_wait(dfull(sd), (li / ND) & 1, fail) && tc_wait(xbfull(xs), (li / kTcXbSlots) & 1, fail); \
+        if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                         \
+            *fail = 1;                                                                                              \
+            break;                                                                                                  \
+        }                                                                                                           \
+        tc_fence_after();                                                                                           \
+        /* D holds sum (128 + q) x: y += s D + (b - 128 s) X; b - 128 s is exact in fp32 */                      \
+        const float sf = tc_pick_bf16<J>(s8), bf = fmaf(-128.0f, sf, tc_pick_bf16<J>(b8));                          \
+        const float *xg = xb_h + xs * kTcMaxN;                                                                      \
+        _Pragma("unroll") for (int c = 0; c < NT; c += CH) {                                                        \
+            uint32_t d[CH];                                                                                         \
+            tc_ld<CH>(d_lane + (uint32_t)(N * sd) + c, d);                                                                   \
+            tc_wait_ld();                                                                                           \
+            _Pragma("unroll") for (int j = 0; j < CH; j += 4) {                                                     \
+                const float4 xv = *reinterpret_cast<const float4 *>(xg + c + j);                                    \
+                acc[c + j + 0] = fmaf(bf, xv.x, fmaf(sf, __uint_as_float(d[j + 0]), acc[c + j + 0]));               \
+                acc[c + j + 1] = fmaf(bf, xv.y, fmaf(sf, __uint_as_float(d[j + 1]), acc[c + j + 1]));               \
+                acc[c + j + 2] = fmaf(bf, xv.z, fmaf(sf, __uint_as_float(d[j + 2]), acc[c + j + 2]));               \
+                acc[c + j + 3] = fmaf(bf, xv.w, fmaf(sf, __uint_as_float(d[j + 3]), acc[c + j + 3]));               \
+            }                                                                                                       \
+        }                                                                                                           \
+        tc_fence_before();                                                                                          \
+        __syncwarp();                                                                                               \
+        if (lane == 0) {                                                                                            \
+            tc_arrive(dfree(sd));                                                                                   \
+            tc_arrive(xbfree(xs));                                                                                  \
+        }                                                                                                           \
+        ++li;                                                                                                       \
     }
             do {
-                TC_STAGE(0) TC_STAGE(1) TC_STAGE(2) TC_STAGE(3) TC_STAGE(4) TC_STAGE(5) TC_STAGE(6) TC_STAGE(7)
+                TC_GROUP(0) TC_GROUP(1) TC_GROUP(2) TC_GROUP(3) TC_GROUP(4) TC_GROUP(5) TC_GROUP(6) TC_GROUP(7)
             } while (0);
-#undef TC_STAGE
+#undef TC_GROUP
             s8 = sn;
             b8 = bn;
         }
-        // ---- accumulator -> shared memory, as part[m][t]
-        bool ok = !*fail && tc_wait(acc_full, 0, fail);
-        if (!ok) *fail = 1;
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        tc_fence_after();
-        if (ok) {
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16);
-            for (int c0 = 0; c0 < n_mma; c0 += 16) {
-                uint32_t r[16];
-                tc_ld16(taddr + c0, r);
+        // this CTA's partial sums -> shared memory, as part[m][t]
 #pragma unroll
-                for (int j = 0; j < 16; ++j) part[(c0 + j) * kTcRows + t] = __uint_as_float(r[j]);
-            }
-        }
+        for (int j = 0; j < NT; ++j) part[(h * NT + j) * kTcRows + t] = acc[j];
     }
     __syncwarp();
     tc_fence_before();
     tc_cluster_sync();   // every partial sum and failure flag of the cluster is in place
 
-    if (warp >= 2) {
-        const int t = 32 * (warp & 3) + lane;
+    if (warp >= 2 + DW) {
+        const int tid = threadIdx.x - 32 * (2 + DW);   // 0 .. 32 SW - 1
+        constexpr int RT = 32 * SW;                              // reducing threads
         int bad = 0;
         for (int j = 0; j < ks; ++j) bad |= tc_ld_cluster_s32(tc_mapa(tc_smem((const void *)fail), j));
         const int mper = (a.M + ks - 1) / ks;
@@ -427,9 +611,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             return acc;
         };
         if (a.glu) {
-            const int pr = t & 63;
+            const int pr = tid & 63;
             if (pr < validA) {
-                for (int m = m0 + (t >> 6); m < m1; m += 2) {
+                for (int m = m0 + (tid >> 6); m < m1; m += RT / 64) {
                     uint16_t out = (uint16_t)TF_NAN_BF16;
                     if (!bad) {
                         const float g = bf16_bits_to_f32(f32_to_bf16_rne(total(m, pr)));
@@ -439,16 +623,19 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     a.y[(size_t)m * a.ldy + col_base + pr] = out;
                 }
             }
-        } else if (t < validA + validB) {
-            for (int m = m0; m < m1; ++m)
-                a.y[(size_t)m * a.ldy + col_base + t] = bad ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(total(m, t));
+        } else {
+            const int t = tid & 127;
+            if (t < validA + validB) {
+                for (int m = m0 + (tid >> 7); m < m1; m += RT / 128)
+                    a.y[(size_t)m * a.ldy + col_base + t] = bad ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(total(m, t));
+            }
         }
     }
     __syncwarp();
     tc_cluster_sync();   // no CTA leaves while another still reads its shared memory
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TCOLS) : "memory");
     }
 }
 
@@ -467,7 +654,7 @@ static cudaError_t get_encode() {
 
 // K slices per tile: from K and the whole matrix's row count alone.  The whole
 // matrix should give about 512 CTAs; a slice keeps at least four periods of
-// eight stages unless the periods divide evenly.
+// eight groups unless the periods divide evenly.
 int qmm_tc_split(int K, int n_whole) {
     const int periods = K / 512;
     const int tiles = (n_whole + kTcRows - 1) / kTcRows;
@@ -488,7 +675,32 @@ bool qmm_tc_eligible(const QmmArgs &a) {
            aligned(a.biases, 16);
 }
 
-static bool g_tc_smem_set[64];
+template <int N>
+static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const CUtensorMap &cmap, const TcPlan &plan,
+                               cudaStream_t stream) {
+    static bool smem_set[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!smem_set[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(qmm_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes(N));
+        if (e != cudaSuccess) return e;
+        smem_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)(plan.ntiles * plan.ks));
+    cfg.blockDim = dim3(tc_threads(N));
+    cfg.dynamicSmemBytes = tc_smem_bytes(N);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)plan.ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, qmm_tc_kernel<N>, a, xmap, cmap, plan);
+}
 
 cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
     cudaError_t e = get_encode();
@@ -497,7 +709,7 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
     std::memset(&plan, 0, sizeof plan);
     plan.ks = qmm_tc_split(a.K, a.n_whole);
     plan.periods = a.K / 512;
-    plan.n_mma = ((a.M + 15) / 16) * 16;
+    const int n_mma = a.M <= 16 ? 16 : a.M <= 32 ? 32 : a.M <= 64 ? 64 : 128;
     if (a.glu) {
         plan.ntiles = (a.seg.ncols + 63) / 64;
     } else {
@@ -515,7 +727,7 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
     {
         const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
         const cuuint64_t strides[1] = {(cuuint64_t)a.ldx * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)plan.n_mma};
+        const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)n_mma};
         const cuuint32_t estr[2] = {1, 1};
         if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.x), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -532,27 +744,12 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (!g_tc_smem_set[dev]) {
-        e = cudaFuncSetAttribute(qmm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
-        if (e != cudaSuccess) return e;
-        g_tc_smem_set[dev] = true;
+    switch (n_mma) {
+        case 16: return launch_tc_n<16>(a, xmap, cmap, plan, stream);
+        case 32: return launch_tc_n<32>(a, xmap, cmap, plan, stream);
+        case 64: return launch_tc_n<64>(a, xmap, cmap, plan, stream);
+        default: return launch_tc_n<128>(a, xmap, cmap, plan, stream);
     }
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3((unsigned)(plan.ntiles * plan.ks));
-    cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = kTcSmem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)plan.ks;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, qmm_tc_kernel, a, xmap, cmap, plan);
 }
 
 }  // namespace tf

@@ -10,6 +10,21 @@
 #include "tf_kernels.h"
 
 
+namespace tf {
+
+// The CUDA error behind the last TF_E_CUDA returned on this host thread.
+static thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+tf_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return TF_OK;
+    g_last_cuda = e;
+    return TF_E_CUDA;
+}
+
+cudaError_t last_cuda_error() { return g_last_cuda; }
+
+}  // namespace tf
+
 using namespace tf;
 
 extern "C" {
@@ -60,6 +75,8 @@ size_t tf_seam_bytes(int rows, int width) {
     return (size_t)rows * (size_t)width * 2u;
 }
 
+const char *tf_last_cuda_error(void) { return cudaGetErrorString(last_cuda_error()); }
+
 tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
                       const void *biases, int N_whole, const tf_seg *segs, int nseg, tf_epi epi, void *y,
                       int ldy, tf_stream stream) {
@@ -108,7 +125,7 @@ tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, c
     a.y = static_cast<uint16_t *>(y);
     a.ldy = ldy;
     a.n_whole = N_whole;
-    return launch_qmm(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_E_CUDA;
+    return cuda_status(launch_qmm(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tf_status tf_gather_rows(void *dst, int ld_dst, const void *const *parts, const int *widths, int nparts, int M,
@@ -141,7 +158,7 @@ tf_status tf_gather_rows(void *dst, int ld_dst, const void *const *parts, const 
     g.ld_dst = ld_dst;
     g.nparts = nparts;
     g.M = M;
-    if (launch_gather(g, vec, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TF_E_CUDA;
+    if (cuda_status(launch_gather(g, vec, reinterpret_cast<cudaStream_t>(stream))) != TF_OK) return TF_E_CUDA;
     return broken ? TF_E_BROKEN : TF_OK;
 }
 
@@ -168,7 +185,7 @@ tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_b
     a.partial = static_cast<uint64_t *>(scratch);
     a.words = words;
     a.vec = aligned(logits, 16) && (ld % 8 == 0);
-    return launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_E_CUDA;
+    return cuda_status(launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_stream stream) {
@@ -176,8 +193,7 @@ tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_st
     if (M == 0) return TF_OK;
     if (!words || !ids) return TF_E_ARG;
     if (!aligned(words, 8) || !aligned(ids, 4)) return TF_E_ALIGN;
-    return launch_pick(words, nparts, M, ids, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK
-                                                                                                     : TF_E_CUDA;
+    return cuda_status(launch_pick(words, nparts, M, ids, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -64,6 +64,9 @@ bool qmm_tc_eligible(const QmmArgs &a);
 cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream);
 cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream);
 int argmax_blocks_per_row(int M, int n);
+// TF_OK for cudaSuccess; otherwise remembers e for tf_last_cuda_error and returns TF_E_CUDA.
+tf_status cuda_status(cudaError_t e);
+cudaError_t last_cuda_error();
 int num_sms();
 
 }  // namespace tf

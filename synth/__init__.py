@@ -31,6 +31,7 @@ TAG_W = 1
 TAG_X = 2
 TAG_W2 = 3
 TAG_HEAD = 4
+TAG_ATTN = 6
 
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
