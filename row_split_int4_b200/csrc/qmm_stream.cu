@@ -213,16 +213,21 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
         fence_mbar_init();
     }
     __syncwarp();
-    for (int t = 0; t < kStages && t < steps; ++t) issue_next();
+    // Wide units send only their first slot's copies before the limb preparation:
+    // with every warp queueing its whole ring at once the copy queue fills and the
+    // issuing lanes wait, which would hold the preparation back; the rest follow
+    // it.  Narrow units, whose warps have few steps, queue their whole ring now.
+    constexpr int kPreStages = kRU >= 4 ? 1 : kStages;
+    for (int t = 0; t < kPreStages && t < steps; ++t) issue_next();
 
     // fixed-point limbs of x, one warp per lane-chunk, one lane per value, on the
     // bf16 fields alone: x = sign * M * 2^(e-134), M = 128 + mantissa (e >= 1) or
     // the mantissa (e = 0, subnormal, read with e = 1).  With emax the chunk's
     // largest e, F = x * 2^(23-E), E = emax - 126, is sign * M * 2^(e - emax + 15):
     // a left shift when e >= emax - 15 (exact), else a right shift rounded to nearest even.
-    // (loads are issued eight lane-chunks at a time so that one L2 round trip
-    // covers all eight)
-    constexpr int kPrepBatch = 8;
+    // (loads are issued sixteen lane-chunks at a time so that one L2 round trip
+    // covers all of them)
+    constexpr int kPrepBatch = 16;
     for (int lc0 = warp; lc0 < nch * 32; lc0 += W * kPrepBatch) {
       uint32_t hb[kPrepBatch];
 #pragma unroll
@@ -270,6 +275,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
       }
     }
     __syncthreads();
+    for (int t = kPreStages; t < kStages && t < steps; ++t) issue_next();
 
     float acc[kRU];
 #pragma unroll
