@@ -175,6 +175,36 @@ tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_b
                          uint64_t *words, void *scratch, size_t scratch_bytes, tf_stream stream);
 
 /*
+ * tf_qmm_argmax_rows -- the head of one rank in one call: the logits of one row
+ * slice (tf_qmm_rows, TF_EPI_NONE, one segment) and their argmax word
+ * (tf_argmax_rows over those logits with ids id_base + j).  The step-1 body of
+ * TensorFold PR #1433 has each rank compute its half of the lm_head and then
+ * pair_argmax over it; here, at M = 1, the qmm's warps keep the best key of the
+ * rows they write and the kernel's last CTA to finish combines them (a 4-byte
+ * asynchronous memset clears its counter first), so the argmax needs neither a
+ * pass over the logits nor a second kernel.  The results are bit for bit those of the two separate
+ * calls: the logits equal tf_qmm_rows' and the word equals tf_argmax_rows' on
+ * them.  For M > 1, or a weight layout the M = 1 streaming kernel does not take,
+ * the same two kernels run one after the other.
+ *
+ *   x, M, K, ldx, wq, scales, biases, N_whole   as tf_qmm_rows.
+ *   seg     the slice: whole-matrix rows [row0, row0 + nrows), nrows >= 1.
+ *   id_base global id of logit column 0 (usually seg.row0); id_base + nrows
+ *           <= 2^31 (TF_E_RANGE).
+ *   logits  bf16 [M][ld_logits], ld_logits >= nrows: written, as tf_qmm_rows' y.
+ *   words   uint64 [M], the argmax words (format of tf_argmax_rows).
+ *   scratch device buffer of at least tf_qmm_argmax_scratch_bytes(M, nrows)
+ *           bytes, 8-byte aligned, owned by the caller; contents on entry do not
+ *           matter and on return are unspecified.  Calls in flight at the same
+ *           time need separate scratch buffers.
+ * Errors: TF_E_ARG, TF_E_RANGE, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+size_t tf_qmm_argmax_scratch_bytes(int M, int nrows);
+tf_status tf_qmm_argmax_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
+                             const void *biases, int N_whole, tf_seg seg, uint32_t id_base, void *logits,
+                             int ld_logits, uint64_t *words, void *scratch, size_t scratch_bytes, tf_stream stream);
+
+/*
  * tf_pick -- the better of the per-slice winners (TensorFold PR #1433 step-1
  * body: pair_pick; the sixth control's test ((am | ap) & PAIR_FLAG) != 0u).
  *

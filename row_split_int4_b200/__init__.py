@@ -39,7 +39,7 @@ TF_EPI_NONE, TF_EPI_GLU = 0, 1
 
 EXPORTS = ["tf_qmm_rows", "tf_gather_rows", "tf_argmax_scratch_bytes", "tf_argmax_rows", "tf_pick",
            "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str", "tf_last_cuda_error",
-           "tf_abi_version", "tf_argmax_rows_static"]
+           "tf_abi_version", "tf_argmax_rows_static", "tf_qmm_argmax_rows", "tf_qmm_argmax_scratch_bytes"]
 
 
 class tf_seg(ctypes.Structure):
@@ -55,6 +55,11 @@ lib.tf_argmax_scratch_bytes.restype = _sz
 lib.tf_argmax_scratch_bytes.argtypes = [_i, _i]
 lib.tf_argmax_rows.restype = _i
 lib.tf_argmax_rows.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _sz, _vp]
+lib.tf_qmm_argmax_scratch_bytes.restype = _sz
+lib.tf_qmm_argmax_scratch_bytes.argtypes = [_i, _i]
+lib.tf_qmm_argmax_rows.restype = _i
+lib.tf_qmm_argmax_rows.argtypes = [_vp, _i, _i, _i, _vp, _vp, _vp, _i, tf_seg, ctypes.c_uint32, _vp, _i, _vp, _vp, _sz,
+                                   _vp]
 lib.tf_argmax_rows_static.restype = _i
 lib.tf_argmax_rows_static.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp]
 lib.tf_pick.restype = _i
@@ -155,6 +160,24 @@ def tf_qmm_rows(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases:
     st = lib.tf_qmm_rows(_ptr(x), x.shape[0], x.shape[1], _ld(x), _ptr(wq), _ptr(scales), _ptr(biases),
                          wq.shape[0], arr, len(segs), int(epi), _ptr(y), _ld(y), _stream(stream))
     return _ret(st, "tf_qmm_rows", check)
+
+
+def tf_qmm_argmax_scratch_bytes(M: int, nrows: int) -> int:
+    return lib.tf_qmm_argmax_scratch_bytes(int(M), int(nrows))
+
+
+def tf_qmm_argmax_rows(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases: torch.Tensor,
+                       seg: Tuple[int, int], id_base: int, logits: torch.Tensor, words: torch.Tensor,
+                       scratch: torch.Tensor, stream=None, check: bool = True) -> int:
+    """logits[M, nrows] = the qmm rows of ``seg`` = (row0, nrows) and words[M] their
+    argmax words (ids id_base + j), in one call; see tf.h."""
+    assert x.dtype == torch.bfloat16 and logits.dtype == torch.bfloat16
+    assert wq.dtype == torch.uint8 and scales.dtype == torch.bfloat16 and biases.dtype == torch.bfloat16
+    assert words.dtype == torch.int64 and scratch.dtype == torch.uint8
+    st = lib.tf_qmm_argmax_rows(_ptr(x), x.shape[0], x.shape[1], _ld(x), _ptr(wq), _ptr(scales), _ptr(biases),
+                                wq.shape[0], tf_seg(int(seg[0]), int(seg[1])), int(id_base), _ptr(logits),
+                                _ld(logits), _ptr(words), _ptr(scratch), scratch.numel(), _stream(stream))
+    return _ret(st, "tf_qmm_argmax_rows", check)
 
 
 def tf_gather_rows(dst: torch.Tensor, parts: Sequence[Optional[torch.Tensor]], widths: Sequence[int],

@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     float acc[kRU];
 #pragma unroll
     for (int r = 0; r < kRU; ++r) acc[r] = 0.0f;
+    uint64_t best = 0;   // fused head: the largest argmax key of the rows this warp wrote
     int u = u0, j = 0, slot = 0;
     uint32_t par = 0;
     const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
@@ -331,7 +332,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
 #pragma unroll
                     for (int r = 0; r < kRU; ++r) {
                         const int col = u * kRU + r;
-                        if (col < a.seg.ncols) a.y[col] = failed ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(tot[r]);
+                        if (col < a.seg.ncols) {
+                            const uint16_t h = failed ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(tot[r]);
+                            a.y[col] = h;
+                            if (a.cand) best = umax64(best, cand_key(h, a.id_base + (uint32_t)col));
+                        }
                     }
                 }
             }
@@ -350,12 +355,41 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     if (failed) {
         for (int s2 = 0; s2 < kStages; ++s2) wait_slot(bar0 + 8 * s2, 0, 1024);
     }
+    if (a.cand) {
+        // fused head: publish this warp's best key; the last CTA to finish reduces all
+        // of them into the argmax word (fence, then a ticket: the usual last-block pattern)
+        if (lane == 0) a.cand[gw] = best;
+        __threadfence();
+        __syncthreads();
+        __shared__ unsigned int ticket;
+        if (tid == 0) ticket = atomicAdd(a.done, 1u);
+        __syncthreads();
+        if (ticket == gridDim.x - 1) {
+            __threadfence();
+            const int ncand = (int)(gridDim.x * W);
+            uint64_t v = 0;
+            for (int i = tid; i < ncand; i += blockDim.x) v = umax64(v, ((volatile uint64_t *)a.cand)[i]);
+            v = warp_max64(v);
+            __shared__ uint64_t red[32];
+            if (lane == 0) red[warp] = v;
+            __syncthreads();
+            if (warp == 0) {
+                v = lane < W ? red[lane] : 0ull;
+                v = warp_max64(v);
+                if (lane == 0) {
+                    *a.word = word_of_key(v, a.y, a.id_base);
+                    *a.done = 0u;
+                }
+            }
+        }
+    }
 }
 
-// The widest warp count whose shared memory fits 227 KB.
+// The widest warp count whose shared memory fits 227 KB with 1 KB left for the
+// kernel's static shared memory.
 static int stream_warps(int K, int ru) {
     for (int w = kMaxWarps; w >= 4; --w)
-        if (stream_layout(K, w, ru).total <= 227 * 1024) return w;
+        if (stream_layout(K, w, ru).total <= 226 * 1024) return w;
     return 0;
 }
 
@@ -376,9 +410,9 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     if (g_stream_smem_set[dev][ri] < L.total) {
-        cudaError_t e = cudaFuncSetAttribute(qmm_m1_stream_kernel<RU>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(qmm_m1_stream_kernel<RU>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
         if (e != cudaSuccess) return e;
-        g_stream_smem_set[dev][ri] = 227 * 1024;
+        g_stream_smem_set[dev][ri] = 226 * 1024;
     }
     const int units = a.glu ? (a.seg.ncols + RU / 2 - 1) / (RU / 2) : (a.seg.ncols + RU - 1) / RU;
     int blocks = num_sms();
@@ -398,5 +432,7 @@ cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream) {
     if (rows >= 2 * warps || a.glu) return launch_ru<2>(a, 1, stream);
     return launch_ru<1>(a, 2, stream);
 }
+
+int qmm_m1_stream_max_cand() { return num_sms() * kMaxWarps; }
 
 }  // namespace tf

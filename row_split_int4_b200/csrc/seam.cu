@@ -60,29 +60,6 @@ cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- argmax --
-// A candidate is one 64-bit key whose unsigned order is the selection order:
-//   bit 63      non-finite flag (flagged beats every finite value)
-//   bits 62..31 16-bit order-preserving image of the bf16 value (finite only;
-//               -0 is mapped to +0 so that the two tie)
-//   bits 30..0  0x7FFFFFFF - id (the lower id wins among equals)
-// max() over keys is associative and commutative, so the block and grid
-// reduction trees cannot change the result.  0 is below every real key.
-__device__ __forceinline__ uint64_t cand_key(uint32_t h, uint32_t id) {
-    const uint64_t idpart = (uint64_t)(0x7FFFFFFFu - id);
-    if ((h & 0x7F80u) == 0x7F80u) return (1ull << 63) | idpart;   // NaN or +-Inf
-    if (h == 0x8000u) h = 0u;
-    const uint32_t mono = (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u);
-    return ((uint64_t)mono << 31) | idpart;
-}
-
-__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
-
-__device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = umax64(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    return v;
-}
-
 constexpr int kArgmaxThreads = 256;
 
 __global__ void __launch_bounds__(kArgmaxThreads) argmax_partial_kernel(ArgmaxArgs a) {
@@ -118,8 +95,7 @@ __global__ void __launch_bounds__(kArgmaxThreads) argmax_partial_kernel(ArgmaxAr
     }
 }
 
-// One warp per row: max over the row's partial keys, then the word.  The
-// winning value is read back from the logits so that a winning -0 keeps its sign.
+// One warp per row: max over the row's partial keys, then the word.
 __global__ void argmax_final_kernel(ArgmaxArgs a) {
     const int m = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (m >= a.M) return;
@@ -127,21 +103,7 @@ __global__ void argmax_final_kernel(ArgmaxArgs a) {
     uint64_t best = 0;
     for (int b = lane; b < a.blocks_per_row; b += 32) best = umax64(best, a.partial[(long long)m * a.blocks_per_row + b]);
     best = warp_max64(best);
-    if (lane == 0) {
-        const uint32_t id = 0x7FFFFFFFu - (uint32_t)(best & 0x7FFFFFFFull);
-        uint64_t word;
-        if (best == 0) {
-            // unreachable for n >= 1 (every element yields a nonzero key); kept so that
-            // no input can make the read below leave the row
-            word = ((uint64_t)(TF_PAIR_FLAG | a.id_base) << 32) | 0x7FC00000ull;
-        } else if (best >> 63) {
-            word = ((uint64_t)(TF_PAIR_FLAG | id) << 32) | 0x7FC00000ull;
-        } else {
-            const uint32_t h = a.logits[(long long)m * a.ld + (id - a.id_base)];
-            word = ((uint64_t)id << 32) | ((uint64_t)h << 16);
-        }
-        a.words[m] = word;
-    }
+    if (lane == 0) a.words[m] = word_of_key(best, a.logits + (long long)m * a.ld, a.id_base);
 }
 
 // Blocks per row: enough CTAs to cover the GPU a few times over for small M,

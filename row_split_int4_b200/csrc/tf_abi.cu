@@ -77,9 +77,12 @@ size_t tf_seam_bytes(int rows, int width) {
 
 const char *tf_last_cuda_error(void) { return cudaGetErrorString(last_cuda_error()); }
 
-tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
-                      const void *biases, int N_whole, const tf_seg *segs, int nseg, tf_epi epi, void *y,
-                      int ldy, tf_stream stream) {
+// Validation and argument block shared by tf_qmm_rows and tf_qmm_argmax_rows.
+// TF_OK with *empty set means there is nothing to compute.
+static tf_status qmm_args(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
+                          const void *biases, int N_whole, const tf_seg *segs, int nseg, tf_epi epi, void *y, int ldy,
+                          QmmArgs *out, bool *empty) {
+    *empty = false;
     if (M < 0 || M > TF_BATCH_ROWS) return TF_E_ARG;
     if (K < TF_GROUP || K > TF_MAX_K || K % TF_GROUP != 0) return TF_E_ARG;
     if (N_whole < 1) return TF_E_ARG;
@@ -106,13 +109,17 @@ tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, c
     t.ncols = (epi == TF_EPI_GLU) ? segs[0].nrows : (int)cols;
     if (cols > INT_MAX) return TF_E_RANGE;
     if (ldx < K || ldy < t.ncols) return TF_E_ARG;
-    if (M == 0 || t.ncols == 0) return TF_OK;
+    if (M == 0 || t.ncols == 0) {
+        *empty = true;
+        return TF_OK;
+    }
     if (!x || !wq || !scales || !biases || !y) return TF_E_ARG;
     if (!aligned(x, 16) || ldx % 8 != 0 || !aligned(wq, 16) || !aligned(scales, 2) || !aligned(biases, 2) ||
         !aligned(y, 2))
         return TF_E_ALIGN;
 
-    QmmArgs a;
+    QmmArgs &a = *out;
+    std::memset(&a, 0, sizeof a);
     a.x = static_cast<const uint16_t *>(x);
     a.M = M;
     a.K = K;
@@ -125,7 +132,70 @@ tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, c
     a.y = static_cast<uint16_t *>(y);
     a.ldy = ldy;
     a.n_whole = N_whole;
+    a.cand = nullptr;
+    a.id_base = 0;
+    a.done = nullptr;
+    a.word = nullptr;
+    return TF_OK;
+}
+
+tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
+                      const void *biases, int N_whole, const tf_seg *segs, int nseg, tf_epi epi, void *y,
+                      int ldy, tf_stream stream) {
+    QmmArgs a;
+    bool empty = false;
+    const tf_status st = qmm_args(x, M, K, ldx, wq, scales, biases, N_whole, segs, nseg, epi, y, ldy, &a, &empty);
+    if (st != TF_OK || empty) return st;
     return cuda_status(launch_qmm(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t tf_qmm_argmax_scratch_bytes(int M, int nrows) {
+    if (M <= 0 || nrows <= 0) return 0;
+    // fused: one key per warp of the grid, then the finish counter
+    const size_t fused = (size_t)qmm_m1_stream_max_cand() * sizeof(uint64_t) + 16;
+    const size_t plain = tf_argmax_scratch_bytes(M, nrows);
+    return fused > plain ? fused : plain;
+}
+
+tf_status tf_qmm_argmax_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, const void *scales,
+                             const void *biases, int N_whole, tf_seg seg, uint32_t id_base, void *logits,
+                             int ld_logits, uint64_t *words, void *scratch, size_t scratch_bytes, tf_stream stream) {
+    if (seg.nrows < 1) return TF_E_ARG;
+    if ((unsigned long long)id_base + (unsigned long long)seg.nrows > 0x80000000ull) return TF_E_RANGE;
+    QmmArgs a;
+    bool empty = false;
+    const tf_status st =
+        qmm_args(x, M, K, ldx, wq, scales, biases, N_whole, &seg, 1, TF_EPI_NONE, logits, ld_logits, &a, &empty);
+    if (st != TF_OK || empty) return st;
+    if (!words || !scratch) return TF_E_ARG;
+    if (!aligned(words, 8) || !aligned(scratch, 8)) return TF_E_ALIGN;
+    if (scratch_bytes < tf_qmm_argmax_scratch_bytes(M, seg.nrows)) return TF_E_ARG;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (M == 1 && qmm_m1_stream_eligible(a)) {
+        // fused: the qmm warps leave their best keys in scratch and the kernel's last
+        // CTA turns them into the word; the finish counter starts at zero
+        a.cand = static_cast<uint64_t *>(scratch);
+        a.id_base = id_base;
+        a.done = reinterpret_cast<unsigned int *>(a.cand + qmm_m1_stream_max_cand());
+        a.word = words;
+        const tf_status z = cuda_status(cudaMemsetAsync(a.done, 0, sizeof(unsigned int), s));
+        if (z != TF_OK) return z;
+        return cuda_status(launch_qmm_m1_stream(a, s));
+    }
+    // otherwise the two steps: the rows, then the argmax over them
+    const tf_status q = cuda_status(launch_qmm(a, s));
+    if (q != TF_OK) return q;
+    ArgmaxArgs g;
+    std::memset(&g, 0, sizeof g);
+    g.logits = a.y;
+    g.ld = ld_logits;
+    g.n = seg.nrows;
+    g.id_base = id_base;
+    g.M = M;
+    g.partial = static_cast<uint64_t *>(scratch);
+    g.words = words;
+    g.vec = aligned(logits, 16) && (ld_logits % 8 == 0);
+    return cuda_status(launch_argmax(g, s));
 }
 
 tf_status tf_gather_rows(void *dst, int ld_dst, const void *const *parts, const int *widths, int nparts, int M,

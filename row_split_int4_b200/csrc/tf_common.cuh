@@ -38,6 +38,44 @@ __device__ __forceinline__ float glu_f32(float g, float u) {
     return g * s;
 }
 
+// A candidate is one 64-bit key whose unsigned order is the selection order:
+//   bit 63      non-finite flag (flagged beats every finite value)
+//   bits 62..31 16-bit order-preserving image of the bf16 value (finite only;
+//               -0 is mapped to +0 so that the two tie)
+//   bits 30..0  0x7FFFFFFF - id (the lower id wins among equals)
+// max() over keys is associative and commutative, so the block and grid
+// reduction trees cannot change the result.  0 is below every real key.
+__device__ __forceinline__ uint64_t cand_key(uint32_t h, uint32_t id) {
+    const uint64_t idpart = (uint64_t)(0x7FFFFFFFu - id);
+    if ((h & 0x7F80u) == 0x7F80u) return (1ull << 63) | idpart;   // NaN or +-Inf
+    if (h == 0x8000u) h = 0u;
+    const uint32_t mono = (h & 0x8000u) ? (~h & 0xFFFFu) : (h | 0x8000u);
+    return ((uint64_t)mono << 31) | idpart;
+}
+
+__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = umax64(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// The word of a row from its best key: the id, and the winning value read back
+// from the logits so that a winning -0 keeps its sign; a flagged key gives the
+// flag and the first non-finite id.
+__device__ __forceinline__ uint64_t word_of_key(uint64_t best, const uint16_t *row, uint32_t id_base) {
+    const uint32_t id = 0x7FFFFFFFu - (uint32_t)(best & 0x7FFFFFFFull);
+    if (best == 0) {
+        // unreachable for n >= 1 (every element yields a nonzero key); kept so that
+        // no input can make the read below leave the row
+        return ((uint64_t)(TF_PAIR_FLAG | id_base) << 32) | 0x7FC00000ull;
+    }
+    if (best >> 63) return ((uint64_t)(TF_PAIR_FLAG | id) << 32) | 0x7FC00000ull;
+    const uint32_t h = row[id - id_base];
+    return ((uint64_t)id << 32) | ((uint64_t)h << 16);
+}
+
 __host__ __forceinline__ bool aligned(const void *p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }

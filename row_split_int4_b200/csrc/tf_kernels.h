@@ -30,6 +30,14 @@ struct QmmArgs {
     uint16_t *y;
     int ldy;
     int n_whole;   // rows of the whole matrix (the call may cover only some of them)
+    // fused head (M = 1 stream kernel only): when cand is set, every warp of the grid
+    // writes the largest argmax key of the rows it wrote (ids id_base + column) to
+    // cand[warp of the grid] (0 when it wrote none); the last CTA to finish, counted
+    // on *done (zero at launch, zero again at exit), reduces them into *word
+    uint64_t *cand;
+    uint32_t id_base;
+    unsigned int *done;
+    uint64_t *word;
 };
 
 struct GatherArgs {
@@ -63,6 +71,8 @@ bool qmm_m1_stream_eligible(const QmmArgs &a);
 bool qmm_tc_eligible(const QmmArgs &a);
 cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream);
 cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream);
+int qmm_m1_stream_max_cand();   // an upper bound of the warps of any stream launch
+
 int argmax_blocks_per_row(int M, int n);
 // TF_OK for cudaSuccess; otherwise remembers e for tf_last_cuda_error and returns TF_E_CUDA.
 tf_status cuda_status(cudaError_t e);

@@ -154,6 +154,34 @@ def test_argmax_refusals(tf):
     assert tf.tf_argmax_scratch_bytes(0, 10) == 0 and tf.tf_argmax_scratch_bytes(3, 0) == 0
 
 
+def test_fused_head_refusals(tf):
+    L = tf.lib
+    seg = tf.tf_seg(0, 2048)
+
+    def call(M=1, K=512, seg=seg, id_base=0, logits=A, ld=2048, words=A, scratch=A, nbytes=None):
+        nb = tf.tf_qmm_argmax_scratch_bytes(max(M, 1), max(seg.nrows, 1)) if nbytes is None else nbytes
+        return L.tf_qmm_argmax_rows(A, M, K, K, A, A, A, 4096, seg, id_base, logits, ld, words, scratch, nb, None)
+
+    assert call(seg=tf.tf_seg(0, 0)) == tf.TF_E_ARG                 # an empty slice has no argmax
+    assert call(id_base=0x7FFFFFFF - 100) == tf.TF_E_RANGE           # ids past 2^31
+    assert call(seg=tf.tf_seg(4000, 200)) == tf.TF_E_RANGE           # rows past the matrix
+    assert call(M=129) == tf.TF_E_ARG
+    assert call(ld=100) == tf.TF_E_ARG
+    assert call(words=0) == tf.TF_E_ARG
+    assert call(scratch=0) == tf.TF_E_ARG
+    assert call(words=A + 4) == tf.TF_E_ALIGN
+    assert call(nbytes=8) == tf.TF_E_ARG
+    assert call(M=0, words=0, scratch=0) == tf.TF_OK                # nothing to do, nothing read
+    need1 = tf.tf_qmm_argmax_scratch_bytes(1, 124160)
+    assert need1 >= tf.tf_argmax_scratch_bytes(1, 124160) and need1 % 8 == 0
+    assert tf.tf_qmm_argmax_scratch_bytes(16, 124160) >= tf.tf_argmax_scratch_bytes(16, 124160)
+    assert tf.tf_qmm_argmax_scratch_bytes(0, 5) == 0 and tf.tf_qmm_argmax_scratch_bytes(1, 0) == 0
+
+
+def test_last_cuda_error_is_static_text(tf):
+    assert tf.tf_last_cuda_error() == "no error"
+
+
 def test_pick_refusals(tf):
     L = tf.lib
     assert L.tf_pick(A, 0, 1, A, None) == tf.TF_E_ARG
