@@ -49,6 +49,8 @@ PINS = {
     "pick": "exhaustive flag x flag x {<,=,>} truth table; split-then-pick == whole on every split point",
     "half_rows": "the pages' spans 2,560/8,704/124,160 of 5,120/17,408/248,320",
     "top2_gap": "hand cases (ties give 0, n=1 gives inf)",
+    "residual_add": "exact sums bf16 cannot hold; the fp32 round-to-even tie; IEEE specials; numpy float32 addition",
+    "embed_rows": "brute-force row lookup; bound refusals incl. the pages' 124,160-of-248,320 shard width; NaN rows past the bound",
     "end_to_end_on_real_weights": "parity unpinned: the pages print no numeric worked example",
 }
 
@@ -105,6 +107,10 @@ class Oracle:
         L.orc_pick.argtypes = [_P, _I32, _I32, _P]
         L.orc_top2_gap.restype = None
         L.orc_top2_gap.argtypes = [_P, _I32, _I64, _P]
+        L.orc_residual_add.restype = None
+        L.orc_residual_add.argtypes = [_P, _P, _P, _I64]
+        L.orc_embed_rows.restype = _I32
+        L.orc_embed_rows.argtypes = [_P, _I64, _I64, _I64, _I64, _P, _I32, _P, _I64]
         self.L = L
 
     # -- scalar helpers ------------------------------------------------------
@@ -155,6 +161,27 @@ class Oracle:
         a64 = np.empty(g.shape, dtype=np.float64) if want_f64 else None
         self.L.orc_glu(_ptr(g), _ptr(u), _ptr(a), _ptr(a64), g.size)
         return (a, a64) if want_f64 else a
+
+    # -- residual stream and embedding rows -----------------------------------
+    def residual_add(self, h: np.ndarray, y: np.ndarray) -> np.ndarray:
+        """fp32(h + y) elementwise: the fp32 residual stream plus a bf16 row."""
+        h = np.ascontiguousarray(h, dtype=np.float32)
+        y = np.ascontiguousarray(y, dtype=np.uint16)
+        assert h.shape == y.shape
+        out = np.empty_like(h)
+        self.L.orc_residual_add(_ptr(h), _ptr(y), _ptr(out), h.size)
+        return out
+
+    def embed_rows(self, table: np.ndarray, ids: np.ndarray, bound: int) -> np.ndarray:
+        """Rows of ``table`` (bf16 bits [rows, H]) for token ``ids``; an id at or
+        past ``bound`` gives a NaN row.  ValueError when bound != rows."""
+        table = np.ascontiguousarray(table, dtype=np.uint16)
+        ids = np.ascontiguousarray(ids, dtype=np.uint32)
+        rows, H = table.shape
+        out = np.empty((ids.size, H), dtype=np.uint16)
+        if self.L.orc_embed_rows(_ptr(table), rows, H, H, int(bound), _ptr(ids), ids.size, _ptr(out), H) != 0:
+            raise ValueError("orc_embed_rows: the bound must be the whole table's row count")
+        return out
 
     # -- split / gather -------------------------------------------------------
     def half_rows(self, h: int, nparts: int, N: int):

@@ -25,6 +25,14 @@
  *   pick     any flagged word -> 0xFFFFFFFF, else the larger value, lower id on
  *            ties (PR #1433 step-1 body; step-2 body: the pick is the better of
  *            the two half-vocab winners).
+ *   residual h' = fp32(h + y): a gathered bf16 projection row added to the fp32
+ *            residual stream (PR #1433 step-2 body: o_proj and down_proj gather
+ *            whole bf16 rows and add in the fp32 stream).
+ *   embed    out[m] = table[id_m], the whole table on every rank, ids checked
+ *            against the whole table's bound (PR #1433 step-2 body and the
+ *            "Rank-slice the qwen27 family and gather the whole embedding
+ *            table" commit: embedBound takes the whole table, refuses a smaller
+ *            bound).
  *
  * Readings taken where the pages are silent:
  *   nibble order  element k lives in byte k/2 of its row, low nibble for even k;
@@ -47,6 +55,8 @@
  *   7 dequant drops the bias term
  *   8 dequant swaps the nibble order inside a byte
  *   9 GLU uses SiLU(g)*u instead of g*SiLU(u)
+ *  10 the residual add rounds the sum to bf16 instead of fp32
+ *  11 the embedding gather checks ids against half of the bound (the shard's width)
  */
 #include <math.h>
 #include <stddef.h>
@@ -262,6 +272,56 @@ void orc_gather_rows(uint16_t *dst, int64_t ld_dst, const uint16_t *const *parts
                     src ? src[(int64_t)m * sw + (j < sw ? j : sw - 1)] : (uint16_t)ORC_NAN_BF16;
         off += widths[h];
     }
+}
+
+/* -------------------------------------------------------------- residual -- */
+
+/* out[i] = fp32(h[i] + y[i]) for n elements: a gathered bf16 projection row
+ * added to the fp32 residual stream (TensorFold PR #1433 step-2 body: o_proj
+ * and down_proj stage their rows, gather the peer's as whole bf16 rows and add
+ * in the fp32 stream, so no two bf16 partials are summed).  The sum is formed
+ * in double and rounded once to fp32 (round to nearest even): every fp32 + bf16
+ * sum whose exponents lie within 29 of each other is exact in double, and when
+ * they lie further apart the smaller term is far below half an fp32 ulp of the
+ * larger, so the one rounding is the fp32 addition's result.  NaN and +-Inf
+ * follow IEEE.  out may be h. */
+void orc_residual_add(const float *h, const uint16_t *y, float *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const double s = (double)h[i] + orc_bf16_to_f64(y[i]);
+#if ORC_PLANT == 10
+        out[i] = (float)orc_bf16_to_f64(orc_bf16_rne(s));
+#else
+        out[i] = (float)s;
+#endif
+    }
+}
+
+/* ----------------------------------------------------------------- embed -- */
+
+/* out[m, :H] = table[ids[m], :H]: the embedding rows of M token ids from the
+ * whole table, which every rank keeps whole (TensorFold PR #1433 step-2 body:
+ * "Embeddings and norms stay whole on every rank", the gather's bound is the
+ * whole 248,320-row table; the "Rank-slice the qwen27 family and gather the
+ * whole embedding table" commit: embedBound takes the whole table and refuses
+ * a bound below it).  Returns -1 and writes nothing when bound differs from the
+ * table's row count (below it is the shard-width bug; above it would read past
+ * the table).  An id at or past the bound fills its row with the bf16 NaN
+ * 0x7FC0, so the error reaches the head and fails closed. */
+int orc_embed_rows(const uint16_t *table, int64_t rows, int64_t H, int64_t ld, int64_t bound,
+                   const uint32_t *ids, int M, uint16_t *out, int64_t ld_out)
+{
+    if (bound != rows || H < 0 || ld < H || ld_out < H)
+        return -1;
+#if ORC_PLANT == 11
+    bound = bound / 2;
+#endif
+    for (int m = 0; m < M; ++m) {
+        const uint32_t id = ids[m];
+        for (int64_t j = 0; j < H; ++j)
+            out[(int64_t)m * ld_out + j] = (int64_t)id < bound ? table[(int64_t)id * ld + j] : (uint16_t)ORC_NAN_BF16;
+    }
+    return 0;
 }
 
 /* ---------------------------------------------------------------- argmax -- */

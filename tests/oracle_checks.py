@@ -371,9 +371,66 @@ def check_top2_gap(o):
     assert o.top2_gap(np.array([[2.0]]))[0] == math.inf
 
 
+def check_residual_add(o, seed=21):
+    """fp32(h + y) for an fp32 stream h and a bf16 row y (PR #1433 step-2 body:
+    the gathered rows are added in the fp32 stream)."""
+    f32 = np.float32
+    # exact sums that bf16 could not hold: 1 + 2^-10 and a 24-bit result
+    assert o.residual_add(np.array([1.0], f32), np.array([bf16_of(2.0 ** -10)], np.uint16))[0] == f32(1.0 + 2.0 ** -10)
+    h = np.array([2.0 ** 23 + 1], f32)
+    assert o.residual_add(h, np.array([bf16_of(1.0)], np.uint16))[0] == f32(2.0 ** 23 + 2)
+    # a tie at fp32 precision rounds to even: (1 + 2^-23) + 2^-24 -> 1 + 2^-22
+    r = o.residual_add(np.array([1.0 + 2.0 ** -23], f32), np.array([bf16_of(2.0 ** -24)], np.uint16))[0]
+    assert r == f32(1.0 + 2.0 ** -22)
+    # 1 + 2^-24 alone is the tie below, which rounds down to 1
+    assert o.residual_add(np.array([1.0], f32), np.array([bf16_of(2.0 ** -24)], np.uint16))[0] == f32(1.0)
+    # IEEE specials
+    inf = float("inf")
+    out = o.residual_add(np.array([inf, inf, 1.0, float("nan"), -0.0], f32),
+                         np.array([bf16_of(1.0), 0xFF80, 0x7FC0, bf16_of(1.0), 0x8000], np.uint16))
+    assert out[0] == inf and np.isnan(out[1]) and np.isnan(out[2]) and np.isnan(out[3])
+    assert out[4] == 0.0 and np.signbit(out[4])   # -0 + -0 = -0
+    # against numpy's IEEE float32 addition on random streams and rows
+    rng = np.random.default_rng(seed)
+    h = (rng.standard_normal(4096) * np.exp2(rng.integers(-20, 20, 4096))).astype(f32)
+    y = synth.to_bf16_bits((rng.standard_normal(4096) * np.exp2(rng.integers(-30, 30, 4096))).astype(f32))
+    want = h + synth.bf16_bits_to_f32(y)
+    assert np.array_equal(o.residual_add(h, y).view(np.uint32), want.view(np.uint32))
+
+
+def check_embed_rows(o, seed=22):
+    """Rows of the whole table by token id; the bound is the whole table (the
+    pages' fix: a bound below the table, e.g. the shard's 124,160 of 248,320,
+    is refused), and an id at or past it gives a NaN row."""
+    rng = np.random.default_rng(seed)
+    rows, H = 64, 24
+    table = rng.integers(0, 1 << 16, size=(rows, H), dtype=np.uint16)
+    ids = np.array([0, 63, 5, 32, 31, 64, 1000, 0xFFFFFFFF], dtype=np.uint32)
+    out = o.embed_rows(table, ids, rows)
+    for m, i in enumerate(ids):
+        want = table[i] if i < rows else np.full(H, NAN, np.uint16)
+        assert np.array_equal(out[m], want), (m, int(i))
+    for bad in (rows // 2, rows - 1, rows + 1):      # half the table: the shard-width bound
+        try:
+            o.embed_rows(table, ids, bad)
+        except ValueError:
+            continue
+        raise AssertionError(f"bound {bad} of a {rows}-row table was accepted")
+    # the pages' numbers: a 248,320-row table with the shard's 124,160 as the bound
+    big = np.zeros((synth.VOCAB, 1), dtype=np.uint16)
+    big[200000, 0] = 0x3F80
+    got = o.embed_rows(big, np.array([200000], dtype=np.uint32), synth.VOCAB)
+    assert got[0, 0] == 0x3F80
+    try:
+        o.embed_rows(big, np.array([200000], dtype=np.uint32), synth.VOCAB // 2)
+        raise AssertionError("the shard width was accepted as the embedding bound")
+    except ValueError:
+        pass
+
+
 ALL_CHECKS = [
     check_bf16_rne_hand, check_bf16_rne_vs_torch, check_hand_cases, check_dequant_closed_forms,
     check_one_hot, check_zero_rows, check_constant_q, check_vs_numpy_matmul, check_rows_order_free,
     check_glu, check_spans, check_gather, check_split_equals_whole_mlp, check_argmax_bruteforce,
-    check_pick_truth_table, check_split_pick_equals_whole, check_top2_gap,
+    check_pick_truth_table, check_split_pick_equals_whole, check_top2_gap, check_residual_add, check_embed_rows,
 ]

@@ -4,7 +4,8 @@ controls for the seam (TensorFold PR #1433, step-1 body: a stage on the
 peer's half, a gather writing its own half twice, an argmax and a pick that
 tie to the higher id, an argmax that does not flag, a pick whose flag test is
 dropped) plus three for the arithmetic (bias dropped, nibbles swapped, GLU
-orientation swapped).  Only the oracle is ever broken; no broken kernel is
+orientation swapped) and two for the adjacent steps (a residual add rounded to
+bf16, an embedding bound taken from the shard's width).  Only the oracle is ever broken; no broken kernel is
 built or run."""
 import pytest
 
@@ -21,6 +22,8 @@ PLANTS = {
     7: [C.check_hand_cases, C.check_vs_numpy_matmul, C.check_dequant_closed_forms],
     8: [C.check_hand_cases, C.check_one_hot],
     9: [C.check_glu],
+    10: [C.check_residual_add],
+    11: [C.check_embed_rows],
 }
 
 
