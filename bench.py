@@ -323,6 +323,39 @@ KERNELS = {   # name: (rows, K, segments, epilogue)
 }
 
 
+ADJACENT = ("residual_add", "embed_rows")
+
+
+def run_adjacent(args):
+    """The steps either side of the seam, --reps times: the fp32 residual add of
+    a 5,120-wide bf16 row (10 B per element) and the embedding rows of M token
+    ids from the whole 248,320 x 5,120 table (4 B per element)."""
+    import torch
+    import row_split_int4_b200 as tf
+    H, V, M = 5120, 248320, args.M
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    if args.kernel == "residual_add":
+        h = torch.randn(M, H, device="cuda", generator=g)
+        y = torch.randn(M, H, device="cuda", generator=g).to(torch.bfloat16)
+        call, nbytes = (lambda: tf.tf_residual_add(h, y)), 10 * M * H
+    else:
+        table = torch.randn(V, H, device="cuda", generator=g).to(torch.bfloat16)
+        ids = torch.randint(0, V, (M,), device="cuda", generator=g, dtype=torch.int32)
+        out = torch.empty(M, H, dtype=torch.bfloat16, device="cuda")
+        call, nbytes = (lambda: tf.tf_embed_rows(table, V, ids, out)), 4 * M * H
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.reps)]
+    for a, b in ev:
+        a.record()
+        call()
+        b.record()
+    torch.cuda.synchronize()
+    us = [a.elapsed_time(b) * 1e3 for a, b in ev]
+    best = min(us[1:] or us)
+    print(json.dumps({"kernel": args.kernel, "M": M, "H": H, "us": [round(u, 2) for u in us[:8]],
+                      "best_us": round(best, 2), "GB/s": round(nbytes / best / 1e3, 1), "bytes": nbytes}))
+    return 0
+
+
 def run_kernel(args):
     """One qmm call of the decode step, --reps times, on random bytes (the small
     case the kernel profiles are captured on)."""
@@ -452,7 +485,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="per-point sweep over M and the four shapes")
     ap.add_argument("--reps", type=int, default=1000)
-    ap.add_argument("--kernel", choices=sorted(KERNELS), help="time one qmm call of the step (profiling driver)")
+    ap.add_argument("--kernel", choices=sorted(KERNELS) + list(ADJACENT),
+                    help="time one call of a step of the path (profiling driver)")
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--shapes", default="", help="sweep: comma-separated subset of " + ",".join(SWEEP_SHAPES))
     ap.add_argument("--sweep-m", default="", help="sweep: comma-separated M values")
@@ -462,6 +496,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.kernel in ADJACENT:
+        return run_adjacent(args)
     if args.kernel:
         return run_kernel(args)
 

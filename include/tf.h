@@ -205,6 +205,44 @@ tf_status tf_qmm_argmax_rows(const void *x, int M, int K, int ldx, const uint8_t
                              int ld_logits, uint64_t *words, void *scratch, size_t scratch_bytes, tf_stream stream);
 
 /*
+ * tf_residual_add -- the fp32 residual stream after a seam (TensorFold PR #1433
+ * step-2 body: o_proj and down_proj stage their own output rows, gather the
+ * peer's as whole bf16 rows, and add in the fp32 stream, so no two bf16
+ * partials are summed).
+ *
+ * h[m][j] = fp32(h[m][j] + y[m][j]) for m < M, j < n: the IEEE fp32 addition,
+ * one rounding to nearest even; NaN and +-Inf follow IEEE.
+ *   h   fp32 [M][ld_h], ld_h >= n, 4-byte aligned, updated in place.
+ *   y   bf16 [M][ld_y], ld_y >= n, 2-byte aligned (e.g. a tf_gather_rows frame).
+ *   16-byte aligned pointers with ld_h % 4 == 0 and ld_y % 8 == 0 take the vector
+ *   path; both paths give the same bits.  M == 0 or n == 0 does nothing.
+ * Errors: TF_E_ARG, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+tf_status tf_residual_add(float *h, int ld_h, const void *y, int ld_y, int M, int n, tf_stream stream);
+
+/*
+ * tf_embed_rows -- the embedding rows of M token ids from the whole table
+ * (TensorFold PR #1433 step-2 body: embeddings stay whole on every rank, so a
+ * token id means the same thing on both, and the gather's bound stays the whole
+ * 248,320-row table; the "Rank-slice the qwen27 family and gather the whole
+ * embedding table" commit: embedBound takes the whole table and refuses a bound
+ * below it).
+ *
+ * out[m][:H] = table[ids[m]][:H]; an id >= bound makes row m the bf16 NaN
+ * 0x7FC0 everywhere, so the error reaches the head and fails closed.
+ *   table  bf16 [rows][ld_table], ld_table >= H, 2-byte aligned.
+ *   bound  must equal rows: a smaller bound (the shard's width, e.g. 124,160 of
+ *          248,320) is the bug the pages fixed and a larger one would read past
+ *          the table; either is refused with TF_E_RANGE before any launch.
+ *   ids    uint32 [M] on the device.   out  bf16 [M][ld_out], ld_out >= H.
+ *   16-byte aligned table and out with both leading dimensions % 8 == 0 take
+ *   the vector path.  M == 0 or H == 0 does nothing.
+ * Errors: TF_E_ARG, TF_E_RANGE, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+tf_status tf_embed_rows(const void *table, int rows, int H, int ld_table, int bound, const uint32_t *ids, int M,
+                        void *out, int ld_out, tf_stream stream);
+
+/*
  * tf_pick -- the better of the per-slice winners (TensorFold PR #1433 step-1
  * body: pair_pick; the sixth control's test ((am | ap) & PAIR_FLAG) != 0u).
  *

@@ -39,7 +39,8 @@ TF_EPI_NONE, TF_EPI_GLU = 0, 1
 
 EXPORTS = ["tf_qmm_rows", "tf_gather_rows", "tf_argmax_scratch_bytes", "tf_argmax_rows", "tf_pick",
            "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str", "tf_last_cuda_error",
-           "tf_abi_version", "tf_argmax_rows_static", "tf_qmm_argmax_rows", "tf_qmm_argmax_scratch_bytes"]
+           "tf_abi_version", "tf_argmax_rows_static", "tf_qmm_argmax_rows", "tf_qmm_argmax_scratch_bytes",
+           "tf_residual_add", "tf_embed_rows"]
 
 
 class tf_seg(ctypes.Structure):
@@ -60,6 +61,10 @@ lib.tf_qmm_argmax_scratch_bytes.argtypes = [_i, _i]
 lib.tf_qmm_argmax_rows.restype = _i
 lib.tf_qmm_argmax_rows.argtypes = [_vp, _i, _i, _i, _vp, _vp, _vp, _i, tf_seg, ctypes.c_uint32, _vp, _i, _vp, _vp, _sz,
                                    _vp]
+lib.tf_residual_add.restype = _i
+lib.tf_residual_add.argtypes = [_vp, _i, _vp, _i, _i, _i, _vp]
+lib.tf_embed_rows.restype = _i
+lib.tf_embed_rows.argtypes = [_vp, _i, _i, _i, _i, _vp, _i, _vp, _i, _vp]
 lib.tf_argmax_rows_static.restype = _i
 lib.tf_argmax_rows_static.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp]
 lib.tf_pick.restype = _i
@@ -178,6 +183,25 @@ def tf_qmm_argmax_rows(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, 
                                 wq.shape[0], tf_seg(int(seg[0]), int(seg[1])), int(id_base), _ptr(logits),
                                 _ld(logits), _ptr(words), _ptr(scratch), scratch.numel(), _stream(stream))
     return _ret(st, "tf_qmm_argmax_rows", check)
+
+
+def tf_residual_add(h: torch.Tensor, y: torch.Tensor, stream=None, check: bool = True) -> int:
+    """h[M, n] (fp32, in place) += y[M, n] (bf16), each sum rounded once to fp32."""
+    assert h.dtype == torch.float32 and y.dtype == torch.bfloat16 and h.shape == y.shape
+    M, n = h.shape
+    st = lib.tf_residual_add(_ptr(h), _ld(h), _ptr(y), _ld(y), M, n, _stream(stream))
+    return _ret(st, "tf_residual_add", check)
+
+
+def tf_embed_rows(table: torch.Tensor, bound: int, ids: torch.Tensor, out: torch.Tensor, stream=None,
+                  check: bool = True) -> int:
+    """out[M, H] = table[ids[m]] (bf16 rows); ids past ``bound`` give NaN rows.
+    ``bound`` must be the whole table's row count (TF_E_RANGE otherwise)."""
+    assert table.dtype == torch.bfloat16 and out.dtype == torch.bfloat16 and ids.dtype == torch.int32
+    rows, H = table.shape
+    st = lib.tf_embed_rows(_ptr(table), rows, H, _ld(table), int(bound), _ptr(ids), ids.numel(), _ptr(out),
+                           _ld(out), _stream(stream))
+    return _ret(st, "tf_embed_rows", check)
 
 
 def tf_gather_rows(dst: torch.Tensor, parts: Sequence[Optional[torch.Tensor]], widths: Sequence[int],

@@ -258,6 +258,29 @@ tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_b
     return cuda_status(launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tf_status tf_residual_add(float *h, int ld_h, const void *y, int ld_y, int M, int n, tf_stream stream) {
+    if (M < 0 || n < 0 || ld_h < n || ld_y < n) return TF_E_ARG;
+    if (M == 0 || n == 0) return TF_OK;
+    if (!h || !y) return TF_E_ARG;
+    if (!aligned(h, 4) || !aligned(y, 2)) return TF_E_ALIGN;
+    const bool vec = aligned(h, 16) && ld_h % 4 == 0 && aligned(y, 16) && ld_y % 8 == 0;
+    return cuda_status(launch_residual_add(h, ld_h, static_cast<const uint16_t *>(y), ld_y, M, n, vec,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tf_status tf_embed_rows(const void *table, int rows, int H, int ld_table, int bound, const uint32_t *ids, int M,
+                        void *out, int ld_out, tf_stream stream) {
+    if (rows < 1 || H < 0 || ld_table < H || ld_out < H || M < 0) return TF_E_ARG;
+    if (bound != rows) return TF_E_RANGE;   // below: the shard-width bound; above: past the table
+    if (M == 0 || H == 0) return TF_OK;
+    if (!table || !ids || !out) return TF_E_ARG;
+    if (!aligned(table, 2) || !aligned(out, 2) || !aligned(ids, 4)) return TF_E_ALIGN;
+    const bool vec = aligned(table, 16) && ld_table % 8 == 0 && aligned(out, 16) && ld_out % 8 == 0;
+    return cuda_status(launch_embed_rows(static_cast<const uint16_t *>(table), ld_table, (uint32_t)bound, H, ids, M,
+                                         static_cast<uint16_t *>(out), ld_out, vec,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_stream stream) {
     if (nparts < 1 || nparts > TF_MAX_PARTS || M < 0 || M > 65535) return TF_E_ARG;
     if (M == 0) return TF_OK;

@@ -74,6 +74,10 @@ cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream);
 int qmm_m1_stream_max_cand();   // an upper bound of the warps of any stream launch
 
 int argmax_blocks_per_row(int M, int n);
+cudaError_t launch_residual_add(float *h, long long ld_h, const uint16_t *y, long long ld_y, int M, int n, bool vec,
+                                cudaStream_t stream);
+cudaError_t launch_embed_rows(const uint16_t *table, long long ld_table, uint32_t bound, int H, const uint32_t *ids,
+                              int M, uint16_t *out, long long ld_out, bool vec, cudaStream_t stream);
 // TF_OK for cudaSuccess; otherwise remembers e for tf_last_cuda_error and returns TF_E_CUDA.
 tf_status cuda_status(cudaError_t e);
 cudaError_t last_cuda_error();

@@ -178,6 +178,25 @@ def test_fused_head_refusals(tf):
     assert tf.tf_qmm_argmax_scratch_bytes(0, 5) == 0 and tf.tf_qmm_argmax_scratch_bytes(1, 0) == 0
 
 
+def test_residual_and_embed_refusals(tf):
+    L = tf.lib
+    assert L.tf_residual_add(A, 8, A, 8, -1, 8, None) == tf.TF_E_ARG
+    assert L.tf_residual_add(A, 4, A, 8, 1, 8, None) == tf.TF_E_ARG        # ld_h < n
+    assert L.tf_residual_add(0, 8, A, 8, 1, 8, None) == tf.TF_E_ARG
+    assert L.tf_residual_add(A + 2, 8, A, 8, 1, 8, None) == tf.TF_E_ALIGN
+    assert L.tf_residual_add(A, 8, A + 1, 8, 1, 8, None) == tf.TF_E_ALIGN
+    assert L.tf_residual_add(0, 8, 0, 8, 0, 8, None) == tf.TF_OK          # nothing to do
+    V, H = 248320, 5120
+    # the pages' regression: the shard's 124,160 as the bound of the whole table is refused
+    assert L.tf_embed_rows(A, V, H, H, V // 2, A, 1, A, H, None) == tf.TF_E_RANGE
+    assert L.tf_embed_rows(A, V, H, H, V + 1, A, 1, A, H, None) == tf.TF_E_RANGE
+    assert L.tf_embed_rows(A, 0, H, H, 0, A, 1, A, H, None) == tf.TF_E_ARG
+    assert L.tf_embed_rows(A, V, H, H - 1, V, A, 1, A, H, None) == tf.TF_E_ARG
+    assert L.tf_embed_rows(A, V, H, H, V, 0, 1, A, H, None) == tf.TF_E_ARG
+    assert L.tf_embed_rows(A, V, H, H, V, A + 2, 1, A, H, None) == tf.TF_E_ALIGN
+    assert L.tf_embed_rows(A, V, H, H, V, A, 0, A, H, None) == tf.TF_OK
+
+
 def test_last_cuda_error_is_static_text(tf):
     assert tf.tf_last_cuda_error() == "no error"
 
