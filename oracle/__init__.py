@@ -49,6 +49,7 @@ PINS = {
     "pick": "exhaustive flag x flag x {<,=,>} truth table; split-then-pick == whole on every split point",
     "half_rows": "the pages' spans 2,560/8,704/124,160 of 5,120/17,408/248,320",
     "top2_gap": "hand cases (ties give 0, n=1 gives inf)",
+    "qmm8_rows": "one-hot x; constant-code closed form; numpy float64 matmul; the sign of the codes",
     "residual_add": "exact sums bf16 cannot hold; the fp32 round-to-even tie; IEEE specials; numpy float32 addition",
     "embed_rows": "brute-force row lookup; bound refusals incl. the pages' 124,160-of-248,320 shard width; NaN rows past the bound",
     "end_to_end_on_real_weights": "parity unpinned: the pages print no numeric worked example",
@@ -107,6 +108,8 @@ class Oracle:
         L.orc_pick.argtypes = [_P, _I32, _I32, _P]
         L.orc_top2_gap.restype = None
         L.orc_top2_gap.argtypes = [_P, _I32, _I64, _P]
+        L.orc_qmm8_rows.restype = _I32
+        L.orc_qmm8_rows.argtypes = [_P, _I32, _I32, _I64, _P, _P, _P, _I64, _P, _I64, _P, _P, _I32]
         L.orc_residual_add.restype = None
         L.orc_residual_add.argtypes = [_P, _P, _P, _I64]
         L.orc_embed_rows.restype = _I32
@@ -161,6 +164,29 @@ class Oracle:
         a64 = np.empty(g.shape, dtype=np.float64) if want_f64 else None
         self.L.orc_glu(_ptr(g), _ptr(u), _ptr(a), _ptr(a64), g.size)
         return (a, a64) if want_f64 else a
+
+    def qmm8_rows(self, x: np.ndarray, q8: np.ndarray, scales: np.ndarray, rows: Sequence[int],
+                  nthreads: int = 1, want_f64: bool = False):
+        """The int8 head: bf16 of s[n] * sum_k x q8[n,k] for the listed rows.
+        q8: int8 [N, K]; scales: uint16 [N] bf16 bits."""
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        if x.ndim == 1:
+            x = x[None, :]
+        M, K = x.shape
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nr = rows.size
+        assert q8.dtype == np.int8 and q8.flags.c_contiguous and q8.shape[1] == K
+        assert scales.dtype == np.uint16 and scales.shape == (q8.shape[0],)
+        if nr:
+            assert rows.min() >= 0 and rows.max() < q8.shape[0]
+        y = np.empty((M, nr), dtype=np.uint16)
+        y64 = np.empty((M, nr), dtype=np.float64) if want_f64 else None
+        ad = np.empty((M, nr), dtype=np.float64) if want_f64 else None
+        rc = self.L.orc_qmm8_rows(_ptr(x), M, K, K, _ptr(q8), _ptr(np.ascontiguousarray(scales)), _ptr(rows), nr,
+                                  _ptr(y), nr, _ptr(y64), _ptr(ad), int(nthreads))
+        if rc != 0:
+            raise ValueError("orc_qmm8_rows: bad arguments")
+        return (y, y64, ad) if want_f64 else y
 
     # -- residual stream and embedding rows -----------------------------------
     def residual_add(self, h: np.ndarray, y: np.ndarray) -> np.ndarray:

@@ -28,6 +28,9 @@
  *   residual h' = fp32(h + y): a gathered bf16 projection row added to the fp32
  *            residual stream (PR #1433 step-2 body: o_proj and down_proj gather
  *            whole bf16 rows and add in the fp32 stream).
+ *   qmm8     y[m,n] = bf16_RNE( s[n] * sum_k x[m,k] q8[n,k] ): the int8 lm_head
+ *            with one bf16 scale per row (the b70 lab's "runtime INT8 target
+ *            LM-head", bf16 scale).
  *   embed    out[m] = table[id_m], the whole table on every rank, ids checked
  *            against the whole table's bound (PR #1433 step-2 body and the
  *            "Rank-slice the qwen27 family and gather the whole embedding
@@ -57,6 +60,7 @@
  *   9 GLU uses SiLU(g)*u instead of g*SiLU(u)
  *  10 the residual add rounds the sum to bf16 instead of fp32
  *  11 the embedding gather checks ids against half of the bound (the shard's width)
+ *  12 the int8 head reads its codes as unsigned bytes
  */
 #include <math.h>
 #include <stddef.h>
@@ -206,6 +210,49 @@ int orc_qmm_rows(const uint16_t *x, int M, int K, int64_t ldx,
                 y64[(int64_t)m * nrows + i] = acc;
             if (absdot)
                 absdot[(int64_t)m * nrows + i] = aacc;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ qmm8 -- */
+
+/* The int8 head: y[m,i] = bf16_RNE( s[n] * sum_k x[m,k] * q[n,k] ), n = rows[i],
+ * with q the signed byte q8[n,k] (row-major [N][K]) and s[n] one bf16 scale per
+ * row -- the "runtime INT8 target LM-head" with a bf16 scale of the b70 lab's
+ * Qwen3.6 27B profile ("Reproduce Qwen3.6 27B AutoRound Bring-Up", *Reproduce
+ * The TP1 One-Replica Result*); the pages give no other detail, so the codes
+ * are symmetric (no zero point).  Each product x*q is exact in double and the
+ * sum runs over ascending k, as for the 4-bit format.  y64/absdot as there. */
+int orc_qmm8_rows(const uint16_t *x, int M, int K, int64_t ldx, const int8_t *q8, const uint16_t *scales,
+                  const int64_t *rows, int64_t nrows, uint16_t *y, int64_t ldy, double *y64, double *absdot,
+                  int nthreads)
+{
+    if (M < 0 || K < 0 || nrows < 0 || ldx < K || ldy < nrows)
+        return -1;
+#pragma omp parallel for schedule(dynamic, 16) num_threads(nthreads > 0 ? nthreads : 1) if (nthreads > 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t n = rows[i];
+        const int8_t *qrow = q8 + n * (int64_t)K;
+        const double s = orc_bf16_to_f64(scales[n]);
+        for (int m = 0; m < M; ++m) {
+            const uint16_t *xr = x + (int64_t)m * ldx;
+            double acc = 0.0, aacc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+#if ORC_PLANT == 12
+                const double q = (double)(uint8_t)qrow[k];
+#else
+                const double q = (double)qrow[k];
+#endif
+                const double p = orc_bf16_to_f64(xr[k]) * q;
+                acc += p;
+                aacc += fabs(p);
+            }
+            y[(int64_t)m * ldy + i] = orc_bf16_rne(s * acc);
+            if (y64)
+                y64[(int64_t)m * nrows + i] = s * acc;
+            if (absdot)
+                absdot[(int64_t)m * nrows + i] = fabs(s) * aacc;
         }
     }
     return 0;

@@ -32,6 +32,7 @@ TAG_X = 2
 TAG_W2 = 3
 TAG_HEAD = 4
 TAG_ATTN = 6
+TAG_HEAD8 = 7
 
 
 def to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -89,6 +90,40 @@ def make_weights(N: int, K: int, seed: int = 0, tag: int = TAG_W) -> QWeights:
         sc[r0:r1] = s
         bi[r0:r1] = b
     return QWeights(wq, sc, bi)
+
+
+@dataclass
+class Q8Weights:
+    """An int8 matrix with one bf16 scale per row (the int8 head)."""
+    q8: np.ndarray      # int8   [N, K]
+    scales: np.ndarray  # uint16 [N]
+
+    @property
+    def N(self) -> int:
+        return self.q8.shape[0]
+
+    @property
+    def K(self) -> int:
+        return self.q8.shape[1]
+
+    def astuple(self):
+        return (self.q8, self.scales)
+
+
+def make_weights8(N: int, K: int, seed: int = 0, tag: int = TAG_HEAD8) -> Q8Weights:
+    """Symmetric int8 codes, uniform over [-127, 127], and a bf16 row scale
+    uniform over [1e-4, 2e-4] (|w| up to ~0.025, the 4-bit head's range)."""
+    rng = np.random.default_rng([seed, tag])
+    q8 = np.empty((N, K), dtype=np.int8)
+    for r0 in range(0, N, BLOCK_ROWS):
+        r1 = min(N, r0 + BLOCK_ROWS)
+        q8[r0:r1] = rng.integers(-127, 128, size=(r1 - r0, K), dtype=np.int8)
+    sc = to_bf16_bits(rng.uniform(1e-4, 2e-4, size=N).astype(np.float32))
+    return Q8Weights(q8, sc)
+
+
+def weights8_to_device(w: Q8Weights, device="cuda"):
+    return (torch.from_numpy(w.q8).to(device), to_device(w.scales, device))
 
 
 def make_x(M: int, K: int, seed: int = 0, tag: int = TAG_X) -> np.ndarray:

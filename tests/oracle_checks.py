@@ -371,6 +371,41 @@ def check_top2_gap(o):
     assert o.top2_gap(np.array([[2.0]]))[0] == math.inf
 
 
+def check_qmm8(o, seed=23):
+    """The int8 head y = bf16(s * sum x q8): one-hot x (an exact product), a
+    constant code (closed form s * q * sum x), numpy's float64 matmul, and the
+    sign of the codes (-128 and 127 at the ends of the range)."""
+    rng = np.random.default_rng(seed)
+    N, K = 6, 256
+    w = synth.make_weights8(N, K, seed=seed)
+    # one-hot x: y = bf16(s_n * c * q[n, k])
+    for k in (0, 77, K - 1):
+        x = np.zeros((1, K), np.uint16)
+        x[0, k] = bf16_of(-1.5)
+        y = o.qmm8_rows(x, w.q8, w.scales, range(N))
+        # s * -1.5 * q is exact in fp32 (8 + 2 + 8 bits): torch's fp32 -> bf16 rounds it independently
+        prod = np.array([synth.bf16_bits_to_f32(w.scales[n]).item() * -1.5 * int(w.q8[n, k]) for n in range(N)], np.float32)
+        want = list(synth.to_bf16_bits(prod))
+        assert list(y[0]) == want, (k, list(y[0]), want)
+    # constant code: y = bf16(s * q * sum x)
+    q = np.full((2, K), -128, np.int8)
+    q[1] = 127
+    sc = np.array([bf16_of(0.25), bf16_of(2.0 ** -7)], np.uint16)
+    x = synth.to_bf16_bits(rng.standard_normal((3, K)).astype(np.float32))
+    xs = synth.bf16_bits_to_f32(x).astype(np.float64).sum(axis=1)
+    y = o.qmm8_rows(x, q, sc, [0, 1])
+    # (the rounding of the closed form uses the oracle's bf16_rne, pinned on its own above)
+    want = o.bf16_rne(np.stack([0.25 * -128 * xs, 2.0 ** -7 * 127 * xs], axis=1))
+    assert np.array_equal(y, want)
+    # numpy float64 matmul
+    x = synth.to_bf16_bits(rng.standard_normal((4, K)).astype(np.float32))
+    y, y64, _ = o.qmm8_rows(x, w.q8, w.scales, range(N), want_f64=True)
+    ref = (synth.bf16_bits_to_f32(x).astype(np.float64) @ w.q8.astype(np.float64).T) * \
+        synth.bf16_bits_to_f32(w.scales).astype(np.float64)[None, :]
+    assert np.allclose(y64, ref, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(y, o.bf16_rne(ref))
+
+
 def check_residual_add(o, seed=21):
     """fp32(h + y) for an fp32 stream h and a bf16 row y (PR #1433 step-2 body:
     the gathered rows are added in the fp32 stream)."""
@@ -432,5 +467,5 @@ ALL_CHECKS = [
     check_bf16_rne_hand, check_bf16_rne_vs_torch, check_hand_cases, check_dequant_closed_forms,
     check_one_hot, check_zero_rows, check_constant_q, check_vs_numpy_matmul, check_rows_order_free,
     check_glu, check_spans, check_gather, check_split_equals_whole_mlp, check_argmax_bruteforce,
-    check_pick_truth_table, check_split_pick_equals_whole, check_top2_gap, check_residual_add, check_embed_rows,
+    check_pick_truth_table, check_split_pick_equals_whole, check_top2_gap, check_residual_add, check_embed_rows, check_qmm8,
 ]

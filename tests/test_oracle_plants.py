@@ -24,6 +24,7 @@ PLANTS = {
     9: [C.check_glu],
     10: [C.check_residual_add],
     11: [C.check_embed_rows],
+    12: [C.check_qmm8],
 }
 
 
