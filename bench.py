@@ -323,7 +323,7 @@ KERNELS = {   # name: (rows, K, segments, epilogue)
 }
 
 
-ADJACENT = ("residual_add", "embed_rows")
+ADJACENT = ("residual_add", "embed_rows", "lm_head8_half")
 
 
 def run_adjacent(args):
@@ -338,6 +338,14 @@ def run_adjacent(args):
         h = torch.randn(M, H, device="cuda", generator=g)
         y = torch.randn(M, H, device="cuda", generator=g).to(torch.bfloat16)
         call, nbytes = (lambda: tf.tf_residual_add(h, y)), 10 * M * H
+    elif args.kernel == "lm_head8_half":
+        # the int8 head's half: 124,160 rows x 5,120 int8 codes and a bf16 scale per row
+        rows = V // 2
+        q8 = torch.randint(-128, 128, (rows, H), dtype=torch.int8, device="cuda", generator=g)
+        sc = (1e-4 + 1e-4 * torch.rand(rows, device="cuda", generator=g)).to(torch.bfloat16)
+        x = torch.randn(M, H, device="cuda", generator=g).to(torch.bfloat16)
+        y = torch.empty(M, rows, dtype=torch.bfloat16, device="cuda")
+        call, nbytes = (lambda: tf.tf_qmm8_rows(x, q8, sc, [(0, rows)], y)), rows * H + 2 * rows + 2 * M * H + 2 * M * rows
     else:
         table = torch.randn(V, H, device="cuda", generator=g).to(torch.bfloat16)
         ids = torch.randint(0, V, (M,), device="cuda", generator=g, dtype=torch.int32)

@@ -175,6 +175,26 @@ tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_b
                          uint64_t *words, void *scratch, size_t scratch_bytes, tf_stream stream);
 
 /*
+ * tf_qmm8_rows -- the int8 head variant: the b70 lab's "runtime INT8 target
+ * LM-head" with a bf16 scale ("Reproduce Qwen3.6 27B AutoRound Bring-Up",
+ * *Reproduce The TP1 One-Replica Result*; the pages give no other detail).
+ *
+ * y[m][c] = bf16_RNE( s[n] * sum_{k<K} x[m][k] * q8[n][k] ), n the whole-matrix
+ * row of output column c (segments as in tf_qmm_rows, TF_EPI_NONE), the sum in
+ * fp32 over the whole K on this device, in an order fixed by K alone.
+ *   x       bf16 [M][ldx], 1 <= K <= TF_MAX_K, ldx >= K, 0 <= M <= TF_BATCH_ROWS.
+ *   q8      int8 [N_whole][K], row-major, signed codes (no zero point).
+ *   scales  bf16 [N_whole], one per row.
+ *   y       bf16 [M][ldy], ldy >= the number of columns.
+ *   M = 1 with K % 32 == 0 and a 16-byte aligned q8 streams the codes through
+ *   shared memory (bulk copies, dp4a); other calls take a plain warp-per-output
+ *   kernel.  A row's bits depend on which of the two ran, never on the other rows.
+ * Errors: TF_E_ARG, TF_E_RANGE, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+tf_status tf_qmm8_rows(const void *x, int M, int K, int ldx, const int8_t *q8, const void *scales, int N_whole,
+                       const tf_seg *segs, int nseg, void *y, int ldy, tf_stream stream);
+
+/*
  * tf_qmm_argmax_rows -- the head of one rank in one call: the logits of one row
  * slice (tf_qmm_rows, TF_EPI_NONE, one segment) and their argmax word
  * (tf_argmax_rows over those logits with ids id_base + j).  The step-1 body of

@@ -40,7 +40,7 @@ TF_EPI_NONE, TF_EPI_GLU = 0, 1
 EXPORTS = ["tf_qmm_rows", "tf_gather_rows", "tf_argmax_scratch_bytes", "tf_argmax_rows", "tf_pick",
            "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str", "tf_last_cuda_error",
            "tf_abi_version", "tf_argmax_rows_static", "tf_qmm_argmax_rows", "tf_qmm_argmax_scratch_bytes",
-           "tf_residual_add", "tf_embed_rows"]
+           "tf_residual_add", "tf_embed_rows", "tf_qmm8_rows"]
 
 
 class tf_seg(ctypes.Structure):
@@ -61,6 +61,8 @@ lib.tf_qmm_argmax_scratch_bytes.argtypes = [_i, _i]
 lib.tf_qmm_argmax_rows.restype = _i
 lib.tf_qmm_argmax_rows.argtypes = [_vp, _i, _i, _i, _vp, _vp, _vp, _i, tf_seg, ctypes.c_uint32, _vp, _i, _vp, _vp, _sz,
                                    _vp]
+lib.tf_qmm8_rows.restype = _i
+lib.tf_qmm8_rows.argtypes = [_vp, _i, _i, _i, _vp, _vp, _i, ctypes.POINTER(tf_seg), _i, _vp, _i, _vp]
 lib.tf_residual_add.restype = _i
 lib.tf_residual_add.argtypes = [_vp, _i, _vp, _i, _i, _i, _vp]
 lib.tf_embed_rows.restype = _i
@@ -165,6 +167,17 @@ def tf_qmm_rows(x: torch.Tensor, wq: torch.Tensor, scales: torch.Tensor, biases:
     st = lib.tf_qmm_rows(_ptr(x), x.shape[0], x.shape[1], _ld(x), _ptr(wq), _ptr(scales), _ptr(biases),
                          wq.shape[0], arr, len(segs), int(epi), _ptr(y), _ld(y), _stream(stream))
     return _ret(st, "tf_qmm_rows", check)
+
+
+def tf_qmm8_rows(x: torch.Tensor, q8: torch.Tensor, scales: torch.Tensor, segs: Sequence[Tuple[int, int]],
+                 y: torch.Tensor, stream=None, check: bool = True) -> int:
+    """The int8 head: y[M, cols] = bf16(s[n] * x . q8[n]) for the listed rows."""
+    assert x.dtype == torch.bfloat16 and y.dtype == torch.bfloat16
+    assert q8.dtype == torch.int8 and scales.dtype == torch.bfloat16 and q8.is_contiguous()
+    arr = (tf_seg * max(1, len(segs)))(*[tf_seg(int(r0), int(n)) for r0, n in segs])
+    st = lib.tf_qmm8_rows(_ptr(x), x.shape[0], x.shape[1], _ld(x), _ptr(q8), _ptr(scales), q8.shape[0], arr,
+                          len(segs), _ptr(y), _ld(y), _stream(stream))
+    return _ret(st, "tf_qmm8_rows", check)
 
 
 def tf_qmm_argmax_scratch_bytes(M: int, nrows: int) -> int:

@@ -35,6 +35,7 @@
 // A unit is kRU rows: four consecutive output columns (TF_EPI_NONE), or the
 // gate and up rows of two consecutive columns (TF_EPI_GLU, rows g0 u0 g1 u1).
 #include "qmm_common.cuh"
+#include "stream_common.cuh"
 
 namespace tf {
 
@@ -68,53 +69,6 @@ __host__ __device__ inline StreamLayout stream_layout(int K, int warps, int ru) 
     L.ring_off = round_up(L.bar_off + (size_t)warps * stages_for(ru) * 8, 128);
     L.total = L.ring_off + (size_t)warps * stages_for(ru) * slot_bytes(ru);
     return L;
-}
-
-// ------------------------------------------------------------ PTX helpers --
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-// global -> this CTA's shared memory, completion counted on `bar` (no multicast)
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Wait for a slot's copies with an iteration limit.  A copy from valid global
-// memory always lands, so running out of iterations means the GPU is in
-// trouble: the warp then writes NaN for what it could not compute.
-__device__ __forceinline__ bool wait_slot(uint32_t bar, uint32_t parity, long long limit) {
-    for (long long it = 0; it < limit; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
-__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
-    int d;
-    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
 }
 
 // sum over the lane's 32 codes of q_k * F_k, as a float.  limb[j] (j = limb*2 +

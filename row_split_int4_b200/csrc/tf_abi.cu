@@ -149,6 +149,45 @@ tf_status tf_qmm_rows(const void *x, int M, int K, int ldx, const uint8_t *wq, c
     return cuda_status(launch_qmm(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tf_status tf_qmm8_rows(const void *x, int M, int K, int ldx, const int8_t *q8, const void *scales, int N_whole,
+                       const tf_seg *segs, int nseg, void *y, int ldy, tf_stream stream) {
+    if (M < 0 || M > TF_BATCH_ROWS) return TF_E_ARG;
+    if (K < 1 || K > TF_MAX_K) return TF_E_ARG;
+    if (N_whole < 1) return TF_E_ARG;
+    if (segs == nullptr || nseg < 1 || nseg > TF_MAX_SEGS) return TF_E_ARG;
+    Qmm8Args a;
+    std::memset(&a, 0, sizeof a);
+    long long cols = 0;
+    for (int i = 0; i < nseg; ++i) {
+        const long long r0 = segs[i].row0, nr = segs[i].nrows;
+        if (r0 < 0 || nr < 0 || r0 + nr > N_whole) return TF_E_RANGE;
+        for (int j = 0; j < i; ++j) {
+            const long long a0 = segs[j].row0, an = segs[j].nrows;
+            if (nr > 0 && an > 0 && r0 < a0 + an && a0 < r0 + nr) return TF_E_RANGE;
+        }
+        a.seg.row0[i] = (int)r0;
+        a.seg.nrows[i] = (int)nr;
+        a.seg.col0[i] = (int)cols;
+        cols += nr;
+    }
+    if (cols > INT_MAX) return TF_E_RANGE;
+    a.seg.nseg = nseg;
+    a.seg.ncols = (int)cols;
+    if (ldx < K || ldy < a.seg.ncols) return TF_E_ARG;
+    if (M == 0 || a.seg.ncols == 0) return TF_OK;
+    if (!x || !q8 || !scales || !y) return TF_E_ARG;
+    if (!aligned(x, 2) || !aligned(scales, 2) || !aligned(y, 2)) return TF_E_ALIGN;
+    a.x = static_cast<const uint16_t *>(x);
+    a.M = M;
+    a.K = K;
+    a.ldx = ldx;
+    a.q8 = q8;
+    a.scales = static_cast<const uint16_t *>(scales);
+    a.y = static_cast<uint16_t *>(y);
+    a.ldy = ldy;
+    return cuda_status(launch_qmm8(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t tf_qmm_argmax_scratch_bytes(int M, int nrows) {
     if (M <= 0 || nrows <= 0) return 0;
     // fused: one key per warp of the grid, then the finish counter

@@ -40,6 +40,17 @@ struct QmmArgs {
     uint64_t *word;
 };
 
+// The int8 head: codes [N][K] int8, one bf16 scale per row.
+struct Qmm8Args {
+    const uint16_t *x;
+    int M, K, ldx;
+    const int8_t *q8;
+    const uint16_t *scales;
+    SegTable seg;
+    uint16_t *y;
+    int ldy;
+};
+
 struct GatherArgs {
     uint16_t *dst;
     long long ld_dst;
@@ -64,6 +75,7 @@ struct ArgmaxArgs {
 };
 
 cudaError_t launch_qmm(const QmmArgs &a, cudaStream_t stream);
+cudaError_t launch_qmm8(const Qmm8Args &a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream);
 cudaError_t launch_argmax(ArgmaxArgs a, cudaStream_t stream);
 cudaError_t launch_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, cudaStream_t stream);

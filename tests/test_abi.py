@@ -197,6 +197,24 @@ def test_residual_and_embed_refusals(tf):
     assert L.tf_embed_rows(A, V, H, H, V, A, 0, A, H, None) == tf.TF_OK
 
 
+def test_qmm8_refusals(tf):
+    L = tf.lib
+
+    def call(x=A, M=1, K=1024, ldx=1024, q=A, sc=A, N=512, segs=((0, 256),), y=A, ldy=256):
+        arr = (tf.tf_seg * max(1, len(segs)))(*[tf.tf_seg(a, b) for a, b in segs])
+        return L.tf_qmm8_rows(x, M, K, ldx, q, sc, N, arr, len(segs), y, ldy, None)
+
+    assert call(M=129) == tf.TF_E_ARG
+    assert call(K=0) == tf.TF_E_ARG
+    assert call(ldx=1000) == tf.TF_E_ARG
+    assert call(segs=((400, 200),)) == tf.TF_E_RANGE
+    assert call(segs=((0, 100), (50, 100))) == tf.TF_E_RANGE
+    assert call(ldy=100) == tf.TF_E_ARG
+    assert call(q=0) == tf.TF_E_ARG
+    assert call(x=A + 1) == tf.TF_E_ALIGN
+    assert call(M=0, x=0, q=0, sc=0, y=0) == tf.TF_OK
+
+
 def test_last_cuda_error_is_static_text(tf):
     assert tf.tf_last_cuda_error() == "no error"
 
