@@ -10,9 +10,13 @@ two row halves on one GPU (TensorFold PR #1433, step-1 and step-2 bodies):
   gather   the two 8,704-wide activated halves         (tf_gather_rows)
   down     K=17,408 -> 5,120 rows as 2 x 2,560          (tf_qmm_rows)
   gather   the two 2,560-wide halves                    (tf_gather_rows)
-  lm_head  K=5,120 -> 248,320 rows as 2 x 124,160, each  (tf_qmm_argmax_rows: the
-           half's logits and its argmax word, global ids, fused)
+  lm_head  K=5,120 -> 248,320 rows as 2 x 124,160       (tf_qmm_rows)
+  argmax   per half, global ids                         (tf_argmax_rows)
   pick     the better half-winner                       (tf_pick)
+
+(tf_qmm_argmax_rows fuses the last three into one call per half; it measures the
+same time as the three launches, and the separate calls let the event pairs
+time the lm_head qmm kernel alone for the roofline.)
 
 The metric is the int4 dequant-GEMV HBM throughput (GB/s of algorithmic
 bytes: 0.5625 B per weight plus activations in and out), with the
@@ -195,13 +199,12 @@ class DecodeStep:
         self.logits = [torch.empty(1, V // 2, **bf) for _ in range(2)]
         self.words = torch.empty(2, 1, dtype=torch.int64, device="cuda")
         self.ids = torch.empty(1, dtype=torch.int32, device="cuda")
-        self.scratch = [torch.empty(tf.tf_qmm_argmax_scratch_bytes(1, V // 2), dtype=torch.uint8, device="cuda")
-                        for _ in range(2)]
+        self.scratch = torch.empty(tf.tf_argmax_scratch_bytes(1, V // 2), dtype=torch.uint8, device="cuda")
         self.member = [tf.tf_member_segs(F, 2, h) for h in range(2)]
         self.down_rows = [tf.tf_split_rows(H, 2, h) for h in range(2)]
         self.head_rows = [tf.tf_split_rows(V, 2, h) for h in range(2)]
         self.window = synth.WINDOW_BYTES
-        self.launches_per_step = 2 + 1 + 2 + 1 + 2 + 1   # the fused head: one qmm launch (and a 4-byte memset) per half
+        self.launches_per_step = 2 + 1 + 2 + 1 + 2 + 2 * 2 + 1
 
     def run(self, stream, lm_events=None, head_events=None):
         tf = self.tf
@@ -216,10 +219,11 @@ class DecodeStep:
         for h in range(2):
             if lm_events is not None:
                 lm_events[h][0].record(stream)
-            tf.tf_qmm_argmax_rows(self.x_head, *self.Wlm, self.head_rows[h], self.head_rows[h][0], self.logits[h],
-                                  self.words[h], self.scratch[h], stream=stream)
+            tf.tf_qmm_rows(self.x_head, *self.Wlm, [self.head_rows[h]], self.logits[h], stream=stream)
             if lm_events is not None:
                 lm_events[h][1].record(stream)
+        for h in range(2):
+            tf.tf_argmax_rows(self.logits[h], self.head_rows[h][0], self.words[h], self.scratch, stream=stream)
         tf.tf_pick(self.words, self.ids, stream=stream)
         if head_events is not None:
             head_events[1].record(stream)
@@ -606,8 +610,7 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "one GPU, two row halves"},
             "lm_head_argmax_us_per_token": round(statistics.fmean(head_ms) * 1e3, 2),
             "tokens_per_s_equiv": round(1e3 / ms_step, 1),
-            "roofline": {"bound": "hbm", "kernel": "qmm_m1_stream_kernel (lm_head half, 124,160 x 5,120; the fused "
-                                                "head call: the half's logits and argmax word)",
+            "roofline": {"bound": "hbm", "kernel": "qmm_m1_stream_kernel (lm_head half, 124,160 x 5,120)",
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic_from_profiles(src),
                          "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_avg_ms * 1e3, 3)},
