@@ -4,10 +4,12 @@
 // Why this shape on B200.  At M = 1 every weight byte is used once, and the 148
 // SMs must turn ~40 weights per clock each into products to keep up with HBM.
 // Two limits meet there:
-//   * bytes in flight: ~64 KB per SM are needed to cover HBM latency.  Each warp
-//     owns a ring of kStages shared-memory slots that its lanes refill with
-//     cp.async.bulk (the TMA engine's 1-D copy), so the copies stay in flight
-//     while the warp computes, independent of the register budget;
+//   * bytes in flight: ~130 KB per SM are needed to cover HBM latency under
+//     load.  Copies land in shared-memory rings through the TMA engine, so they
+//     stay in flight while the warps compute, independent of the register budget.
+//     Wide calls use the tile ring (2-D tensor copies of 16-row tiles filled by
+//     producer warps, below); narrow ones a ring per warp refilled by 1-D
+//     cp.async.bulk copies, one per row and array;
 //   * instructions per weight: floating-point nibble decoding costs 3-4 issue
 //     slots per weight, most of them integer-pipe work.  Here a word of 8 codes
 //     is split into two words of 4 bytes (2 lop3 + 1 shift) and multiplied with
@@ -36,6 +38,7 @@
 // gate and up rows of two consecutive columns (TF_EPI_GLU, rows g0 u0 g1 u1).
 #include "qmm_common.cuh"
 #include "stream_common.cuh"
+#include "tmap.h"
 
 namespace tf {
 
@@ -92,95 +95,16 @@ __device__ __forceinline__ float lane_chunk_idot(const uint4 &q, const uint4 *li
     return fmaf((float)a2, 65536.0f, fmaf((float)a1, 256.0f, (float)a0));
 }
 
-// ------------------------------------------------------------------ kernel --
-template <int kRU>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArgs a, int units) {
-    constexpr int kSlotBytes = slot_bytes(kRU);
-    constexpr int kStages = stages_for(kRU);
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int W = blockDim.x >> 5;
-    const StreamLayout L = stream_layout(a.K, W, kRU);
-    const int K = a.K, nch = L.nch;
-    const int nsl = (K + kKS - 1) / kKS;
-    const int G = K / kGroup;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint8_t *limbs = smem + L.limb_off;
-    float *Xs = reinterpret_cast<float *>(smem + L.X_off);
-    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
-    uint8_t *ring = smem + L.ring_off + (size_t)warp * kStages * kSlotBytes;
-    const uint32_t ring_s = smem_addr(ring);
-    const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kStages * 8);
-
-    const long long gw = (long long)blockIdx.x * W + warp;
-    const long long nw = (long long)gridDim.x * W;
-    const int u0 = (int)(gw * units / nw);
-    const int u1 = (int)((gw + 1) * units / nw);
-    const int steps = (u1 - u0) * nsl;
-
-    // copy role of this lane: array (lane % 3: codes, scales, biases) of unit row lane / 3
-    const int my_r = lane / 3, my_a = lane % 3;
-    const bool copier = lane < 3 * kRU;
-    const uint8_t *gbase = my_a == 0 ? a.wq
-                         : (my_a == 1 ? reinterpret_cast<const uint8_t *>(a.scales)
-                                      : reinterpret_cast<const uint8_t *>(a.biases));
-    const size_t grow = my_a == 0 ? (size_t)K / 2 : (size_t)G * 2;       // bytes per matrix row
-    const int kdiv = my_a == 0 ? 2 : 32;                                 // bytes of a K range = len / kdiv
-    const uint32_t doff = my_a == 0 ? my_r * kSlotQ
-                        : (my_a == 1 ? kRU * kSlotQ + my_r * kSlotS : kRU * kSlotQ + kRU * kSlotS + my_r * kSlotS);
-    constexpr int kCols = kRU / 2 > 0 ? kRU / 2 : 1;   // output columns of a GLU unit
-    auto unit_row = [&](int u, int r) {   // whole-matrix row of unit row r, -1 past the end
-        const int col = a.glu ? u * kCols + (r >> 1) : u * kRU + r;
-        return col < a.seg.ncols ? seg_row(a.seg, col, a.glu, a.glu ? (r & 1) : 0) : -1;
-    };
-    // rows of a unit that exist (the last unit of a launch may be short)
-    auto unit_live_rows = [&](int u) {
-        const int cols_left = a.seg.ncols - (a.glu ? u * kCols : u * kRU);
-        return a.glu ? 2 * min(kCols, cols_left) : min(kRU, cols_left);
-    };
-    // issue pointer: unit iu, K-slice ij of the next step whose copies go out
-    int iu = u0, ij = 0, it_ = 0;
-    int my_row = copier && u0 < u1 ? unit_row(u0, my_r) : -1;
-    int live = u0 < u1 ? unit_live_rows(u0) : 0;
-    bool failed = false;
-    auto issue_next = [&]() {
-        const int slot = it_ % kStages;
-        const int k0 = ij * kKS, len = min(kKS, K - k0);
-        const uint32_t bar = bar0 + 8 * slot;
-        if (lane == 0) mbar_expect_tx(bar, (uint32_t)(live * (len / 2 + 2 * (len / 32))));
-        __syncwarp();
-        if (copier && my_row >= 0)
-            bulk_g2s(ring_s + slot * kSlotBytes + doff, gbase + (size_t)my_row * grow + k0 / kdiv, (uint32_t)(len / kdiv),
-                     bar);
-        if (++ij == nsl) {
-            ij = 0;
-            ++iu;
-            if (iu < u1) {
-                my_row = copier ? unit_row(iu, my_r) : -1;
-                live = unit_live_rows(iu);
-            }
-        }
-        ++it_;
-    };
-
-    if (lane == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-    // Wide units send only their first slot's copies before the limb preparation:
-    // with every warp queueing its whole ring at once the copy queue fills and the
-    // issuing lanes wait, which would hold the preparation back; the rest follow
-    // it.  Narrow units, whose warps have few steps, queue their whole ring now.
-    constexpr int kPreStages = kRU >= 4 ? 1 : kStages;
-    for (int t = 0; t < kPreStages && t < steps; ++t) issue_next();
-
-    // fixed-point limbs of x, one warp per lane-chunk, one lane per value, on the
-    // bf16 fields alone: x = sign * M * 2^(e-134), M = 128 + mantissa (e >= 1) or
-    // the mantissa (e = 0, subnormal, read with e = 1).  With emax the chunk's
-    // largest e, F = x * 2^(23-E), E = emax - 126, is sign * M * 2^(e - emax + 15):
-    // a left shift when e >= emax - 15 (exact), else a right shift rounded to nearest even.
-    // (loads are issued sixteen lane-chunks at a time so that one L2 round trip
-    // covers all of them)
+// Fixed-point limbs of x for every lane-chunk, one warp per lane-chunk and one
+// lane per value, on the bf16 fields alone: x = sign * M * 2^(e-134), M = 128 +
+// mantissa (e >= 1) or the mantissa (e = 0, subnormal, read with e = 1).  With emax
+// the chunk's largest e, F = x * 2^(23-E), E = emax - 126, is sign * M * 2^(e - emax
+// + 15): a left shift when e >= emax - 15 (exact), else a right shift rounded to
+// nearest even.  Xs gets the fp32 sum of the chunk's 32 x, Ss the power of two
+// 2^(E-23) (NaN when the chunk holds a NaN or an infinity).
+__device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, float *Xs, float *Ss, int W,
+                                           int warp, int lane) {
+    // loads go out sixteen lane-chunks at a time so that one L2 round trip covers them
     constexpr int kPrepBatch = 16;
     for (int lc0 = warp; lc0 < nch * 32; lc0 += W * kPrepBatch) {
       uint32_t hb[kPrepBatch];
@@ -188,7 +112,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
       for (int i = 0; i < kPrepBatch; ++i) {
           const int lc = lc0 + i * W;
           const int k = (lc >> 5) * kChunk + (lc & 31) * 32 + lane;
-          hb[i] = (lc < nch * 32 && k < K) ? (uint32_t)a.x[k] : 0u;
+          hb[i] = (lc < nch * 32 && k < K) ? (uint32_t)x[k] : 0u;
       }
 #pragma unroll
       for (int i = 0; i < kPrepBatch; ++i) {
@@ -228,115 +152,501 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
         }
       }
     }
+}
+
+// Fused head: every warp publishes the largest argmax key of the rows it wrote;
+// the last CTA to finish (a fence, then a ticket: the usual last-block pattern)
+// reduces all of them into the argmax word and clears the ticket counter.
+__device__ __forceinline__ void fused_head_tail(const QmmArgs &a, uint64_t best, int W, int tid, int warp, int lane) {
+    if (lane == 0) a.cand[(long long)blockIdx.x * W + warp] = best;
+    __threadfence();
     __syncthreads();
-    for (int t = kPreStages; t < kStages && t < steps; ++t) issue_next();
+    __shared__ unsigned int ticket;
+    if (tid == 0) ticket = atomicAdd(a.done, 1u);
+    __syncthreads();
+    if (ticket == gridDim.x - 1) {
+        __threadfence();
+        const int ncand = (int)(gridDim.x * W);
+        uint64_t v = 0;
+        for (int i = tid; i < ncand; i += blockDim.x) v = umax64(v, ((volatile uint64_t *)a.cand)[i]);
+        v = warp_max64(v);
+        __shared__ uint64_t red[32];
+        if (lane == 0) red[warp] = v;
+        __syncthreads();
+        if (warp == 0) {
+            v = lane < W ? red[lane] : 0ull;
+            v = warp_max64(v);
+            if (lane == 0) {
+                *a.word = word_of_key(v, a.y, a.id_base);
+                *a.done = 0u;
+            }
+        }
+    }
+}
+
+// acc[r] += the x.w of unit row r over the chunks of one slot: chunk c0 + cc sits
+// at position cc of the slot.  A lane whose 32 values start at or past kend (K
+// covered by the slot) stops there.  Full slots pass compile-time nc and kend, so
+// their bounds fold away.
+template <int kRU>
+__device__ __forceinline__ void slot_dot(float (&acc)[kRU], const uint8_t *sl, const uint4 *limb_l, const float *Xs,
+                                         const float *Ss, int c0, int nc, int kend, int lane) {
+    const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
+    const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kRU * kSlotQ) + (lane >> 1);
+#pragma unroll
+    for (int cc = 0; cc < kKS / kChunk; ++cc) {
+        if (cc >= nc || cc * kChunk + lane * 32 >= kend) break;
+        const int c = c0 + cc;
+        uint4 lm[6];
+#pragma unroll
+        for (int q = 0; q < 6; ++q) lm[q] = limb_l[(c * 6 + q) * 32];
+        const float X = Xs[c * 32 + lane];
+        const float scale = Ss[c * 32 + lane];
+#pragma unroll
+        for (int r = 0; r < kRU; ++r) {
+            const uint4 qv = ql[(r * kSlotQ + cc * (kChunk / 2)) / 16];
+            const float s = bf16_bits_to_f32(sc16[r * (kKS / kGroup) + cc * 16]);
+            const float b = bf16_bits_to_f32(sc16[kRU * (kKS / kGroup) + r * (kKS / kGroup) + cc * 16]);
+            const float P = lane_chunk_idot(qv, lm);
+            acc[r] = fmaf(s, P * scale, acc[r]);   // P * 2^(E-23): exact power-of-two scaling
+            acc[r] = fmaf(b, X, acc[r]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ kernel --
+template <int kRU>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArgs a, int units) {
+    constexpr int kSlotBytes = slot_bytes(kRU);
+    constexpr int kStages = stages_for(kRU);
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int W = blockDim.x >> 5;
+    const StreamLayout L = stream_layout(a.K, W, kRU);
+    const int K = a.K, nch = L.nch;
+    const int nsl = (K + kKS - 1) / kKS;
+    const int G = K / kGroup;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t *limbs = smem + L.limb_off;
+    float *Xs = reinterpret_cast<float *>(smem + L.X_off);
+    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
+    uint8_t *ring = smem + L.ring_off + (size_t)warp * kStages * kSlotBytes;
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kStages * 8);
+
+    const long long gw = (long long)blockIdx.x * W + warp;
+    const long long nw = (long long)gridDim.x * W;
+    const int u0 = (int)(gw * units / nw);
+    const int u1 = (int)((gw + 1) * units / nw);
+    const int steps = (u1 - u0) * nsl;
+
+    // copy role of this lane: array (lane % 3: codes, scales, biases) of unit row lane / 3
+    const int my_r = lane / 3, my_a = lane % 3;
+    const bool copier = lane < 3 * kRU;
+    const uint8_t *gbase = my_a == 0 ? a.wq
+                         : (my_a == 1 ? reinterpret_cast<const uint8_t *>(a.scales)
+                                      : reinterpret_cast<const uint8_t *>(a.biases));
+    const size_t grow = my_a == 0 ? (size_t)K / 2 : (size_t)G * 2;       // bytes per matrix row
+    const int kshift = my_a == 0 ? 1 : 5;                                // bytes of a K range = len >> kshift
+    const uint32_t doff = my_a == 0 ? my_r * kSlotQ
+                        : (my_a == 1 ? kRU * kSlotQ + my_r * kSlotS : kRU * kSlotQ + kRU * kSlotS + my_r * kSlotS);
+    const int len_last = K - (nsl - 1) * kKS;                            // K of the last slice
+    const uint32_t piece_full = (uint32_t)kKS >> kshift, piece_last = (uint32_t)len_last >> kshift;
+    constexpr uint32_t kTxFull = kKS / 2 + kKS / 16;                     // bytes of one unit row, full slice
+    const uint32_t tx_last = (uint32_t)(len_last / 2 + len_last / 16);
+    constexpr int kCols = kRU / 2 > 0 ? kRU / 2 : 1;   // output columns of a GLU unit
+    auto unit_row = [&](int u, int r) {   // whole-matrix row of unit row r, -1 past the end
+        const int col = a.glu ? u * kCols + (r >> 1) : u * kRU + r;
+        return col < a.seg.ncols ? seg_row(a.seg, col, a.glu, a.glu ? (r & 1) : 0) : -1;
+    };
+    // rows of a unit that exist (the last unit of a launch may be short)
+    auto unit_live_rows = [&](int u) {
+        const int cols_left = a.seg.ncols - (a.glu ? u * kCols : u * kRU);
+        return a.glu ? 2 * min(kCols, cols_left) : min(kRU, cols_left);
+    };
+    // issue state: unit iu, slice ij go out next, into ring slot islot; csrc is
+    // this lane's matrix row of unit iu (null: nothing to copy)
+    int iu = u0, ij = 0, islot = 0, issued = 0, live = 0;
+    const uint8_t *csrc = nullptr;
+    auto set_issue_unit = [&](int uu) {
+        const int row = copier ? unit_row(uu, my_r) : -1;
+        csrc = row >= 0 ? gbase + (size_t)row * grow : nullptr;
+        live = unit_live_rows(uu);
+    };
+    if (u0 < u1) set_issue_unit(u0);
+    bool failed = false;
+    auto issue_next = [&]() {
+        const bool last = ij == nsl - 1;
+        const uint32_t bar = bar0 + 8 * islot;
+        if (lane == 0) mbar_expect_tx(bar, (uint32_t)live * (last ? tx_last : kTxFull));
+        __syncwarp();
+        if (csrc != nullptr)
+            bulk_g2s(ring_s + islot * kSlotBytes + doff, csrc + (size_t)ij * piece_full, last ? piece_last : piece_full, bar);
+        islot = islot + 1 == kStages ? 0 : islot + 1;
+        ++issued;
+        if (++ij == nsl) {
+            ij = 0;
+            if (++iu < u1) set_issue_unit(iu);
+        }
+    };
+
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    // Wide units send only their first slot's copies before the limb preparation:
+    // with every warp queueing its whole ring at once the copy queue fills and the
+    // issuing lanes wait, which would hold the preparation back; the rest follow
+    // it.  Narrow units, whose warps have few steps, queue their whole ring now.
+    constexpr int kPreStages = kRU >= 4 ? 1 : kStages;
+    while (issued < kPreStages && issued < steps) issue_next();
+
+    prep_limbs(a.x, K, nch, limbs, Xs, Ss, W, warp, lane);
+    __syncthreads();
+    while (issued < kStages && issued < steps) issue_next();
 
     float acc[kRU];
 #pragma unroll
     for (int r = 0; r < kRU; ++r) acc[r] = 0.0f;
     uint64_t best = 0;   // fused head: the largest argmax key of the rows this warp wrote
-    int u = u0, j = 0, slot = 0;
+    int slot = 0;
     uint32_t par = 0;
     const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
+    const int nc_last = (len_last + kChunk - 1) / kChunk;
 
-    for (int t = 0; t < steps; ++t) {
-        const bool ok = __all_sync(0xFFFFFFFFu, wait_slot(bar0 + 8 * slot, par, failed ? 64 : kSpinLimit));
-        failed = failed || !ok;
-        const uint8_t *sl = ring + slot * kSlotBytes;
-        const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
-        const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kRU * kSlotQ) + (lane >> 1);
-#pragma unroll
-        for (int cc = 0; cc < kKS / kChunk; ++cc) {
-            const int c = j * (kKS / kChunk) + cc;
-            if (c * kChunk + lane * 32 >= K) break;   // lanes past the end of a short last chunk
-            uint4 lm[6];
-#pragma unroll
-            for (int q = 0; q < 6; ++q) lm[q] = limb_l[(c * 6 + q) * 32];
-            const float X = Xs[c * 32 + lane];
-            const float scale = Ss[c * 32 + lane];
-#pragma unroll
-            for (int r = 0; r < kRU; ++r) {
-                const uint4 qv = ql[(r * kSlotQ + cc * (kChunk / 2)) / 16];
-                const float s = bf16_bits_to_f32(sc16[r * (kKS / kGroup) + cc * 16]);
-                const float b = bf16_bits_to_f32(sc16[kRU * (kKS / kGroup) + r * (kKS / kGroup) + cc * 16]);
-                const float P = lane_chunk_idot(qv, lm);
-                acc[r] = fmaf(s, P * scale, acc[r]);   // P * 2^(E-23): exact power-of-two scaling
-                acc[r] = fmaf(b, X, acc[r]);
+    for (int u = u0; u < u1; ++u) {
+        for (int j = 0; j < nsl; ++j) {
+            const bool ok = __all_sync(0xFFFFFFFFu, wait_slot(bar0 + 8 * slot, par, failed ? 64 : kSpinLimit));
+            failed = failed || !ok;
+            const uint8_t *sl = ring + slot * kSlotBytes;
+            if (j + 1 < nsl)
+                slot_dot<kRU>(acc, sl, limb_l, Xs, Ss, j * (kKS / kChunk), kKS / kChunk, kKS, lane);
+            else
+                slot_dot<kRU>(acc, sl, limb_l, Xs, Ss, j * (kKS / kChunk), nc_last, len_last, lane);
+            if (++slot == kStages) {
+                slot = 0;
+                par ^= 1u;
             }
+            __syncwarp();
+            if (issued < steps && !failed) issue_next();
         }
-        if (++j == nsl) {
-            float tot[kRU];
+        float tot[kRU];
 #pragma unroll
-            for (int r = 0; r < kRU; ++r) {
-                tot[r] = warp_sum_to_lane0(acc[r]);
-                acc[r] = 0.0f;
-            }
-            if (lane == 0) {
-                if (a.glu) {
+        for (int r = 0; r < kRU; ++r) {
+            tot[r] = warp_sum_to_lane0(acc[r]);
+            acc[r] = 0.0f;
+        }
+        if (lane == 0) {
+            if (a.glu) {
 #pragma unroll
-                    for (int p = 0; p < kRU / 2; ++p) {
-                        const int col = u * kCols + p;
-                        if (col < a.seg.ncols) {
-                            const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p]));
-                            const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1]));
-                            a.y[col] = failed ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(glu_f32(g, uu));
-                        }
+                for (int p = 0; p < kRU / 2; ++p) {
+                    const int col = u * kCols + p;
+                    if (col < a.seg.ncols) {
+                        const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p]));
+                        const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1]));
+                        a.y[col] = failed ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(glu_f32(g, uu));
                     }
-                } else {
+                }
+            } else {
 #pragma unroll
-                    for (int r = 0; r < kRU; ++r) {
-                        const int col = u * kRU + r;
-                        if (col < a.seg.ncols) {
-                            const uint16_t h = failed ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(tot[r]);
-                            a.y[col] = h;
-                            if (a.cand) best = umax64(best, cand_key(h, a.id_base + (uint32_t)col));
-                        }
+                for (int r = 0; r < kRU; ++r) {
+                    const int col = u * kRU + r;
+                    if (col < a.seg.ncols) {
+                        const uint16_t h = failed ? (uint16_t)TF_NAN_BF16 : f32_to_bf16_rne(tot[r]);
+                        a.y[col] = h;
+                        if (a.cand) best = umax64(best, cand_key(h, a.id_base + (uint32_t)col));
                     }
                 }
             }
-            j = 0;
-            ++u;
         }
-        if (++slot == kStages) {
-            slot = 0;
-            par ^= 1u;
-        }
-        __syncwarp();
-        if (it_ < steps && !failed) issue_next();
     }
     // every issued slot was waited on above unless a wait gave up; then give the
     // outstanding copies a bounded chance to land before shared memory is released
     if (failed) {
         for (int s2 = 0; s2 < kStages; ++s2) wait_slot(bar0 + 8 * s2, 0, 1024);
     }
-    if (a.cand) {
-        // fused head: publish this warp's best key; the last CTA to finish reduces all
-        // of them into the argmax word (fence, then a ticket: the usual last-block pattern)
-        if (lane == 0) a.cand[gw] = best;
-        __threadfence();
-        __syncthreads();
-        __shared__ unsigned int ticket;
-        if (tid == 0) ticket = atomicAdd(a.done, 1u);
-        __syncthreads();
-        if (ticket == gridDim.x - 1) {
-            __threadfence();
-            const int ncand = (int)(gridDim.x * W);
-            uint64_t v = 0;
-            for (int i = tid; i < ncand; i += blockDim.x) v = umax64(v, ((volatile uint64_t *)a.cand)[i]);
-            v = warp_max64(v);
-            __shared__ uint64_t red[32];
-            if (lane == 0) red[warp] = v;
-            __syncthreads();
-            if (warp == 0) {
-                v = lane < W ? red[lane] : 0ull;
-                v = warp_max64(v);
-                if (lane == 0) {
-                    *a.word = word_of_key(v, a.y, a.id_base);
-                    *a.done = 0u;
+    if (a.cand) fused_head_tail(a, best, W, tid, warp, lane);
+}
+
+// ---------------------------------------------------------- tile ring --
+// The wide M = 1 kernel.  A per-warp ring refilled by one 1-D bulk copy per row
+// and array spends ~15 issue slots on every copy instruction, a tenth of all the
+// kernel issues at 12 copies per 4-row step, and keeps only half of its shared
+// memory in flight.  Here sixteen compute warps form four groups of four; each
+// group owns a ring of slots of one tile (16 matrix rows, or 8 GLU columns' gate and
+// up rows) by one chunk of K, and a producer warp of its own fills a slot with one
+// 2-D tensor copy per array (codes, scales, biases), so three copy instructions
+// move 9 KB, and no compute warp ever waits to refill a slot.  The group's four warps take four rows each from every slot, exactly as the
+// per-warp kernel takes a unit's rows (the per-lane arithmetic, its order and the
+// shuffle tree are the same code, so both kernels give the same bits), and each
+// warp frees a slot by one arrival on the slot's empty barrier.  Tiles are
+// claimed in order from the CTA's share by a counter in shared memory, so the
+// groups stay busy to the end of the share.
+constexpr int kTRows = 16;                                   // rows of a tile
+constexpr int kTGroups = 4, kTGroupWarps = 4, kTWarps = kTGroups * kTGroupWarps;   // compute warps
+constexpr int kTThreads = (kTWarps + kTGroups) * 32;          // and one producer warp per group
+constexpr int kTSlotQ = kChunk / 2;                          // code bytes of one row in a slot
+constexpr int kTSlotS = kChunk / 32;                         // scale (or bias) bytes of one row
+constexpr int kTSlotBytes = kTRows * (kTSlotQ + 2 * kTSlotS);   // 9,216
+constexpr int kTMaxStages = 6;
+
+struct TileLayout {
+    int nch, stages;
+    size_t limb_off, X_off, scale_off, full_off, empty_off, hdr_off, ctl_off, ring_off, total;
+};
+
+__host__ __device__ inline TileLayout tile_layout(int K, int stages) {
+    TileLayout L;
+    L.nch = (K + kChunk - 1) / kChunk;
+    L.stages = stages;
+    L.limb_off = 0;
+    L.X_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
+    L.scale_off = round_up(L.X_off + (size_t)L.nch * 32 * 4, 128);
+    L.full_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
+    L.empty_off = L.full_off + (size_t)kTGroups * stages * 8;
+    L.hdr_off = L.empty_off + (size_t)kTGroups * stages * 8;    // (tile, chunk) of each slot
+    L.ctl_off = L.hdr_off + (size_t)kTGroups * stages * 8;      // claim counter, abort flag
+    L.ring_off = round_up(L.ctl_off + 16, 128);
+    L.total = L.ring_off + (size_t)kTGroups * stages * kTSlotBytes;
+    return L;
+}
+
+// Tiles of a call: segment s (TF_EPI_NONE) owns tiles [tstart[s], tstart[s + 1]),
+// tile i of it rows row0[s] + 16 i ...; a GLU call has one run of tiles over its
+// columns, 8 columns a tile.
+struct TilePlan {
+    int tstart[TF_MAX_SEGS + 1];
+    int ntiles;
+};
+
+__device__ __forceinline__ bool tile_wait(uint32_t bar, uint32_t parity, const volatile int *abort, long long limit) {
+    for (long long it = 0; it < limit; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255) == 255 && *abort) return false;
+    }
+    return false;
+}
+
+// Slot row of a warp's unit row r: rows 4w .. 4w+3 (NONE); for GLU the gate rows
+// sit in slot rows 0..7 and the up rows in 8..15, and unit row r is member r & 1
+// of column 2w + (r >> 1), the order the GLU epilogue reads.
+template <bool kGlu>
+__device__ __forceinline__ int tile_row(int w, int r) {
+    return kGlu ? (r & 1) * 8 + 2 * w + (r >> 1) : 4 * w + r;
+}
+
+template <bool kGlu>
+__global__ void __launch_bounds__(kTThreads, 1)
+    qmm_m1_tile_kernel(QmmArgs a, TilePlan plan, const __grid_constant__ CUtensorMap qmap,
+                       const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap bmap, int S) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const TileLayout L = tile_layout(a.K, S);
+    const int K = a.K, nch = L.nch;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool producer = warp >= kTWarps;
+    const int grp = producer ? warp - kTWarps : warp / kTGroupWarps, w_in = warp % kTGroupWarps;
+    uint8_t *limbs = smem + L.limb_off;
+    float *Xs = reinterpret_cast<float *>(smem + L.X_off);
+    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
+    int2 *hdr = reinterpret_cast<int2 *>(smem + L.hdr_off) + grp * S;
+    int *claim = reinterpret_cast<int *>(smem + L.ctl_off);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.ctl_off) + 1;
+    uint8_t *ring = smem + L.ring_off + (size_t)grp * S * kTSlotBytes;
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t full0 = smem_addr(smem + L.full_off) + (uint32_t)(grp * S * 8);
+    const uint32_t empty0 = smem_addr(smem + L.empty_off) + (uint32_t)(grp * S * 8);
+
+    // this CTA's share of the tiles
+    const int t0 = (int)((long long)blockIdx.x * plan.ntiles / gridDim.x);
+    const int t1 = (int)((long long)(blockIdx.x + 1) * plan.ntiles / gridDim.x);
+
+    if (tid == 0) {
+        for (int i = 0; i < kTGroups * S; ++i) {
+            mbar_init(smem_addr(smem + L.full_off) + 8 * i, 1);
+            mbar_init(smem_addr(smem + L.empty_off) + 8 * i, kTGroupWarps);
+        }
+        claim[0] = 0;
+        claim[1] = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // first matrix row (both members for GLU) and first output column of tile t
+    auto tile_rows = [&](int t, int &r_a, int &r_b, int &col, int &ncol) {
+        if (kGlu) {
+            r_a = a.seg.row0[0] + 8 * t;
+            r_b = a.seg.row0[1] + 8 * t;
+            col = 8 * t;
+            ncol = min(8, a.seg.ncols - col);
+        } else {
+            // the last segment starting at or before t (selected without a
+            // dynamic index into the parameter arrays)
+            int ts = plan.tstart[0], row0 = a.seg.row0[0], col0 = a.seg.col0[0], nr = a.seg.nrows[0];
+#pragma unroll
+            for (int s2 = 1; s2 < TF_MAX_SEGS; ++s2)
+                if (s2 < a.seg.nseg && t >= plan.tstart[s2]) {
+                    ts = plan.tstart[s2];
+                    row0 = a.seg.row0[s2];
+                    col0 = a.seg.col0[s2];
+                    nr = a.seg.nrows[s2];
+                }
+            const int i = t - ts;
+            r_a = row0 + kTRows * i;
+            r_b = 0;
+            col = col0 + kTRows * i;
+            ncol = min(kTRows, nr - kTRows * i);
+        }
+    };
+
+    // issue state of the group's producer (lane 0): the tile being sent (-1: none
+    // left), its next chunk, the slot and its use count
+    int it_tile = -2, it_c = nch, islot = 0, iuse = 0, nissued = 0;
+    bool done_issuing = false;
+    auto issue_next = [&]() {   // lane 0 of the producer warp only
+        if (done_issuing) return;
+        if (it_c == nch) {
+            const int t = t0 + atomicAdd(claim, 1);
+            it_tile = t < t1 ? t : -1;
+            it_c = 0;
+        }
+        const uint32_t full = full0 + 8 * islot, empty = empty0 + 8 * islot;
+        if (iuse > 0 && !tile_wait(empty, (uint32_t)((iuse - 1) & 1), abort_flag, kSpinLimit)) {
+            *abort_flag = 1;
+            done_issuing = true;
+            return;
+        }
+        hdr[islot] = make_int2(it_tile, it_c);
+        if (it_tile >= 0) {
+            int r_a, r_b, col, ncol;
+            tile_rows(it_tile, r_a, r_b, col, ncol);
+            mbar_expect_tx(full, (uint32_t)kTSlotBytes);
+            const uint32_t dst = ring_s + islot * kTSlotBytes;
+            constexpr uint32_t kS0 = kTRows * kTSlotQ, kB0 = kS0 + kTRows * kTSlotS;
+            const int cq = it_c * (kChunk / 8), cs = it_c * (kChunk / 64);   // 4-byte code words, bf16 groups
+            tma_load_2d(dst, &qmap, cq, r_a, full);
+            tma_load_2d(dst + kS0, &smap, cs, r_a, full);
+            tma_load_2d(dst + kB0, &bmap, cs, r_a, full);
+            if (kGlu) {
+                tma_load_2d(dst + 8 * kTSlotQ, &qmap, cq, r_b, full);
+                tma_load_2d(dst + kS0 + 8 * kTSlotS, &smap, cs, r_b, full);
+                tma_load_2d(dst + kB0 + 8 * kTSlotS, &bmap, cs, r_b, full);
+            }
+            ++it_c;
+        } else {
+            mbar_arrive(full);   // the end marker: no copies, the phase completes at once
+            done_issuing = true;
+        }
+        ++nissued;
+        if (++islot == S) {
+            islot = 0;
+            ++iuse;
+        }
+    };
+
+    // the whole ring goes out before the limb preparation (one tile-chunk a slot);
+    // all warps prepare the limbs, then the producers keep the rings full
+    if (producer && lane == 0)
+        for (int i = 0; i < S; ++i) issue_next();
+    __syncwarp();
+    prep_limbs(a.x, K, nch, limbs, Xs, Ss, kTWarps + kTGroups, warp, lane);
+    __syncthreads();
+    if (producer) {
+        if (lane == 0)
+            while (!done_issuing) issue_next();
+        __syncwarp();
+    }
+
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint64_t best = 0;
+    int slot = 0;
+    uint32_t par = 0;
+    const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
+    bool failed = false;
+    for (; !producer;) {
+        const bool ok = __all_sync(0xFFFFFFFFu, tile_wait(full0 + 8 * slot, par, abort_flag, kSpinLimit));
+        if (!ok) {
+            failed = true;
+            break;
+        }
+        const int2 h = hdr[slot];
+        if (h.x < 0) break;
+        const int c = h.y;
+        const uint8_t *sl = ring + slot * kTSlotBytes;
+        if (lane * 32 < K - c * kChunk) {   // lanes past the end of a short last chunk add nothing
+            uint4 lm[6];
+#pragma unroll
+            for (int q = 0; q < 6; ++q) lm[q] = limb_l[(c * 6 + q) * 32];
+            const float X = Xs[c * 32 + lane];
+            const float scale = Ss[c * 32 + lane];
+            const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
+            const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kTRows * kTSlotQ) + (lane >> 1);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int R = tile_row<kGlu>(w_in, r);
+                const uint4 qv = ql[R * (kTSlotQ / 16)];
+                const float s = bf16_bits_to_f32(sc16[R * (kTSlotS / 2)]);
+                const float b = bf16_bits_to_f32(sc16[kTRows * (kTSlotS / 2) + R * (kTSlotS / 2)]);
+                const float P = lane_chunk_idot(qv, lm);
+                acc[r] = fmaf(s, P * scale, acc[r]);   // P * 2^(E-23): exact power-of-two scaling
+                acc[r] = fmaf(b, X, acc[r]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * slot);
+        if (++slot == S) {
+            slot = 0;
+            par ^= 1u;
+        }
+        if (c == nch - 1) {
+            float tot[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                tot[r] = warp_sum_to_lane0(acc[r]);
+                acc[r] = 0.0f;
+            }
+            if (lane == 0) {
+                int r_a, r_b, col, ncol;
+                tile_rows(h.x, r_a, r_b, col, ncol);
+                if (kGlu) {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        if (2 * w_in + p < ncol) {
+                            const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p]));
+                            const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1]));
+                            a.y[col + 2 * w_in + p] = f32_to_bf16_rne(glu_f32(g, uu));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        if (4 * w_in + r < ncol) {
+                            const uint16_t hv = f32_to_bf16_rne(tot[r]);
+                            a.y[col + 4 * w_in + r] = hv;
+                            if (a.cand) best = umax64(best, cand_key(hv, a.id_base + (uint32_t)(col + 4 * w_in + r)));
+                        }
+                    }
                 }
             }
         }
     }
+    if (failed && lane == 0) *abort_flag = 1;
+    __syncthreads();
+    if (*abort_flag) {
+        // a wait gave up: the CTA's whole share of outputs becomes NaN, and the
+        // copies still in flight get a bounded chance to land before exit
+        for (int t = t0; t < t1; ++t) {
+            int r_a, r_b, col, ncol;
+            tile_rows(t, r_a, r_b, col, ncol);
+            for (int i = tid; i < ncol; i += blockDim.x) a.y[col + i] = (uint16_t)TF_NAN_BF16;
+        }
+        if (producer && lane == 0)
+            for (int s2 = 0; s2 < S && s2 < nissued; ++s2) {
+                const int uses = (nissued - 1 - s2) / S + 1;
+                wait_slot(full0 + 8 * s2, (uint32_t)((uses - 1) & 1), 1024);
+            }
+        best = cand_key((uint16_t)TF_NAN_BF16, 0u);
+    }
+    if (a.cand) fused_head_tail(a, best, kTWarps + kTGroups, tid, warp, lane);
 }
 
 // The widest warp count whose shared memory fits 227 KB with 1 KB left for the
@@ -368,7 +678,8 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         g_stream_smem_set[dev][ri] = 226 * 1024;
     }
-    const int units = a.glu ? (a.seg.ncols + RU / 2 - 1) / (RU / 2) : (a.seg.ncols + RU - 1) / RU;
+    constexpr int kCols = RU / 2 > 0 ? RU / 2 : 1;   // output columns of a GLU unit
+    const int units = a.glu ? (a.seg.ncols + kCols - 1) / kCols : (a.seg.ncols + RU - 1) / RU;
     int blocks = num_sms();
     const int need = (units + W - 1) / W;
     if (need < blocks) blocks = need;
@@ -376,10 +687,89 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-// Rows per unit only change how often a lane reuses its activation limbs, never a
-// row's arithmetic, so the choice may follow N: four rows while every warp of the
-// grid still gets two units, fewer when the slice is narrow.
+// ---------------------------------------------------------- tile ring host --
+static int tile_stages(int K) {
+    for (int st = kTMaxStages; st >= 2; --st)
+        if (tile_layout(K, st).total <= 226 * 1024) return st;
+    return 0;
+}
+
+static TilePlan tile_plan(const QmmArgs &a) {
+    TilePlan plan{};
+    if (a.glu) {
+        plan.ntiles = (a.seg.ncols + 7) / 8;
+        for (int s = 1; s <= TF_MAX_SEGS; ++s) plan.tstart[s] = plan.ntiles;
+    } else {
+        int n = 0;
+        for (int s = 0; s < a.seg.nseg; ++s) {
+            plan.tstart[s] = n;
+            n += (a.seg.nrows[s] + kTRows - 1) / kTRows;
+        }
+        for (int s = a.seg.nseg; s <= TF_MAX_SEGS; ++s) plan.tstart[s] = n;
+        plan.ntiles = n;
+    }
+    return plan;
+}
+
+// The tile ring takes the call when it has at least four tiles per SM (fewer
+// leave groups idle, and the per-warp kernel's finer units balance better), the
+// driver offers the tensor-map encoder and two slots per group fit beside the limbs.
+static bool tile_ring_fits(const QmmArgs &a) {
+    if (!encode_tiled_fn() || tile_stages(a.K) < 2) return false;
+    return tile_plan(a).ntiles >= 4 * num_sms();
+}
+
+static bool g_tile_smem_set[64][2];
+
+template <bool kGlu>
+static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream) {
+    const int S = tile_stages(a.K);
+    const TileLayout L = tile_layout(a.K, S);
+    const TilePlan plan = tile_plan(a);
+    auto enc = encode_tiled_fn();
+    const cuuint32_t box_rows = kGlu ? 8u : (cuuint32_t)kTRows;
+    const cuuint32_t estr[2] = {1, 1};
+    CUtensorMap qmap, smap, bmap;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(a.K / 8), (cuuint64_t)a.n_whole};
+        const cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
+        const cuuint32_t box[2] = {(cuuint32_t)(kChunk / 8), box_rows};
+        if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(a.wq), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const int G = a.K / kGroup;
+        const cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)a.n_whole};
+        const cuuint64_t strides[1] = {(cuuint64_t)G * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)(kChunk / kGroup), box_rows};
+        if (enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(a.scales), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+            enc(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(a.biases), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!g_tile_smem_set[dev][kGlu ? 1 : 0]) {
+        cudaError_t e = cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+        if (e != cudaSuccess) return e;
+        g_tile_smem_set[dev][kGlu ? 1 : 0] = true;
+    }
+    const int blocks = plan.ntiles < num_sms() ? plan.ntiles : num_sms();
+    qmm_m1_tile_kernel<kGlu><<<blocks, kTThreads, L.total, stream>>>(a, plan, qmap, smap, bmap, S);
+    return cudaGetLastError();
+}
+
+// Wide calls take the tile ring.  Otherwise rows per unit only change how often a
+// lane reuses its activation limbs, never a row's arithmetic, so the choice may
+// follow N: four rows while every warp of the grid still gets two units, fewer
+// when the slice is narrow.
 cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream) {
+    if (tile_ring_fits(a)) return a.glu ? launch_tile<true>(a, stream) : launch_tile<false>(a, stream);
     const long long warps = (long long)num_sms() * stream_warps(a.K, 4);
     const long long rows = a.glu ? 2ll * a.seg.ncols : a.seg.ncols;
     if (rows >= 8 * warps) return launch_ru<4>(a, 0, stream);

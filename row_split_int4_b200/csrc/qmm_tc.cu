@@ -52,6 +52,7 @@
 #include <cstring>
 
 #include "qmm_common.cuh"
+#include "tmap.h"
 
 namespace tf {
 
@@ -642,15 +643,18 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
 // ------------------------------------------------------------------ host --
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-static cudaError_t get_encode() {
-    if (g_encode) return cudaSuccess;
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
+    if (g_encode) return g_encode;
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return nullptr;
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    return cudaSuccess;
+    return g_encode;
 }
+
+static cudaError_t get_encode() { return encode_tiled_fn() ? cudaSuccess : cudaErrorNotSupported; }
 
 // K slices per tile: from K and the whole matrix's row count alone.  The whole
 // matrix should give about 512 CTAs; a slice keeps at least four periods of

@@ -1,5 +1,6 @@
 // stream_common.cuh -- the PTX pieces of the streaming (M = 1) kernels: mbarriers,
-// the 1-D bulk copy into shared memory, a bounded wait, and dp4a.
+// the 1-D bulk copy and the 2-D tensor copy into shared memory, a bounded wait,
+// and dp4a.
 #pragma once
 
 #include "tf_common.cuh"
@@ -23,6 +24,17 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// a 2-D tile of a tensor map into this CTA's shared memory, completion counted on
+// `bar` (no multicast); c0 is the inner coordinate in elements
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
