@@ -112,7 +112,7 @@ def step_bytes():
 def traffic_from_profiles(kernel_src):
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
     only while the kernel's source is the one the counters were taken on."""
-    path = os.path.join(ROOT, "profiles", "qmm_m1_stream_lm_head_half.md")
+    path = os.path.join(ROOT, "profiles", "qmm_m1_tile_lm_head_half.md")
     try:
         txt = open(path).read()
     except OSError:
@@ -610,7 +610,7 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "one GPU, two row halves"},
             "lm_head_argmax_us_per_token": round(statistics.fmean(head_ms) * 1e3, 2),
             "tokens_per_s_equiv": round(1e3 / ms_step, 1),
-            "roofline": {"bound": "hbm", "kernel": "qmm_m1_stream_kernel (lm_head half, 124,160 x 5,120)",
+            "roofline": {"bound": "hbm", "kernel": "qmm_m1_tile_kernel (lm_head half, 124,160 x 5,120)",
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic_from_profiles(src),
                          "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_avg_ms * 1e3, 3)},
