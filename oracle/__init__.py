@@ -35,6 +35,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 FLAG = 0x80000000
 SENTINEL = 0xFFFFFFFF
 NAN_BF16 = 0x7FC0
+TOP2_NONE = (0x7FFFFFFF << 32) | 0xFF800000   # "no second place" (a slice of one element)
 GROUP = 64
 
 # What pins each oracle function to something other than itself (tests that
@@ -49,6 +50,8 @@ PINS = {
     "pick": "exhaustive flag x flag x {<,=,>} truth table; split-then-pick == whole on every split point",
     "half_rows": "the pages' spans 2,560/8,704/124,160 of 5,120/17,408/248,320",
     "top2_gap": "hand cases (ties give 0, n=1 gives inf)",
+    "top2_rows": "hand cases (a tie keeps both ids, +-0 tie, one element has no second, NaN flags both); a numpy lexsort of every small row",
+    "top2_merge": "merge of the slices' top two == top two of the whole row at every split point; the lowest flagged part wins",
     "qmm8_rows": "one-hot x; constant-code closed form; numpy float64 matmul; the sign of the codes",
     "residual_add": "exact sums bf16 cannot hold; the fp32 round-to-even tie; IEEE specials; numpy float32 addition",
     "embed_rows": "brute-force row lookup; bound refusals incl. the pages' 124,160-of-248,320 shard width; NaN rows past the bound",
@@ -106,6 +109,10 @@ class Oracle:
         L.orc_argmax_rows.argtypes = [_P, _I32, _I64, _I64, ctypes.c_uint32, _P]
         L.orc_pick.restype = None
         L.orc_pick.argtypes = [_P, _I32, _I32, _P]
+        L.orc_top2_rows.restype = _I32
+        L.orc_top2_rows.argtypes = [_P, _I32, _I64, _I64, ctypes.c_uint32, _P]
+        L.orc_top2_merge.restype = None
+        L.orc_top2_merge.argtypes = [_P, _I32, _I32, _P]
         L.orc_top2_gap.restype = None
         L.orc_top2_gap.argtypes = [_P, _I32, _I64, _P]
         L.orc_qmm8_rows.restype = _I32
@@ -255,6 +262,28 @@ class Oracle:
         ids = np.empty(M, dtype=np.uint32)
         self.L.orc_pick(_ptr(w), nparts, M, _ptr(ids))
         return ids
+
+    def top2_rows(self, v: np.ndarray, id_base: int = 0) -> np.ndarray:
+        """bf16 bits [M, n] -> uint64 words [M, 2]: the winner and the second place
+        in the argmax order (oracle.c, merged top two)."""
+        v = np.ascontiguousarray(v, dtype=np.uint16)
+        if v.ndim == 1:
+            v = v[None, :]
+        M, n = v.shape
+        words2 = np.empty((M, 2), dtype=np.uint64)
+        if self.L.orc_top2_rows(_ptr(v), M, n, n, int(id_base), _ptr(words2)) != 0:
+            raise ValueError("orc_top2_rows: n must be >= 1")
+        return words2
+
+    def top2_merge(self, words2: np.ndarray) -> np.ndarray:
+        """uint64 [nparts, M, 2] -> uint64 [M, 2]: the merged top two."""
+        w = np.ascontiguousarray(words2, dtype=np.uint64)
+        if w.ndim == 2:
+            w = w[None]
+        nparts, M, _ = w.shape
+        out = np.empty((M, 2), dtype=np.uint64)
+        self.L.orc_top2_merge(_ptr(w), nparts, M, _ptr(out))
+        return out
 
     def top2_gap(self, logits64: np.ndarray) -> np.ndarray:
         a = np.ascontiguousarray(logits64, dtype=np.float64)

@@ -61,6 +61,8 @@
  *  10 the residual add rounds the sum to bf16 instead of fp32
  *  11 the embedding gather checks ids against half of the bound (the shard's width)
  *  12 the int8 head reads its codes as unsigned bytes
+ *  13 the top two's second place skips values equal to the winner's (a tie reads as no tie)
+ *  14 the top-two merge takes the second place from the winning part only
  */
 #include <math.h>
 #include <stddef.h>
@@ -470,6 +472,127 @@ void orc_pick(const uint64_t *words, int nparts, int M, uint32_t *ids)
             }
         }
         ids[m] = best_id;
+    }
+}
+
+/* ------------------------------------------------------- merged top two -- */
+
+/* The session keeps the merged top two of the head for its cross-block tie test
+ * (TensorFold PR #1433, step-1 and step-2 bodies: session.zig keeps the merged
+ * top two and reads the pick's sentinel as a failure).  Reading: for each row,
+ * the two highest entries in the argmax's own order -- the larger value first,
+ * the lower id among equal values, +0 equal to -0 -- as two argmax words:
+ * words2[2m] the winner (orc_argmax_rows' word) and words2[2m+1] the best of the
+ * other ids.  A row holding any NaN, +Inf or -Inf is flagged: both words are the
+ * argmax's flagged word.  A slice of one element has no second place: the word
+ * ORC_TOP2_NONE (id 0x7FFFFFFF with the bits of -Inf, a value no unflagged
+ * word carries).  Returns -1 for n < 1. */
+#define ORC_TOP2_NONE ((((uint64_t)0x7FFFFFFFu) << 32) | 0xFF800000u)
+
+static uint64_t orc_word_of(const uint16_t *r, int64_t j, uint32_t id_base)
+{
+    return ((uint64_t)(id_base + (uint32_t)j) << 32) | ((uint32_t)r[j] << 16);
+}
+
+int orc_top2_rows(const uint16_t *v, int M, int64_t n, int64_t ld, uint32_t id_base, uint64_t *words2)
+{
+    if (n < 1 || M < 0 || ld < n)
+        return -1;
+    for (int m = 0; m < M; ++m) {
+        const uint16_t *r = v + (int64_t)m * ld;
+        int flagged = 0;
+        int64_t first_nf = 0, best = -1, second = -1;
+        double bestv = 0.0, secondv = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            double x = orc_bf16_to_f64(r[j]);
+            if (!isfinite(x)) {
+                if (!flagged) {
+                    flagged = 1;
+                    first_nf = j;
+                }
+                continue;
+            }
+            /* strict comparisons: among equal values the earlier (lower) id keeps its place */
+            if (best < 0 || x > bestv) {
+                second = best;
+                secondv = bestv;
+                best = j;
+                bestv = x;
+#if ORC_PLANT == 13
+            } else if (x < bestv && (second < 0 || x > secondv)) {
+#else
+            } else if (second < 0 || x > secondv) {
+#endif
+                second = j;
+                secondv = x;
+            }
+        }
+        uint64_t *o = words2 + 2 * (int64_t)m;
+        if (flagged) {
+            uint32_t idw = ORC_FLAG | (id_base + (uint32_t)first_nf);
+            o[0] = o[1] = ((uint64_t)idw << 32) | 0x7FC00000u;
+        } else {
+            o[0] = orc_word_of(r, best, id_base);
+            o[1] = second < 0 ? ORC_TOP2_NONE : orc_word_of(r, second, id_base);
+        }
+    }
+    return 0;
+}
+
+/* a ahead of b in the argmax order (NONE is behind everything) */
+static int orc_word_ahead(uint64_t a, uint64_t b)
+{
+    if (a == ORC_TOP2_NONE)
+        return 0;
+    if (b == ORC_TOP2_NONE)
+        return 1;
+    double va = orc_word_value(a), vb = orc_word_value(b);
+    return va > vb || (va == vb && (uint32_t)(a >> 32) < (uint32_t)(b >> 32));
+}
+
+/* words2 is [nparts][M][2] as orc_top2_rows writes it for slices of one
+ * vocabulary.  For each row: if any part is flagged, both merged words are the
+ * flagged word of the lowest such part (the pick fails closed on it); otherwise
+ * the two highest of all the parts' words in the argmax order. */
+void orc_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out2)
+{
+    for (int m = 0; m < M; ++m) {
+        uint64_t *o = out2 + 2 * (int64_t)m;
+        int done = 0;
+        for (int p = 0; p < nparts && !done; ++p) {
+            uint64_t w = words2[((int64_t)p * M + m) * 2];
+            if ((uint32_t)(w >> 32) & ORC_FLAG) {
+                o[0] = o[1] = w;
+                done = 1;
+            }
+        }
+        if (done)
+            continue;
+        uint64_t best = ORC_TOP2_NONE, second = ORC_TOP2_NONE;
+#if ORC_PLANT == 14
+        int best_part = -1;
+        for (int p = 0; p < nparts; ++p) {
+            uint64_t w = words2[((int64_t)p * M + m) * 2];
+            if (orc_word_ahead(w, best)) {
+                best = w;
+                best_part = p;
+            }
+        }
+        second = words2[((int64_t)best_part * M + m) * 2 + 1];
+#else
+        for (int p = 0; p < nparts; ++p)
+            for (int i = 0; i < 2; ++i) {
+                uint64_t w = words2[((int64_t)p * M + m) * 2 + i];
+                if (orc_word_ahead(w, best)) {
+                    second = best;
+                    best = w;
+                } else if (orc_word_ahead(w, second)) {
+                    second = w;
+                }
+            }
+#endif
+        o[0] = best;
+        o[1] = second;
     }
 }
 

@@ -371,6 +371,74 @@ def check_top2_gap(o):
     assert o.top2_gap(np.array([[2.0]]))[0] == math.inf
 
 
+TOP2_NONE = (0x7FFFFFFF << 32) | 0xFF800000
+
+
+def ref_top2(vals, base):
+    """Reference top two by an independent route: sort the ids by (-value, id)."""
+    fv = [bf16_val(int(b)) for b in vals]
+    nf = [j for j, v in enumerate(fv) if not math.isfinite(v)]
+    if nf:
+        w = ((0x80000000 | (base + nf[0])) << 32) | 0x7FC00000
+        return [w, w]
+    order = sorted(range(len(fv)), key=lambda i: (-fv[i], i))
+    words = [((base + j) << 32) | (int(vals[j]) << 16) for j in order[:2]]
+    return words + [TOP2_NONE] * (2 - len(words))
+
+
+def check_top2_hand(o):
+    """Hand-worked rows: an exact tie keeps both ids (lower first), +0 ties -0,
+    one element has no second place, and any non-finite value flags both words."""
+    def w(id_, v):
+        return (id_ << 32) | (bf16_of(v) << 16)
+    rows = [([1.0, 3.0, 2.5, 3.0], [w(1, 3.0), w(3, 3.0)]),
+            ([0.0, -1.0, 5.0, 4.0], [w(2, 5.0), w(3, 4.0)]),
+            ([2.0, 1.0, 1.0, -4.0], [w(0, 2.0), w(1, 1.0)])]
+    for vals, want in rows:
+        got = o.top2_rows(np.array([bf16_of(v) for v in vals], dtype=np.uint16))
+        assert [int(g) for g in got[0]] == want, (vals, [hex(int(g)) for g in got[0]])
+    got = o.top2_rows(np.array([0x8000, 0x0000], dtype=np.uint16), 100)[0]
+    assert [int(g) for g in got] == [(100 << 32) | 0x80000000, 101 << 32]
+    got = o.top2_rows(np.array([bf16_of(7.0)], dtype=np.uint16), 5)[0]
+    assert [int(g) for g in got] == [w(5, 7.0), TOP2_NONE]
+    got = o.top2_rows(np.array([bf16_of(1.0), 0x7FC0, bf16_of(2.0), 0x7F80], dtype=np.uint16), 10)[0]
+    flagged = ((0x80000000 | 11) << 32) | 0x7FC00000
+    assert [int(g) for g in got] == [flagged, flagged]
+
+
+def check_top2_bruteforce(o):
+    """Every 5-vector over {-1, -0, +0, 1, NaN, +Inf, -Inf} and random shorter rows
+    against the sort above; the winner equals the argmax word."""
+    vecs = np.array(list(itertools.product(ALPHABET, repeat=5)), dtype=np.uint16)
+    got = o.top2_rows(vecs, 3)
+    for i in range(0, len(vecs), 7):
+        assert [int(g) for g in got[i]] == ref_top2(vecs[i], 3), (vecs[i], [hex(int(g)) for g in got[i]])
+    assert np.array_equal(got[:, 0], o.argmax_rows(vecs, 3))
+    rng = np.random.default_rng(29)
+    vals = [bf16_of(v) for v in (-2.0, -1.0, -0.0, 0.0, 0.5, 1.0, 3.0)]
+    for n in (1, 2, 3, 4, 9):
+        rows = rng.choice(vals, size=(64, n)).astype(np.uint16)
+        got = o.top2_rows(rows, 40)
+        for i in range(64):
+            assert [int(g) for g in got[i]] == ref_top2(rows[i], 40), (rows[i], [hex(int(g)) for g in got[i]])
+
+
+def check_top2_merge_split(o):
+    """The merge of the slices' top two equals the top two of the whole row, at
+    every split into two parts and at every split into three."""
+    vecs = np.array(list(itertools.product(ALPHABET, repeat=5)), dtype=np.uint16)
+    whole = o.top2_rows(vecs, 0)
+    for cut in range(1, 5):
+        parts = np.stack([o.top2_rows(vecs[:, :cut], 0), o.top2_rows(vecs[:, cut:], cut)])
+        merged = o.top2_merge(parts)
+        bad = np.nonzero((merged != whole).any(axis=1))[0]
+        assert bad.size == 0, (cut, vecs[bad[0]], [hex(int(g)) for g in merged[bad[0]]])
+    for c1, c2 in ((1, 3), (2, 4), (1, 2)):
+        parts = np.stack([o.top2_rows(vecs[:, :c1], 0), o.top2_rows(vecs[:, c1:c2], c1),
+                          o.top2_rows(vecs[:, c2:], c2)])
+        assert np.array_equal(o.top2_merge(parts), whole), (c1, c2)
+
+
 def check_qmm8(o, seed=23):
     """The int8 head y = bf16(s * sum x q8): one-hot x (an exact product), a
     constant code (closed form s * q * sum x), numpy's float64 matmul, and the
@@ -468,4 +536,5 @@ ALL_CHECKS = [
     check_one_hot, check_zero_rows, check_constant_q, check_vs_numpy_matmul, check_rows_order_free,
     check_glu, check_spans, check_gather, check_split_equals_whole_mlp, check_argmax_bruteforce,
     check_pick_truth_table, check_split_pick_equals_whole, check_top2_gap, check_residual_add, check_embed_rows, check_qmm8,
+    check_top2_hand, check_top2_bruteforce, check_top2_merge_split,
 ]

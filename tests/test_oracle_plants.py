@@ -5,7 +5,9 @@ peer's half, a gather writing its own half twice, an argmax and a pick that
 tie to the higher id, an argmax that does not flag, a pick whose flag test is
 dropped) plus three for the arithmetic (bias dropped, nibbles swapped, GLU
 orientation swapped) and two for the adjacent steps (a residual add rounded to
-bf16, an embedding bound taken from the shard's width).  Only the oracle is ever broken; no broken kernel is
+bf16, an embedding bound taken from the shard's width) and two for the merged
+top two (a second place that skips ties, a merge that keeps the winning part's
+second).  Only the oracle is ever broken; no broken kernel is
 built or run."""
 import pytest
 
@@ -25,6 +27,8 @@ PLANTS = {
     10: [C.check_residual_add],
     11: [C.check_embed_rows],
     12: [C.check_qmm8],
+    13: [C.check_top2_hand, C.check_top2_bruteforce],
+    14: [C.check_top2_merge_split],
 }
 
 
