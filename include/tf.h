@@ -59,6 +59,9 @@ typedef enum {
 /* tf_pick's result for a flagged row; never a token id
  * (TensorFold PR #1433 step-2 body: the session reads maxInt(u32) as error.PairFailed). */
 #define TF_PICK_FAILED 0xFFFFFFFFu
+/* the second place of a one-element slice (tf_top2_rows): id 0x7FFFFFFF with the
+ * fp32 bits of -Inf, a value no unflagged word carries */
+#define TF_TOP2_NONE ((0x7FFFFFFFull << 32) | 0xFF800000ull)
 /* The bf16 NaN a missing gather part reads as (TensorFold PR #1433 step-1 body). */
 #define TF_NAN_BF16 0x7FC0u
 /* Rows one qmm call may carry: chunk(requested) = min(requested, 128)
@@ -275,6 +278,42 @@ tf_status tf_embed_rows(const void *table, int rows, int H, int ld_table, int bo
  * Errors: TF_E_ARG (before any launch), TF_E_CUDA.
  */
 tf_status tf_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, tf_stream stream);
+
+/*
+ * tf_top2_rows -- the top two of one slice of the vocabulary for each row (the
+ * merged top two of TensorFold PR #1433, step-1 and step-2 bodies: the session
+ * keeps the merged top two for its cross-block tie test, and reads the pick's
+ * sentinel as a failure).
+ *
+ * For each row m of logits[m][0..n), two words in tf_argmax_rows' format and
+ * order (larger value first, the lower id among equal values, +0 equal to -0):
+ *     words2[2m]     the winner -- the word tf_argmax_rows writes;
+ *     words2[2m + 1] the best of the other ids; an exact tie gives the same
+ *                    value with the next id; TF_TOP2_NONE when n == 1.
+ * A row holding any NaN, +Inf or -Inf gets its flagged argmax word twice.
+ *   logits, M, n, ld, id_base   as tf_argmax_rows (same limits and vector path).
+ *   words2  uint64 [M][2].
+ *   scratch device buffer of at least tf_top2_scratch_bytes(M, n) bytes, 8-byte
+ *           aligned, owned by the caller; contents on entry do not matter.
+ * Errors: TF_E_ARG, TF_E_RANGE, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+size_t tf_top2_scratch_bytes(int M, int n);
+tf_status tf_top2_rows(const void *logits, int M, int n, int ld, uint32_t id_base, uint64_t *words2, void *scratch,
+                       size_t scratch_bytes, tf_stream stream);
+
+/*
+ * tf_top2_merge -- the merged top two across slices (the same passage).
+ *
+ * words2 is uint64 [nparts][M][2] as tf_top2_rows writes it for slices of one
+ * vocabulary (part p, row m at (p*M + m)*2).  For each row: if any part's winner
+ * is flagged, both merged words are the flagged word of the lowest such part
+ * (tf_pick fails closed on the same rows); otherwise the two highest of all the
+ * parts' words in the argmax order.  The merged winner's id is tf_pick's id.
+ * 1 <= nparts <= TF_MAX_PARTS, 0 <= M <= 65535.
+ *   out2    uint64 [M][2] (not overlapping words2).
+ * Errors: TF_E_ARG, TF_E_ALIGN (before any launch), TF_E_CUDA.
+ */
+tf_status tf_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out2, tf_stream stream);
 
 /*
  * tf_argmax_rows_static -- tf_argmax_rows for callers that cannot allocate

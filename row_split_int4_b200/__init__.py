@@ -27,6 +27,7 @@ lib = ctypes.CDLL(LIB_PATH)
 TF_OK, TF_E_ARG, TF_E_RANGE, TF_E_ALIGN, TF_E_WINDOW, TF_E_BROKEN, TF_E_CUDA, TF_E_UNIMPL = range(8)
 TF_PAIR_FLAG = 0x80000000
 TF_PICK_FAILED = 0xFFFFFFFF
+TF_TOP2_NONE = (0x7FFFFFFF << 32) | 0xFF800000   # no second place (a one-element slice)
 TF_NAN_BF16 = 0x7FC0
 TF_BATCH_ROWS = 128
 TF_GROUP = 64
@@ -40,7 +41,7 @@ TF_EPI_NONE, TF_EPI_GLU = 0, 1
 EXPORTS = ["tf_qmm_rows", "tf_gather_rows", "tf_argmax_scratch_bytes", "tf_argmax_rows", "tf_pick",
            "tf_split_rows", "tf_member_segs", "tf_chunk_rows", "tf_seam_bytes", "tf_status_str", "tf_last_cuda_error",
            "tf_abi_version", "tf_argmax_rows_static", "tf_qmm_argmax_rows", "tf_qmm_argmax_scratch_bytes",
-           "tf_residual_add", "tf_embed_rows", "tf_qmm8_rows"]
+           "tf_residual_add", "tf_embed_rows", "tf_qmm8_rows", "tf_top2_scratch_bytes", "tf_top2_rows", "tf_top2_merge"]
 
 
 class tf_seg(ctypes.Structure):
@@ -56,6 +57,12 @@ lib.tf_argmax_scratch_bytes.restype = _sz
 lib.tf_argmax_scratch_bytes.argtypes = [_i, _i]
 lib.tf_argmax_rows.restype = _i
 lib.tf_argmax_rows.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _sz, _vp]
+lib.tf_top2_scratch_bytes.restype = _sz
+lib.tf_top2_scratch_bytes.argtypes = [_i, _i]
+lib.tf_top2_rows.restype = _i
+lib.tf_top2_rows.argtypes = [_vp, _i, _i, _i, ctypes.c_uint32, _vp, _vp, _sz, _vp]
+lib.tf_top2_merge.restype = _i
+lib.tf_top2_merge.argtypes = [_vp, _i, _i, _vp, _vp]
 lib.tf_qmm_argmax_scratch_bytes.restype = _sz
 lib.tf_qmm_argmax_scratch_bytes.argtypes = [_i, _i]
 lib.tf_qmm_argmax_rows.restype = _i
@@ -258,6 +265,33 @@ def tf_pick(words: torch.Tensor, ids: torch.Tensor, stream=None, check: bool = T
     nparts, M = words.shape
     st = lib.tf_pick(_ptr(words), nparts, M, _ptr(ids), _stream(stream))
     return _ret(st, "tf_pick", check)
+
+
+def tf_top2_scratch_bytes(M: int, n: int) -> int:
+    return lib.tf_top2_scratch_bytes(int(M), int(n))
+
+
+def tf_top2_rows(logits: torch.Tensor, id_base: int, words2: torch.Tensor, scratch: torch.Tensor,
+                 stream=None, check: bool = True) -> int:
+    """words2[M, 2] (int64 tensor holding u64 words) = per-row winner and second
+    place of logits[M, n] in the argmax order."""
+    assert logits.dtype == torch.bfloat16 and words2.dtype == torch.int64 and scratch.dtype == torch.uint8
+    assert words2.is_contiguous()
+    M, n = logits.shape
+    st = lib.tf_top2_rows(_ptr(logits), M, n, _ld(logits), int(id_base), _ptr(words2), _ptr(scratch),
+                          scratch.numel(), _stream(stream))
+    return _ret(st, "tf_top2_rows", check)
+
+
+def tf_top2_merge(words2: torch.Tensor, out2: torch.Tensor, stream=None, check: bool = True) -> int:
+    """out2[M, 2] = the merged top two of words2[nparts, M, 2]."""
+    assert words2.dtype == torch.int64 and out2.dtype == torch.int64
+    assert words2.is_contiguous() and out2.is_contiguous()
+    if words2.dim() == 2:
+        words2 = words2[None]
+    nparts, M, _ = words2.shape
+    st = lib.tf_top2_merge(_ptr(words2), nparts, M, _ptr(out2), _stream(stream))
+    return _ret(st, "tf_top2_merge", check)
 
 
 def tf_abi_version() -> int:

@@ -131,6 +131,157 @@ cudaError_t launch_argmax(ArgmaxArgs a, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------- top two --
+// The merged top two of the head (TensorFold PR #1433, step-1 and step-2
+// bodies: the session keeps the merged top two for its cross-block tie test).
+// Keys are the argmax's (flag, order-preserving value, inverted id), unique per
+// element, so a pair (k1 > k2) of the two largest keys is the top two; 0 is an
+// empty place.  Two pairs merge into max(a1, b1), max(min(a1, b1), a2, b2).
+__device__ __forceinline__ void top2_insert(uint64_t &k1, uint64_t &k2, uint64_t k) {
+    if (k > k1) {
+        k2 = k1;
+        k1 = k;
+    } else if (k > k2) {
+        k2 = k;
+    }
+}
+__device__ __forceinline__ void top2_merge_pair(uint64_t &k1, uint64_t &k2, uint64_t b1, uint64_t b2) {
+    const uint64_t lo = umin64(k1, b1);
+    k1 = umax64(k1, b1);
+    k2 = umax64(lo, umax64(k2, b2));
+}
+__device__ __forceinline__ void warp_top2(uint64_t &k1, uint64_t &k2) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t b1 = __shfl_xor_sync(0xFFFFFFFFu, k1, o);
+        const uint64_t b2 = __shfl_xor_sync(0xFFFFFFFFu, k2, o);
+        top2_merge_pair(k1, k2, b1, b2);
+    }
+}
+
+__global__ void __launch_bounds__(kArgmaxThreads) top2_partial_kernel(ArgmaxArgs a) {
+    const int m = blockIdx.y;
+    const int b = blockIdx.x;
+    const uint16_t *row = a.logits + (long long)m * a.ld;
+    const int j0 = b * a.span;
+    const int j1 = min(a.n, j0 + a.span);
+    uint64_t k1 = 0, k2 = 0;
+    if (a.vec) {
+        const int jv_end = j0 + ((j1 - j0) / 8) * 8;
+        for (int j = j0 + threadIdx.x * 8; j < jv_end; j += kArgmaxThreads * 8) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + j);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                top2_insert(k1, k2, cand_key(w[e] & 0xFFFFu, a.id_base + j + 2 * e));
+                top2_insert(k1, k2, cand_key(w[e] >> 16, a.id_base + j + 2 * e + 1));
+            }
+        }
+        for (int j = jv_end + threadIdx.x; j < j1; j += kArgmaxThreads) top2_insert(k1, k2, cand_key(row[j], a.id_base + j));
+    } else {
+        for (int j = j0 + threadIdx.x; j < j1; j += kArgmaxThreads) top2_insert(k1, k2, cand_key(row[j], a.id_base + j));
+    }
+    warp_top2(k1, k2);
+    __shared__ uint64_t red[kArgmaxThreads / 32][2];
+    if ((threadIdx.x & 31) == 0) {
+        red[threadIdx.x >> 5][0] = k1;
+        red[threadIdx.x >> 5][1] = k2;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        k1 = threadIdx.x < kArgmaxThreads / 32 ? red[threadIdx.x][0] : 0ull;
+        k2 = threadIdx.x < kArgmaxThreads / 32 ? red[threadIdx.x][1] : 0ull;
+        warp_top2(k1, k2);
+        if (threadIdx.x == 0) {
+            uint64_t *dst = a.partial + ((long long)m * a.blocks_per_row + b) * 2;
+            dst[0] = k1;
+            dst[1] = k2;
+        }
+    }
+}
+
+// One warp per row: the top two of the row's partial pairs, then the two words.
+// A flagged row gives its flagged word twice; an empty second place gives
+// TF_TOP2_NONE.
+__global__ void top2_final_kernel(ArgmaxArgs a) {
+    const int m = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (m >= a.M) return;
+    const int lane = threadIdx.x & 31;
+    uint64_t k1 = 0, k2 = 0;
+    for (int b = lane; b < a.blocks_per_row; b += 32) {
+        const uint64_t *p = a.partial + ((long long)m * a.blocks_per_row + b) * 2;
+        top2_merge_pair(k1, k2, p[0], p[1]);
+    }
+    warp_top2(k1, k2);
+    if (lane == 0) {
+        const uint16_t *row = a.logits + (long long)m * a.ld;
+        const uint64_t w1 = word_of_key(k1, row, a.id_base);
+        uint64_t w2;
+        if (k1 >> 63)
+            w2 = w1;
+        else
+            w2 = k2 == 0 ? TF_TOP2_NONE : word_of_key(k2, row, a.id_base);
+        a.words[2 * (long long)m] = w1;
+        a.words[2 * (long long)m + 1] = w2;
+    }
+}
+
+cudaError_t launch_top2(ArgmaxArgs a, cudaStream_t stream) {
+    a.blocks_per_row = argmax_blocks_per_row(a.M, a.n);
+    int span = (a.n + a.blocks_per_row - 1) / a.blocks_per_row;
+    span = (span + 7) / 8 * 8;
+    a.span = span;
+    dim3 grid(a.blocks_per_row, a.M);
+    top2_partial_kernel<<<grid, kArgmaxThreads, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    top2_final_kernel<<<(a.M + 7) / 8, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// One thread per row: the lowest part whose winner is flagged gives its flagged
+// word twice; otherwise the two highest of all the parts' words, compared by
+// their argmax keys (the words themselves are carried, so a winning -0 keeps
+// its sign).
+__device__ __forceinline__ uint64_t key_of_word(uint64_t w) {
+    if (w == TF_TOP2_NONE) return 0ull;
+    return cand_key((uint32_t)(w & 0xFFFFFFFFull) >> 16, (uint32_t)(w >> 32));
+}
+__global__ void top2_merge_kernel(const uint64_t *words2, int nparts, int M, uint64_t *out2) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M) return;
+    for (int p = 0; p < nparts; ++p) {
+        const uint64_t w = words2[((long long)p * M + m) * 2];
+        if ((uint32_t)(w >> 32) & TF_PAIR_FLAG) {
+            out2[2 * (long long)m] = w;
+            out2[2 * (long long)m + 1] = w;
+            return;
+        }
+    }
+    uint64_t k1 = 0, k2 = 0, w1 = TF_TOP2_NONE, w2 = TF_TOP2_NONE;
+    for (int p = 0; p < nparts; ++p)
+        for (int i = 0; i < 2; ++i) {
+            const uint64_t w = words2[((long long)p * M + m) * 2 + i];
+            const uint64_t k = key_of_word(w);
+            if (k > k1) {
+                k2 = k1;
+                w2 = w1;
+                k1 = k;
+                w1 = w;
+            } else if (k > k2) {
+                k2 = k;
+                w2 = w;
+            }
+        }
+    out2[2 * (long long)m] = w1;
+    out2[2 * (long long)m + 1] = w2;
+}
+
+cudaError_t launch_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out2, cudaStream_t stream) {
+    top2_merge_kernel<<<(M + 127) / 128, 128, 0, stream>>>(words2, nparts, M, out2);
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ pick --
 // One thread per row: any flagged id word -> the sentinel; otherwise the larger
 // value, the lower id on equal values (fp32 compare: +0 == -0).

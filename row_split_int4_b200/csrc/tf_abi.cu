@@ -297,6 +297,43 @@ tf_status tf_argmax_rows(const void *logits, int M, int n, int ld, uint32_t id_b
     return cuda_status(launch_argmax(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t tf_top2_scratch_bytes(int M, int n) {
+    if (M <= 0 || n <= 0) return 0;
+    return (size_t)M * (size_t)argmax_blocks_per_row(M, n) * 2 * sizeof(uint64_t);
+}
+
+tf_status tf_top2_rows(const void *logits, int M, int n, int ld, uint32_t id_base, uint64_t *words2, void *scratch,
+                       size_t scratch_bytes, tf_stream stream) {
+    if (M < 0 || M > 65535 || n < 1 || ld < n) return TF_E_ARG;
+    if ((unsigned long long)id_base + (unsigned long long)n > 0x80000000ull) return TF_E_RANGE;
+    if (M == 0) return TF_OK;
+    if (!logits || !words2 || !scratch) return TF_E_ARG;
+    if (scratch_bytes < tf_top2_scratch_bytes(M, n)) return TF_E_ARG;
+    if (!aligned(logits, 2) || !aligned(words2, 8) || !aligned(scratch, 8)) return TF_E_ALIGN;
+    ArgmaxArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.logits = static_cast<const uint16_t *>(logits);
+    a.ld = ld;
+    a.n = n;
+    a.id_base = id_base;
+    a.M = M;
+    a.partial = static_cast<uint64_t *>(scratch);
+    a.words = words2;
+    a.vec = aligned(logits, 16) && (ld % 8 == 0);
+    return cuda_status(launch_top2(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tf_status tf_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out2, tf_stream stream) {
+    if (nparts < 1 || nparts > TF_MAX_PARTS || M < 0 || M > 65535) return TF_E_ARG;
+    if (M == 0) return TF_OK;
+    if (!words2 || !out2) return TF_E_ARG;
+    if (!aligned(words2, 8) || !aligned(out2, 8)) return TF_E_ALIGN;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(words2), a1 = a0 + (size_t)nparts * M * 16;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(out2), b1 = b0 + (size_t)M * 16;
+    if (a0 < b1 && b0 < a1) return TF_E_ARG;   // out2 must not overlap the inputs
+    return cuda_status(launch_top2_merge(words2, nparts, M, out2, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tf_status tf_residual_add(float *h, int ld_h, const void *y, int ld_y, int M, int n, tf_stream stream) {
     if (M < 0 || n < 0 || ld_h < n || ld_y < n) return TF_E_ARG;
     if (M == 0 || n == 0) return TF_OK;

@@ -54,6 +54,7 @@ __device__ __forceinline__ uint64_t cand_key(uint32_t h, uint32_t id) {
 }
 
 __device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+__device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
 
 __device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
 #pragma unroll

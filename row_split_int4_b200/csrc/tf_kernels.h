@@ -74,6 +74,9 @@ struct ArgmaxArgs {
     int vec;               // 16-byte loads allowed
 };
 
+// top two: ArgmaxArgs with partial [M][blocks_per_row][2] and words [M][2]
+cudaError_t launch_top2(ArgmaxArgs a, cudaStream_t stream);
+cudaError_t launch_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out2, cudaStream_t stream);
 cudaError_t launch_qmm(const QmmArgs &a, cudaStream_t stream);
 cudaError_t launch_qmm8(const Qmm8Args &a, cudaStream_t stream);
 cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream);

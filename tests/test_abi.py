@@ -219,6 +219,27 @@ def test_last_cuda_error_is_static_text(tf):
     assert tf.tf_last_cuda_error() == "no error"
 
 
+def test_top2_refusals(tf):
+    L = tf.lib
+    assert L.tf_top2_rows(A, 1, 0, 8, 0, A, A, 1 << 20, None) == tf.TF_E_ARG
+    assert L.tf_top2_rows(A, 1, 16, 8, 0, A, A, 1 << 20, None) == tf.TF_E_ARG
+    assert L.tf_top2_rows(A, 65536, 16, 16, 0, A, A, 1 << 30, None) == tf.TF_E_ARG
+    assert L.tf_top2_rows(A, 1, 16, 16, 0x7FFFFFF8, A, A, 1 << 20, None) == tf.TF_E_RANGE
+    assert L.tf_top2_rows(A, 0, 16, 16, 0, 0, 0, 0, None) == tf.TF_OK
+    need = tf.tf_top2_scratch_bytes(2, 124160)
+    assert need == 2 * tf.tf_argmax_scratch_bytes(2, 124160)
+    assert L.tf_top2_rows(A, 2, 124160, 124160, 0, A, A, need - 8, None) == tf.TF_E_ARG
+    assert L.tf_top2_rows(A, 2, 124160, 124160, 0, A + 4, A, need, None) == tf.TF_E_ALIGN
+    assert L.tf_top2_rows(A + 1, 2, 124160, 124160, 0, A, A, need, None) == tf.TF_E_ALIGN
+    assert L.tf_top2_merge(A, 0, 1, A + 4096, None) == tf.TF_E_ARG
+    assert L.tf_top2_merge(A, 9, 1, A + 4096, None) == tf.TF_E_ARG
+    assert L.tf_top2_merge(A, 2, -1, A + 4096, None) == tf.TF_E_ARG
+    assert L.tf_top2_merge(A, 2, 4, A + 64, None) == tf.TF_E_ARG       # out2 overlaps the inputs
+    assert L.tf_top2_merge(A + 4, 2, 4, A + 4096, None) == tf.TF_E_ALIGN
+    assert L.tf_top2_merge(A, 2, 0, 0, None) == tf.TF_OK
+    assert tf.TF_TOP2_NONE == C.TOP2_NONE
+
+
 def test_pick_refusals(tf):
     L = tf.lib
     assert L.tf_pick(A, 0, 1, A, None) == tf.TF_E_ARG
