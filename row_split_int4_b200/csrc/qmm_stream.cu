@@ -95,62 +95,95 @@ __device__ __forceinline__ float lane_chunk_idot(const uint4 &q, const uint4 *li
     return fmaf((float)a2, 65536.0f, fmaf((float)a1, 256.0f, (float)a0));
 }
 
-// Fixed-point limbs of x for every lane-chunk, one warp per lane-chunk and one
-// lane per value, on the bf16 fields alone: x = sign * M * 2^(e-134), M = 128 +
-// mantissa (e >= 1) or the mantissa (e = 0, subnormal, read with e = 1).  With emax
+// Fixed-point limbs of x for every lane-chunk, on the bf16 fields alone: x = sign *
+// M * 2^(e-134), M = 128 + mantissa (e >= 1) or the mantissa (e = 0, subnormal, read
+// with e = 1).  With emax
 // the chunk's largest e, F = x * 2^(23-E), E = emax - 126, is sign * M * 2^(e - emax
 // + 15): a left shift when e >= emax - 15 (exact), else a right shift rounded to
 // nearest even.  Xs gets the fp32 sum of the chunk's 32 x, Ss the power of two
 // 2^(E-23) (NaN when the chunk holds a NaN or an infinity).
 __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, float *Xs, float *Ss, int W,
                                            int warp, int lane) {
-    // loads go out sixteen lane-chunks at a time so that one L2 round trip covers them
-    constexpr int kPrepBatch = 16;
-    for (int lc0 = warp; lc0 < nch * 32; lc0 += W * kPrepBatch) {
-      uint32_t hb[kPrepBatch];
-#pragma unroll
-      for (int i = 0; i < kPrepBatch; ++i) {
-          const int lc = lc0 + i * W;
-          const int k = (lc >> 5) * kChunk + (lc & 31) * 32 + lane;
-          hb[i] = (lc < nch * 32 && k < K) ? (uint32_t)x[k] : 0u;
-      }
-#pragma unroll
-      for (int i = 0; i < kPrepBatch; ++i) {
-        const int lc = lc0 + i * W;
-        if (lc >= nch * 32) break;
+    // one thread per lane-chunk, all of it in registers: no cross-lane step, so
+    // the whole CTA prepares up to W * 32 lane-chunks in one pass
+    const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+    for (int lc = warp * 32 + lane; lc < nch * 32; lc += W * 32) {
         const int c = lc >> 5, l = lc & 31;
-        const uint32_t h = hb[i];
-        const uint32_t ef = (h >> 7) & 0xFFu;
-        const bool bad = __any_sync(0xFFFFFFFFu, ef == 0xFFu);
-        const int e = ef == 0 ? 1 : (int)ef;
-        const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
-        const int emax = __reduce_max_sync(0xFFFFFFFFu, M != 0 ? e : 0);
-        const int sh = e - emax + 15;
-        int F;
-        if (sh >= 0) {
-            F = M << sh;
-        } else if (sh > -9) {
-            const int d = -sh;
-            F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
-        } else {
-            F = 0;
-        }
-        if (h & 0x8000u) F = -F;
-        if (bad) F = 0;
-        const int w = lane >> 3, p = lane & 1, byte = (lane & 7) >> 1;
-        uint8_t *base = limbs + (size_t)(c * 6 * 32 + l) * 16 + w * 4 + byte;
-        base[(size_t)(0 * 2 + p) * 32 * 16] = (uint8_t)(F & 0xFF);
-        base[(size_t)(1 * 2 + p) * 32 * 16] = (uint8_t)((F >> 8) & 0xFF);
-        base[(size_t)(2 * 2 + p) * 32 * 16] = (uint8_t)((F >> 16) & 0xFF);
-        float sx = bf16_bits_to_f32(h);
+        const int k0 = c * kChunk + l * 32;
+        uint32_t hv[16];   // the 32 bf16 x of the lane-chunk, two per word (zero past K)
+        if (x16 && k0 + 32 <= K) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(x + k0);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sx += __shfl_down_sync(0xFFFFFFFFu, sx, o);
-        if (lane == 0) {
-            Xs[lc] = sx;
-            // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
-            Ss[lc] = bad ? __int_as_float(0x7FC00000) : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = src[i];
+                hv[4 * i] = v.x;
+                hv[4 * i + 1] = v.y;
+                hv[4 * i + 2] = v.z;
+                hv[4 * i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t lo = k0 + 2 * i < K ? x[k0 + 2 * i] : 0u;
+                const uint32_t hi = k0 + 2 * i + 1 < K ? x[k0 + 2 * i + 1] : 0u;
+                hv[i] = lo | (hi << 16);
+            }
         }
-      }
+        bool bad = false;
+        int emax = 0;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
+            const uint32_t ef = (h >> 7) & 0xFFu;
+            bad = bad || ef == 0xFFu;
+            const int e = ef == 0 ? 1 : (int)ef;
+            if ((h & 0x7FFFu) != 0) emax = max(emax, e);   // M != 0
+        }
+        uint32_t L[6][4];
+#pragma unroll
+        for (int q = 0; q < 6; ++q)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) L[q][w] = 0u;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
+            const uint32_t ef = (h >> 7) & 0xFFu;
+            const int e = ef == 0 ? 1 : (int)ef;
+            const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
+            const int sh = e - emax + 15;
+            int F;
+            if (sh >= 0) {
+                F = M << sh;
+            } else if (sh > -9) {
+                const int d = -sh;
+                F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
+            } else {
+                F = 0;
+            }
+            if (h & 0x8000u) F = -F;
+            if (bad) F = 0;
+            // value t of the lane-chunk: word t >> 3, byte (t & 7) >> 1 of limb vector 2 limb + (t & 1)
+            const int w = t >> 3, p = t & 1, sft = 8 * ((t & 7) >> 1);
+            L[0 + p][w] |= (uint32_t)(F & 0xFF) << sft;
+            L[2 + p][w] |= (uint32_t)((F >> 8) & 0xFF) << sft;
+            L[4 + p][w] |= (uint32_t)((F >> 16) & 0xFF) << sft;
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
+#pragma unroll
+        for (int q = 0; q < 6; ++q) dst[q * 32] = make_uint4(L[q][0], L[q][1], L[q][2], L[q][3]);
+        // sum of the 32 x in the pairing of a five-step warp shuffle tree
+        float sx[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            sx[i] = bf16_bits_to_f32(hv[i >> 1] >> (16 * (i & 1)) & 0xFFFFu) +
+                    bf16_bits_to_f32(hv[(i + 16) >> 1] >> (16 * (i & 1)) & 0xFFFFu);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+            for (int i = 0; i < o; ++i) sx[i] += sx[i + o];
+        Xs[lc] = sx[0];
+        // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
+        Ss[lc] = bad ? __int_as_float(0x7FC00000) : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
     }
 }
 
@@ -382,12 +415,21 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
 // warp frees a slot by one arrival on the slot's empty barrier.  Tiles are
 // claimed in order from the CTA's share by a counter in shared memory, so the
 // groups stay busy to the end of the share.
-constexpr int kTRows = 16;                                   // rows of a tile
+// A tile is 4 kWR rows by 4 / kWR chunks of K: kWR = 4 (16 rows by 1,024) for wide
+// calls, kWR = 1 (4 rows by 4,096) for calls with few rows (down and attn_out
+// halves), so that the four groups of every SM still find tiles.  Every slot
+// holds 9,216 bytes, and each compute warp takes kWR rows of it.
 constexpr int kTGroups = 4, kTGroupWarps = 4, kTWarps = kTGroups * kTGroupWarps;   // compute warps
 constexpr int kTThreads = (kTWarps + kTGroups) * 32;          // and one producer warp per group
-constexpr int kTSlotQ = kChunk / 2;                          // code bytes of one row in a slot
-constexpr int kTSlotS = kChunk / 32;                         // scale (or bias) bytes of one row
-constexpr int kTSlotBytes = kTRows * (kTSlotQ + 2 * kTSlotS);   // 9,216
+constexpr int kTSlotBytes = 16 * (kChunk / 2 + 2 * (kChunk / 32));   // 9,216
+template <int kWR> struct TileShape {
+    static constexpr int rows = kTGroupWarps * kWR;          // rows of a tile
+    static constexpr int cps = 4 / kWR;                      // chunks per slot
+    static constexpr int q = cps * (kChunk / 2);             // code bytes of one row in a slot
+    static constexpr int sb = cps * (kChunk / 32);           // scale (or bias) bytes of one row
+    static constexpr int qelem = q > 1024 ? 8 : 4;           // code element of the tensor map (box <= 256)
+    static_assert(rows * (q + 2 * sb) == kTSlotBytes, "slot size");
+};
 constexpr int kTMaxStages = 6;
 
 struct TileLayout {
@@ -427,21 +469,25 @@ __device__ __forceinline__ bool tile_wait(uint32_t bar, uint32_t parity, const v
     return false;
 }
 
-// Slot row of a warp's unit row r: rows 4w .. 4w+3 (NONE); for GLU the gate rows
-// sit in slot rows 0..7 and the up rows in 8..15, and unit row r is member r & 1
-// of column 2w + (r >> 1), the order the GLU epilogue reads.
-template <bool kGlu>
+// Slot row of a warp's row r: rows kWR w .. kWR w + kWR - 1 (NONE); for GLU the gate
+// rows sit in the first half of the slot and the up rows in the second, and row r
+// is member r & 1 of column (kWR / 2) w + (r >> 1), the order the GLU epilogue reads.
+template <bool kGlu, int kWR>
 __device__ __forceinline__ int tile_row(int w, int r) {
-    return kGlu ? (r & 1) * 8 + 2 * w + (r >> 1) : 4 * w + r;
+    return kGlu ? (r & 1) * (2 * kWR) + (kWR / 2) * w + (r >> 1) : kWR * w + r;
 }
 
-template <bool kGlu>
+template <bool kGlu, int kWR>
 __global__ void __launch_bounds__(kTThreads, 1)
     qmm_m1_tile_kernel(QmmArgs a, TilePlan plan, const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap bmap, int S) {
     extern __shared__ __align__(128) uint8_t smem[];
     const TileLayout L = tile_layout(a.K, S);
+    using Sh = TileShape<kWR>;
+    static_assert(!kGlu || kWR >= 2, "a GLU column needs its gate and up rows in one warp");
+    constexpr int kRows = Sh::rows, kCps = Sh::cps;
     const int K = a.K, nch = L.nch;
+    const int nsl = (nch + kCps - 1) / kCps;   // slots of a tile
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool producer = warp >= kTWarps;
     const int grp = producer ? warp - kTWarps : warp / kTGroupWarps, w_in = warp % kTGroupWarps;
@@ -474,10 +520,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
     // first matrix row (both members for GLU) and first output column of tile t
     auto tile_rows = [&](int t, int &r_a, int &r_b, int &col, int &ncol) {
         if (kGlu) {
-            r_a = a.seg.row0[0] + 8 * t;
-            r_b = a.seg.row0[1] + 8 * t;
-            col = 8 * t;
-            ncol = min(8, a.seg.ncols - col);
+            r_a = a.seg.row0[0] + (kRows / 2) * t;
+            r_b = a.seg.row0[1] + (kRows / 2) * t;
+            col = (kRows / 2) * t;
+            ncol = min(kRows / 2, a.seg.ncols - col);
         } else {
             // the last segment starting at or before t (selected without a
             // dynamic index into the parameter arrays)
@@ -491,20 +537,20 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     nr = a.seg.nrows[s2];
                 }
             const int i = t - ts;
-            r_a = row0 + kTRows * i;
+            r_a = row0 + kRows * i;
             r_b = 0;
-            col = col0 + kTRows * i;
-            ncol = min(kTRows, nr - kTRows * i);
+            col = col0 + kRows * i;
+            ncol = min(kRows, nr - kRows * i);
         }
     };
 
     // issue state of the group's producer (lane 0): the tile being sent (-1: none
     // left), its next chunk, the slot and its use count
-    int it_tile = -2, it_c = nch, islot = 0, iuse = 0, nissued = 0;
+    int it_tile = -2, it_c = nsl, islot = 0, iuse = 0, nissued = 0;
     bool done_issuing = false;
     auto issue_next = [&]() {   // lane 0 of the producer warp only
         if (done_issuing) return;
-        if (it_c == nch) {
+        if (it_c == nsl) {
             const int t = t0 + atomicAdd(claim, 1);
             it_tile = t < t1 ? t : -1;
             it_c = 0;
@@ -521,15 +567,16 @@ __global__ void __launch_bounds__(kTThreads, 1)
             tile_rows(it_tile, r_a, r_b, col, ncol);
             mbar_expect_tx(full, (uint32_t)kTSlotBytes);
             const uint32_t dst = ring_s + islot * kTSlotBytes;
-            constexpr uint32_t kS0 = kTRows * kTSlotQ, kB0 = kS0 + kTRows * kTSlotS;
-            const int cq = it_c * (kChunk / 8), cs = it_c * (kChunk / 64);   // 4-byte code words, bf16 groups
+            constexpr uint32_t kS0 = kRows * Sh::q, kB0 = kS0 + kRows * Sh::sb;
+            // inner coordinates in the maps' elements: code words, bf16 groups
+            const int cq = it_c * (Sh::q / Sh::qelem), cs = it_c * (Sh::sb / 2);
             tma_load_2d(dst, &qmap, cq, r_a, full);
             tma_load_2d(dst + kS0, &smap, cs, r_a, full);
             tma_load_2d(dst + kB0, &bmap, cs, r_a, full);
             if (kGlu) {
-                tma_load_2d(dst + 8 * kTSlotQ, &qmap, cq, r_b, full);
-                tma_load_2d(dst + kS0 + 8 * kTSlotS, &smap, cs, r_b, full);
-                tma_load_2d(dst + kB0 + 8 * kTSlotS, &bmap, cs, r_b, full);
+                tma_load_2d(dst + (kRows / 2) * Sh::q, &qmap, cq, r_b, full);
+                tma_load_2d(dst + kS0 + (kRows / 2) * Sh::sb, &smap, cs, r_b, full);
+                tma_load_2d(dst + kB0 + (kRows / 2) * Sh::sb, &bmap, cs, r_b, full);
             }
             ++it_c;
         } else {
@@ -556,7 +603,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
         __syncwarp();
     }
 
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float acc[kWR];
+#pragma unroll
+    for (int r = 0; r < kWR; ++r) acc[r] = 0.0f;
     uint64_t best = 0;
     int slot = 0;
     uint32_t par = 0;
@@ -570,22 +619,25 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         const int2 h = hdr[slot];
         if (h.x < 0) break;
-        const int c = h.y;
         const uint8_t *sl = ring + slot * kTSlotBytes;
-        if (lane * 32 < K - c * kChunk) {   // lanes past the end of a short last chunk add nothing
+        const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
+        const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kRows * Sh::q) + (lane >> 1);
+#pragma unroll
+        for (int cc = 0; cc < kCps; ++cc) {
+            const int c = h.y * kCps + cc;
+            // chunks past K, and lanes past the end of a short last chunk, add nothing
+            if (c >= nch || lane * 32 >= K - c * kChunk) break;
             uint4 lm[6];
 #pragma unroll
             for (int q = 0; q < 6; ++q) lm[q] = limb_l[(c * 6 + q) * 32];
             const float X = Xs[c * 32 + lane];
             const float scale = Ss[c * 32 + lane];
-            const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
-            const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kTRows * kTSlotQ) + (lane >> 1);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int R = tile_row<kGlu>(w_in, r);
-                const uint4 qv = ql[R * (kTSlotQ / 16)];
-                const float s = bf16_bits_to_f32(sc16[R * (kTSlotS / 2)]);
-                const float b = bf16_bits_to_f32(sc16[kTRows * (kTSlotS / 2) + R * (kTSlotS / 2)]);
+            for (int r = 0; r < kWR; ++r) {
+                const int R = tile_row<kGlu, kWR>(w_in, r);
+                const uint4 qv = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
+                const float s = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+                const float b = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
                 const float P = lane_chunk_idot(qv, lm);
                 acc[r] = fmaf(s, P * scale, acc[r]);   // P * 2^(E-23): exact power-of-two scaling
                 acc[r] = fmaf(b, X, acc[r]);
@@ -597,10 +649,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
             slot = 0;
             par ^= 1u;
         }
-        if (c == nch - 1) {
-            float tot[4];
+        if (h.y == nsl - 1) {
+            float tot[kWR];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < kWR; ++r) {
                 tot[r] = warp_sum_to_lane0(acc[r]);
                 acc[r] = 0.0f;
             }
@@ -609,20 +661,22 @@ __global__ void __launch_bounds__(kTThreads, 1)
                 tile_rows(h.x, r_a, r_b, col, ncol);
                 if (kGlu) {
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        if (2 * w_in + p < ncol) {
+                    for (int p = 0; p < kWR / 2; ++p) {
+                        const int cj = (kWR / 2) * w_in + p;
+                        if (cj < ncol) {
                             const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p]));
                             const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1]));
-                            a.y[col + 2 * w_in + p] = f32_to_bf16_rne(glu_f32(g, uu));
+                            a.y[col + cj] = f32_to_bf16_rne(glu_f32(g, uu));
                         }
                     }
                 } else {
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        if (4 * w_in + r < ncol) {
+                    for (int r = 0; r < kWR; ++r) {
+                        const int cj = kWR * w_in + r;
+                        if (cj < ncol) {
                             const uint16_t hv = f32_to_bf16_rne(tot[r]);
-                            a.y[col + 4 * w_in + r] = hv;
-                            if (a.cand) best = umax64(best, cand_key(hv, a.id_base + (uint32_t)(col + 4 * w_in + r)));
+                            a.y[col + cj] = hv;
+                            if (a.cand) best = umax64(best, cand_key(hv, a.id_base + (uint32_t)(col + cj)));
                         }
                     }
                 }
@@ -694,16 +748,16 @@ static int tile_stages(int K) {
     return 0;
 }
 
-static TilePlan tile_plan(const QmmArgs &a) {
+static TilePlan tile_plan(const QmmArgs &a, int rows) {
     TilePlan plan{};
     if (a.glu) {
-        plan.ntiles = (a.seg.ncols + 7) / 8;
+        plan.ntiles = (a.seg.ncols + rows / 2 - 1) / (rows / 2);
         for (int s = 1; s <= TF_MAX_SEGS; ++s) plan.tstart[s] = plan.ntiles;
     } else {
         int n = 0;
         for (int s = 0; s < a.seg.nseg; ++s) {
             plan.tstart[s] = n;
-            n += (a.seg.nrows[s] + kTRows - 1) / kTRows;
+            n += (a.seg.nrows[s] + rows - 1) / rows;
         }
         for (int s = a.seg.nseg; s <= TF_MAX_SEGS; ++s) plan.tstart[s] = n;
         plan.ntiles = n;
@@ -711,30 +765,36 @@ static TilePlan tile_plan(const QmmArgs &a) {
     return plan;
 }
 
-// The tile ring takes the call when it has at least four tiles per SM (fewer
-// leave groups idle, and the per-warp kernel's finer units balance better), the
-// driver offers the tensor-map encoder and two slots per group fit beside the limbs.
-static bool tile_ring_fits(const QmmArgs &a) {
-    if (!encode_tiled_fn() || tile_stages(a.K) < 2) return false;
-    return tile_plan(a).ntiles >= 4 * num_sms();
+// The tile ring takes the call when the driver offers the tensor-map encoder, two
+// slots per group fit beside the limbs, and the tiles keep every group busy: 16-row
+// tiles with at least four per SM, else (not GLU) 4-row tiles with at least two per
+// SM; otherwise the per-warp kernel's finer units balance better.  Returns the rows
+// per compute warp of the tile shape, 0 for the per-warp kernel.
+static int tile_ring_shape(const QmmArgs &a) {
+    if (!encode_tiled_fn() || tile_stages(a.K) < 2) return 0;
+    if (tile_plan(a, TileShape<4>::rows).ntiles >= 4 * num_sms()) return 4;
+    if (!a.glu && tile_plan(a, TileShape<1>::rows).ntiles >= 2 * num_sms()) return 1;
+    return 0;
 }
 
-static bool g_tile_smem_set[64][2];
+static bool g_tile_smem_set[64][2][2];
 
-template <bool kGlu>
+template <bool kGlu, int kWR>
 static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream) {
+    using Sh = TileShape<kWR>;
     const int S = tile_stages(a.K);
     const TileLayout L = tile_layout(a.K, S);
-    const TilePlan plan = tile_plan(a);
+    const TilePlan plan = tile_plan(a, Sh::rows);
     auto enc = encode_tiled_fn();
-    const cuuint32_t box_rows = kGlu ? 8u : (cuuint32_t)kTRows;
+    const cuuint32_t box_rows = kGlu ? (cuuint32_t)(Sh::rows / 2) : (cuuint32_t)Sh::rows;
     const cuuint32_t estr[2] = {1, 1};
     CUtensorMap qmap, smap, bmap;
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)(a.K / 8), (cuuint64_t)a.n_whole};
+        const cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2 / Sh::qelem), (cuuint64_t)a.n_whole};
         const cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
-        const cuuint32_t box[2] = {(cuuint32_t)(kChunk / 8), box_rows};
-        if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t *>(a.wq), dims, strides, box, estr,
+        const cuuint32_t box[2] = {(cuuint32_t)(Sh::q / Sh::qelem), box_rows};
+        const CUtensorMapDataType qt = Sh::qelem == 8 ? CU_TENSOR_MAP_DATA_TYPE_UINT64 : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+        if (enc(&qmap, qt, 2, const_cast<uint8_t *>(a.wq), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -743,7 +803,7 @@ static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream) {
         const int G = a.K / kGroup;
         const cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)a.n_whole};
         const cuuint64_t strides[1] = {(cuuint64_t)G * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)(kChunk / kGroup), box_rows};
+        const cuuint32_t box[2] = {(cuuint32_t)(Sh::sb / 2), box_rows};
         if (enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(a.scales), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
@@ -754,22 +814,27 @@ static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream) {
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (!g_tile_smem_set[dev][kGlu ? 1 : 0]) {
-        cudaError_t e = cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+    if (!g_tile_smem_set[dev][kGlu ? 1 : 0][kWR == 4 ? 1 : 0]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu, kWR>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
         if (e != cudaSuccess) return e;
-        g_tile_smem_set[dev][kGlu ? 1 : 0] = true;
+        g_tile_smem_set[dev][kGlu ? 1 : 0][kWR == 4 ? 1 : 0] = true;
     }
     const int blocks = plan.ntiles < num_sms() ? plan.ntiles : num_sms();
-    qmm_m1_tile_kernel<kGlu><<<blocks, kTThreads, L.total, stream>>>(a, plan, qmap, smap, bmap, S);
+    qmm_m1_tile_kernel<kGlu, kWR><<<blocks, kTThreads, L.total, stream>>>(a, plan, qmap, smap, bmap, S);
     return cudaGetLastError();
 }
 
-// Wide calls take the tile ring.  Otherwise rows per unit only change how often a
-// lane reuses its activation limbs, never a row's arithmetic, so the choice may
-// follow N: four rows while every warp of the grid still gets two units, fewer
-// when the slice is narrow.
+// Calls with enough tiles take the tile ring.  Otherwise rows per unit only change
+// how often a lane reuses its activation limbs, never a row's arithmetic, so the
+// choice may follow N: four rows while every warp of the grid still gets two
+// units, fewer when the slice is narrow.
 cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream) {
-    if (tile_ring_fits(a)) return a.glu ? launch_tile<true>(a, stream) : launch_tile<false>(a, stream);
+    switch (tile_ring_shape(a)) {
+        case 4: return a.glu ? launch_tile<true, 4>(a, stream) : launch_tile<false, 4>(a, stream);
+        case 1: return launch_tile<false, 1>(a, stream);
+        default: break;
+    }
     const long long warps = (long long)num_sms() * stream_warps(a.K, 4);
     const long long rows = a.glu ? 2ll * a.seg.ncols : a.seg.ncols;
     if (rows >= 8 * warps) return launch_ru<4>(a, 0, stream);
