@@ -1,0 +1,89 @@
+"""The M = 1 tile ring at the edges of its shapes: a ragged last 1,024-K chunk,
+several segments and a partial last tile (16-row tiles), a ragged last slot of
+4-row x 4,096-K tiles, and a GLU call whose column count is not a multiple of
+the 8-column tile.  Each case is checked against the oracle on sampled columns
+(V) and bit for bit against the same rows asked another way (S) -- including
+calls small enough to take the per-warp ring, so the two kernels must agree on
+every bit of a row."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import DevWeights, bits_equal, check_values, dev, empty_bf16, host_bits, need_gpu
+
+pytestmark = pytest.mark.gpu
+NT = os.cpu_count() or 1
+SAMPLE = 160
+
+
+@pytest.fixture(scope="module")
+def tf():
+    need_gpu()
+    import row_split_int4_b200 as tf
+    return tf
+
+
+def qmm(tf, xt, W, segs, epi=0):
+    ncols = segs[0][1] if epi else sum(n for _, n in segs)
+    y = empty_bf16(1, ncols)
+    tf.tf_qmm_rows(xt, *W.t(), segs, y, epi=epi)
+    return y
+
+
+def sampled(orc, x, w, y_bits, rows, K, what, seed=0):
+    rng = np.random.default_rng(seed)
+    pick = np.sort(rng.choice(len(rows), min(SAMPLE, len(rows)), replace=False))
+    pick = np.unique(np.concatenate([pick, [0, len(rows) - 1]]))   # both ends of the call
+    yo, y64, ad = orc.qmm_rows(x, *w.astuple(), np.asarray(rows)[pick], nthreads=NT, want_f64=True)
+    return check_values(y_bits[:, pick], yo, y64, ad, K, what)
+
+
+def columns_of(segs):
+    return np.concatenate([np.arange(r0, r0 + n) for r0, n in segs])
+
+
+@pytest.mark.parametrize("K,N,seg_sets", [
+    # 16-row tiles; K = 5.5 chunks: the last chunk is half empty
+    (5632, 9600, [[(0, 3000), (3000, 6600)], [(6000, 3600), (0, 2999), (2999, 3001)]]),
+    # 4-row x 4,096-K tiles; K = 17.5 chunks: the last slot holds one and a half chunks;
+    # N = 1,203 leaves a partial last tile; a half alone is narrow enough for the per-warp ring
+    (17920, 1203, [[(0, 601), (601, 602)], [(1000, 203), (0, 1000)], [(0, 601)], [(601, 602)]]),
+])
+def test_tile_ring_ragged_and_segments(tf, orc, K, N, seg_sets):
+    w = synth.make_weights(N, K, seed=K % 97, tag=synth.TAG_W2)
+    W = DevWeights(w)
+    x = synth.make_x(1, K, seed=N)
+    xt = dev(x)
+    whole = qmm(tf, xt, W, [(0, N)])
+    torch.cuda.synchronize()
+    sampled(orc, x, w, host_bits(whole), np.arange(N), K, f"K={K} N={N} whole")
+    for segs in seg_sets:
+        y = qmm(tf, xt, W, segs)
+        cols = columns_of(segs)
+        torch.cuda.synchronize()
+        assert bits_equal(y, whole[:, torch.as_tensor(cols, device="cuda")]), segs
+        sampled(orc, x, w, host_bits(y), cols, K, f"K={K} N={N} segs={segs}", seed=1)
+
+
+def test_tile_ring_glu_odd_columns(tf, orc):
+    """F = 4,740 GLU columns: 593 tiles of 8 columns (the last one holding 4), at
+    K = 5,120; the member-split halves (2,370 columns) take the per-warp ring."""
+    F, K = 4740, 5120
+    w = synth.make_weights(2 * F, K, seed=31, tag=synth.TAG_W)
+    W = DevWeights(w)
+    x = synth.make_x(1, K, seed=31)
+    xt = dev(x)
+    whole = qmm(tf, xt, W, [(0, F), (F, F)], epi=tf.TF_EPI_GLU)
+    parts = [qmm(tf, xt, W, tf.tf_member_segs(F, 2, h), epi=tf.TF_EPI_GLU) for h in range(2)]
+    joined = empty_bf16(1, F)
+    tf.tf_gather_rows(joined, parts, [F // 2, F // 2])
+    g = qmm(tf, xt, W, [(0, F)])
+    u = qmm(tf, xt, W, [(F, F)])
+    torch.cuda.synchronize()
+    assert bits_equal(joined, whole), "GLU: member halves != whole"
+    check_values(host_bits(whole), orc.glu(host_bits(g), host_bits(u)), what="GLU stage, tile ring")
+    sampled(orc, x, w, host_bits(g), np.arange(F), K, "gate rows")
+    sampled(orc, x, w, host_bits(u), np.arange(F, 2 * F), K, "up rows", seed=2)
