@@ -10,13 +10,18 @@ two row halves on one GPU (TensorFold PR #1433, step-1 and step-2 bodies):
   gather   the two 8,704-wide activated halves         (tf_gather_rows)
   down     K=17,408 -> 5,120 rows as 2 x 2,560          (tf_qmm_rows)
   gather   the two 2,560-wide halves                    (tf_gather_rows)
-  lm_head  K=5,120 -> 248,320 rows as 2 x 124,160       (tf_qmm_rows)
-  argmax   per half, global ids                         (tf_argmax_rows)
+  head     per half: lm_head K=5,120 -> 124,160 rows and the half's argmax
+           word in one call (tf_qmm_argmax_rows: the qmm's warps keep their
+           best keys, one small kernel makes the word)
   pick     the better half-winner                       (tf_pick)
 
-(tf_qmm_argmax_rows fuses the last three into one call per half; it measures the
-same time as the three launches, and the separate calls let the event pairs
-time the lm_head qmm kernel alone for the roofline.)
+Timed regions (CUDA events on the launching stream, after the warm-up):
+  1. K steps back to back, events only at the two ends: `value`, ms_per_step.
+  2. K steps with an event pair around the head (both halves and the pick):
+     lm_head_argmax_us_per_token.
+  3. K launches of one lm_head half's qmm alone (tf_qmm_rows, the kernel the
+     fused head runs), alternating halves, each in an event pair: the
+     roofline's average launch duration.
 
 The metric is the int4 dequant-GEMV HBM throughput (GB/s of algorithmic
 bytes: 0.5625 B per weight plus activations in and out), with the
@@ -49,6 +54,7 @@ METRIC = "int4 dequant-GEMV HBM GB/s (% B200 peak) at M=1; lm_head+argmax µs/to
 WORKLOAD = ("decode step M=1, two row halves on one GPU: gate_up 5120x34816 int4 g64 (GLU fused) + gather + "
             "down 17408x5120 + gather + lm_head 5120x248320 + per-half argmax + pick")
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0   # B200 spec sheet
 
 
 # --------------------------------------------------------------------------- helpers
@@ -109,20 +115,34 @@ def step_bytes():
     return b
 
 
-def traffic_from_profiles(kernel_src):
+KERNEL_SOURCES = ["row_split_int4_b200/csrc/qmm_stream.cu", "row_split_int4_b200/csrc/qmm_common.cuh",
+                  "row_split_int4_b200/csrc/stream_common.cuh", "row_split_int4_b200/csrc/tf_common.cuh",
+                  "row_split_int4_b200/csrc/tf_kernels.h", "include/tf.h"]
+
+
+def device_source_hash():
+    """sha256 over the files the M = 1 streaming kernels are compiled from, in
+    KERNEL_SOURCES order (profiles record it when their counters are taken)."""
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_from_profiles():
     """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
-    only while the kernel's source is the one the counters were taken on."""
+    only while the kernel's sources are the ones the counters were taken on."""
     path = os.path.join(ROOT, "profiles", "qmm_m1_tile_lm_head_half.md")
     try:
         txt = open(path).read()
     except OSError:
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
-    s = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    s = re.search(r"device_source_sha256:\s*([0-9a-f]{64})", txt)
     if not m or not s:
         return None
-    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
-    return int(m.group(1)) if cur == s.group(1) else None
+    return int(m.group(1)) if device_source_hash() == s.group(1) else None
 
 
 class ClockSampler:
@@ -199,14 +219,16 @@ class DecodeStep:
         self.logits = [torch.empty(1, V // 2, **bf) for _ in range(2)]
         self.words = torch.empty(2, 1, dtype=torch.int64, device="cuda")
         self.ids = torch.empty(1, dtype=torch.int32, device="cuda")
-        self.scratch = torch.empty(tf.tf_argmax_scratch_bytes(1, V // 2), dtype=torch.uint8, device="cuda")
+        self.head_scratch = [torch.empty(tf.tf_qmm_argmax_scratch_bytes(1, V // 2), dtype=torch.uint8, device="cuda")
+                             for _ in range(2)]
         self.member = [tf.tf_member_segs(F, 2, h) for h in range(2)]
         self.down_rows = [tf.tf_split_rows(H, 2, h) for h in range(2)]
         self.head_rows = [tf.tf_split_rows(V, 2, h) for h in range(2)]
         self.window = synth.WINDOW_BYTES
-        self.launches_per_step = 2 + 1 + 2 + 1 + 2 + 2 * 2 + 1
+        # gate_up x2, gather, down x2, gather, per half the head's qmm and its key kernel, pick
+        self.launches_per_step = 2 + 1 + 2 + 1 + 2 * 2 + 1
 
-    def run(self, stream, lm_events=None, head_events=None):
+    def run(self, stream, head_events=None):
         tf = self.tf
         for h in range(2):
             tf.tf_qmm_rows(self.x_mlp, *self.Wgu, self.member[h], self.act_h[h], epi=tf.TF_EPI_GLU, stream=stream)
@@ -217,16 +239,16 @@ class DecodeStep:
         if head_events is not None:
             head_events[0].record(stream)
         for h in range(2):
-            if lm_events is not None:
-                lm_events[h][0].record(stream)
-            tf.tf_qmm_rows(self.x_head, *self.Wlm, [self.head_rows[h]], self.logits[h], stream=stream)
-            if lm_events is not None:
-                lm_events[h][1].record(stream)
-        for h in range(2):
-            tf.tf_argmax_rows(self.logits[h], self.head_rows[h][0], self.words[h], self.scratch, stream=stream)
+            r0, n = self.head_rows[h]
+            tf.tf_qmm_argmax_rows(self.x_head, *self.Wlm, (r0, n), r0, self.logits[h], self.words[h],
+                                  self.head_scratch[h], stream=stream)
         tf.tf_pick(self.words, self.ids, stream=stream)
         if head_events is not None:
             head_events[1].record(stream)
+
+    def lm_head_half(self, h, stream):
+        """One half of the lm_head qmm alone: the kernel the fused head runs."""
+        self.tf.tf_qmm_rows(self.x_head, *self.Wlm, [self.head_rows[h]], self.logits[h], stream=stream)
 
 
 def make_host_weights(synth, seed=0):
@@ -274,7 +296,21 @@ def calibrated_oracle(hw, target_s, nthreads):
     return frac
 
 
-def cpu_baseline(hw, target_s=20.0):
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(hw, target_s=20.0, single_s=5.0):
+    """The oracle on all host cores (OpenMP over rows) on a calibrated sample of the
+    step, and once more on one thread on a smaller sample."""
     nthreads = os.cpu_count() or 1
     frac = calibrated_oracle(hw, target_s, nthreads)
     tot_t, tot_b, reps, desc = 0.0, 0, 0, ""
@@ -283,8 +319,13 @@ def cpu_baseline(hw, target_s=20.0):
         tot_t += dt
         tot_b += nb
         reps += 1
+    f1 = calibrated_oracle(hw, single_s, 1)
+    dt1, nb1, desc1 = oracle_sample(hw, f1, 1)
     return {"value": round(tot_b / tot_t / 1e9, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
-            "sample": desc + f", x{reps}, {tot_t:.1f} s, C fp64 oracle with OpenMP over rows"}
+            "cpu_model": cpu_model(),
+            "sample": desc + f", x{reps}, {tot_t:.1f} s, C fp64 oracle with OpenMP over rows",
+            "single_thread": {"value": round(nb1 / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "sample": desc1 + f", {dt1:.1f} s"}}
 
 
 # --------------------------------------------------------------------------- reference arm
@@ -409,7 +450,7 @@ L2_BYTES = 126 * 1024 * 1024
 
 def run_sweep(args):
     """M in {1..128} over the four shapes, each point the two row halves of the
-    shape (plus both argmaxes and the pick for lm_head), --reps back-to-back
+    shape (for lm_head each half through the fused qmm + argmax call, then the pick), --reps back-to-back
     repetitions timed with CUDA events.  The weights stay in HBM; each shape is
     replicated into enough separate buffers to span 3 x L2 and the repetitions
     rotate through them, so a repetition never finds its weights in L2, and a
@@ -423,6 +464,7 @@ def run_sweep(args):
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     shapes = [s for s in SWEEP_SHAPES if not args.shapes or s in args.shapes.split(",")]
+    points = []
     Ms = [int(m) for m in args.sweep_m.split(",")] if args.sweep_m else list(SWEEP_M)
     for name in shapes:
         N, K, epi = SWEEP_SHAPES[name]
@@ -442,19 +484,22 @@ def run_sweep(args):
         head = name == "lm_head"
         if head:
             ids = torch.empty(max(Ms), dtype=torch.int32, device="cuda")
-            scratch = torch.empty(tf.tf_argmax_scratch_bytes(max(Ms), cols), dtype=torch.uint8, device="cuda")
+            hscr = [torch.empty(tf.tf_qmm_argmax_scratch_bytes(max(Ms), cols), dtype=torch.uint8, device="cuda")
+                    for _ in range(2)]
         for M in Ms:
             if head:
                 words = torch.empty(2, M, dtype=torch.int64, device="cuda")   # [half][M], contiguous
 
             def rep(r):
                 wr = replicas[r % nrep]
+                if head:   # per half the fused qmm + argmax word, then the pick
+                    for h in range(2):
+                        r0, n = segs[h][0]
+                        tf.tf_qmm_argmax_rows(x[:M], *wr, (r0, n), r0, y[h][:M], words[h], hscr[h], stream=stream)
+                    tf.tf_pick(words, ids[:M], stream=stream)
+                    return
                 for h in range(2):
                     tf.tf_qmm_rows(x[:M], *wr, segs[h], y[h][:M], epi=epi, stream=stream)
-                if head:
-                    for h in range(2):
-                        tf.tf_argmax_rows(y[h][:M], segs[h][0][0], words[h], scratch, stream=stream)
-                    tf.tf_pick(words, ids[:M], stream=stream)
             flush.zero_()
             for r in range(max(3, args.warmup)):
                 rep(r)
@@ -472,16 +517,21 @@ def run_sweep(args):
             flops = 2.0 * M * K * N
             t_hbm, t_tc = nbytes / (peak_hbm * 1e3), flops / (peak_tc * 1e6)   # microseconds
             bound = "hbm" if t_hbm >= t_tc else "tensor"
-            print(json.dumps({
+            pt = {
                 "sweep": name, "M": M, "K": K, "rows": N, "reps": args.reps, "us_per_rep": round(us, 3),
                 "GB/s": round(nbytes / us / 1e3, 1), "TFLOP/s": round(flops / us / 1e6, 2),
                 "hbm_frac": round(nbytes / us / 1e3 / peak_hbm, 4), "tensor_frac": round(flops / us / 1e6 / peak_tc, 4),
                 "bound": bound, "roofline_frac": round(max(t_hbm, t_tc) / us, 4),
                 "peaks": {"hbm_gbs": peak_hbm, "bf16_tflops": peak_tc, "kind": f"{hbm_kind}/{tc_kind}"},
                 "weight_replicas": nrep, "l2": "replicas span 3 x L2; L2 flushed between points",
-                "clocks": sampler.summary()}), flush=True)
+                "clocks": sampler.summary()}
+            points.append(pt)
+            print(json.dumps(pt), flush=True)
         del replicas, w, x, y
         torch.cuda.empty_cache()
+    if args.sweep_json:
+        with open(args.sweep_json, "w") as f:
+            json.dump({"gpu": torch.cuda.get_device_name(0), "points": points}, f, indent=1)
     return 0
 
 
@@ -502,6 +552,7 @@ def main():
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--shapes", default="", help="sweep: comma-separated subset of " + ",".join(SWEEP_SHAPES))
     ap.add_argument("--sweep-m", default="", help="sweep: comma-separated M values")
+    ap.add_argument("--sweep-json", default="", help="sweep: also write every point to this JSON file")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
     if args.impl == "reference":
@@ -542,20 +593,34 @@ def main():
     barrier()
 
     K = args.steps
-    lm_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-             for _ in range(2)]
-    hd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def ev_pair():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    t0, t1 = ev_pair()
     sampler = ClockSampler(local)
     barrier()
     with sampler:
+        # 1. the whole step, K times back to back
         t0.record(stream)
         for i in range(K):
-            step.run(stream, lm_events=[lm_ev[0][i], lm_ev[1][i]], head_events=hd_ev[i])
+            step.run(stream)
         t1.record(stream)
         barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    lm_ms = [a.elapsed_time(b) for h in range(2) for (a, b) in lm_ev[h]]
+        elapsed_ms = t0.elapsed_time(t1)
+        # 2. the head chain of each step (both halves' qmm + argmax word, the pick)
+        hd_ev = [ev_pair() for _ in range(K)]
+        for i in range(K):
+            step.run(stream, head_events=hd_ev[i])
+        barrier()
+        # 3. one lm_head half's qmm alone, halves alternating
+        lm_ev = [ev_pair() for _ in range(K)]
+        for i in range(K):
+            lm_ev[i][0].record(stream)
+            step.lm_head_half(i % 2, stream)
+            lm_ev[i][1].record(stream)
+        barrier()
+    lm_ms = [a.elapsed_time(b) for (a, b) in lm_ev]
     head_ms = [a.elapsed_time(b) for (a, b) in hd_ev]
 
     # end to end through the public API: pinned host inputs in, result out, every step
@@ -600,19 +665,24 @@ def main():
         lm_bytes = qmm_bytes(5120, 248320 // 2)
         lm_avg_ms = statistics.fmean(lm_ms)
         achieved = lm_bytes / (lm_avg_ms / 1e3) / 1e9
-        src = os.path.join(ROOT, "row_split_int4_b200", "csrc", "qmm_stream.cu")
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": 1, "bytes_per_step": nb["total"],
                        "l2": "no flush: inputs larger than L2 (866 MB of weights per step vs 126 MB L2)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "one GPU, two row halves"},
+                       "parallelism": f"replicas x{world}" if world > 1 else "one GPU, two row halves",
+                       "timed_regions": "value: K steps between two events; head: event pair per step around "
+                                        "both fused halves and the pick; roofline: K lone lm_head-half qmm "
+                                        "launches, each in an event pair"},
+            "step_hbm_frac": {"measured": round(value / peak, 4), "spec_8000": round(value / SPEC_HBM_GBS, 4),
+                              "peak_kind": peak_kind},
             "lm_head_argmax_us_per_token": round(statistics.fmean(head_ms) * 1e3, 2),
             "tokens_per_s_equiv": round(1e3 / ms_step, 1),
             "roofline": {"bound": "hbm", "kernel": "qmm_m1_tile_kernel (lm_head half, 124,160 x 5,120)",
                          "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": traffic_from_profiles(src),
+                         "frac": round(achieved / peak, 4), "frac_spec_8000": round(achieved / SPEC_HBM_GBS, 4),
+                         "traffic": traffic_from_profiles(),
                          "bytes_per_launch": lm_bytes, "avg_launch_us": round(lm_avg_ms * 1e3, 3)},
             "gpu_launches": step.launches_per_step * K,
             "clocks": sampler.summary(),

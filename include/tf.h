@@ -27,6 +27,13 @@
  *    which is a result, not a refusal (see tf_gather_rows).
  *  - No entry point exits, aborts, traps or prints.  A failed launch returns
  *    TF_E_CUDA (the CUDA error is left for cudaGetLastError to report).
+ *  - Kernels are launched with programmatic dependent launch: a kernel may
+ *    be scheduled while the kernel before it on the stream still runs, and
+ *    waits (griddepcontrol.wait) for that kernel to finish before it reads
+ *    any of its arguments' arrays or writes any output.  Before that wait it
+ *    only asks for weight bytes to be brought into L2, which cannot observe
+ *    stale data, so callers see plain stream order.  Setting the environment
+ *    variable TF_PDL=0 before the first call launches without it.
  *  - Outputs must not overlap inputs.
  */
 #ifndef TF_H
@@ -202,10 +209,10 @@ tf_status tf_qmm8_rows(const void *x, int M, int K, int ldx, const int8_t *q8, c
  * slice (tf_qmm_rows, TF_EPI_NONE, one segment) and their argmax word
  * (tf_argmax_rows over those logits with ids id_base + j).  The step-1 body of
  * TensorFold PR #1433 has each rank compute its half of the lm_head and then
- * pair_argmax over it; here, at M = 1, the qmm's warps keep the best key of the
- * rows they write and the kernel's last CTA to finish combines them (a 4-byte
- * asynchronous memset clears its counter first), so the argmax needs neither a
- * pass over the logits nor a second kernel.  The results are bit for bit those of the two separate
+ * pair_argmax over it; here, at M = 1, every warp of the qmm keeps the best key
+ * of the rows it writes and leaves it in scratch, and one single-CTA kernel
+ * combines those keys into the word, so the argmax makes no pass over the
+ * logits.  The results are bit for bit those of the two separate
  * calls: the logits equal tf_qmm_rows' and the word equals tf_argmax_rows' on
  * them.  For M > 1, or a weight layout the M = 1 streaming kernel does not take,
  * the same two kernels run one after the other.
@@ -330,8 +337,12 @@ tf_status tf_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out
  *   - TF_E_ARG when tf_argmax_scratch_bytes(M, n) > TF_STATIC_SCRATCH_BYTES
  *     (for example M = 8,193 rows of any length); nothing is enqueued.
  *   - The first call on a device looks up that array's device address
- *     (cudaGetSymbolAddress, with the device current) and keeps it; make that
- *     first call before any stream capture.  A failed lookup returns TF_E_CUDA.
+ *     (cudaGetSymbolAddress, with the device current) and keeps it, with the
+ *     id of the CUDA context it belongs to; make that first call before any
+ *     stream capture.  After cudaDeviceReset (or any other teardown of the
+ *     context) the next call finds a new context id and looks the address up
+ *     again, so a stale address is never used.  A failed lookup returns
+ *     TF_E_CUDA.
  *   - Every call on a device uses the same array, and the array keeps what the
  *     last call left there.  Each call writes every entry it later reads, so no
  *     clearing is needed, but two calls whose kernels overlap on the GPU (other

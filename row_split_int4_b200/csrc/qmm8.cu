@@ -9,8 +9,11 @@
 //     exact for every x within 2^15 of the lane-chunk's largest), three dp4a
 //     per four codes, the integer sum scaled by the exact power of two; lanes
 //     add their lane-chunks in K order, a fixed shuffle tree joins the lanes,
-//     and the row scale multiplies the total.  The order of every operation
-//     depends on K alone, so split == whole bit for bit.
+//     and the row scale multiplies the total.  A lane-chunk with a nonzero x
+//     more than 2^15 below its largest keeps its raw x and is taken by the
+//     whole warp in fp32 (lane j forms x_j q_j, exact, a fixed butterfly adds
+//     them), so small x are never rounded to the largest one's precision.  The
+//     order of every operation depends on K alone, so split == whole bit for bit.
 //   * M > 1, or K / pointers the streaming kernel does not take: one warp per
 //     output row and activation row, fp32 products of the bf16 x and the code,
 //     a per-lane sum over K in order and the same shuffle tree.
@@ -69,6 +72,8 @@ __global__ void __launch_bounds__(k8MaxWarps * 32, 1) qmm8_m1_stream_kernel(Qmm8
     const Stream8Layout L = stream8_layout(a.K, W, kRU);
     const int K = a.K, nch = L.nch;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     uint8_t *limbs = smem + L.limb_off;
     float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
     uint8_t *ring = smem + L.ring_off + (size_t)warp * kStages * kSlotBytes;
@@ -141,24 +146,26 @@ __global__ void __launch_bounds__(k8MaxWarps * 32, 1) qmm8_m1_stream_kernel(Qmm8
         const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
         const int emax = __reduce_max_sync(0xFFFFFFFFu, M != 0 ? e : 0);
         const int sh = e - emax + 15;
-        int F;
-        if (sh >= 0) {
-            F = M << sh;
-        } else if (sh > -9) {
-            const int d = -sh;
-            F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
-        } else {
-            F = 0;
-        }
+        // wide: a nonzero x more than 2^15 below the largest, which fixed point would
+        // round; such a lane-chunk keeps its raw x and is taken in fp32 below
+        const bool wide = !bad && __any_sync(0xFFFFFFFFu, sh < 0 && M != 0);
+        int F = sh >= 0 ? M << sh : 0;
         if (h & 0x8000u) F = -F;
         if (bad) F = 0;
         const int w = lane >> 2, byte = lane & 3;   // element `lane` of the lane-chunk: word w, byte j
-        uint8_t *base = limbs + ((size_t)(c * k8LaneVecs) * 32 + l) * 16 + (w & 3) * 4 + byte;
+        uint8_t *lcb = limbs + ((size_t)(c * k8LaneVecs) * 32 + l) * 16;
+        if (wide) {
+            // value j in 16-byte vector j / 8 of the lane-chunk
+            reinterpret_cast<uint16_t *>(lcb + (size_t)(lane >> 3) * 32 * 16)[lane & 7] = (uint16_t)h;
+        } else {
+            uint8_t *base = lcb + (w & 3) * 4 + byte;
 #pragma unroll
-        for (int lb = 0; lb < 3; ++lb) base[(size_t)(lb * 2 + (w >> 2)) * 32 * 16] = (uint8_t)((F >> (8 * lb)) & 0xFF);
+            for (int lb = 0; lb < 3; ++lb) base[(size_t)(lb * 2 + (w >> 2)) * 32 * 16] = (uint8_t)((F >> (8 * lb)) & 0xFF);
+        }
         if (lane == 0)
             Ss[lc] = bad ? __int_as_float(0x7FC00000)
-                         : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
+                         : (wide ? __int_as_float(0x80000000)
+                                 : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149)));
       }
     }
     __syncthreads();
@@ -174,15 +181,34 @@ __global__ void __launch_bounds__(k8MaxWarps * 32, 1) qmm8_m1_stream_kernel(Qmm8
         const bool ok = __all_sync(0xFFFFFFFFu, wait_slot(bar0 + 8 * slot, par, failed ? 64 : k8SpinLimit));
         failed = failed || !ok;
         const uint8_t *sl = ring + slot * kSlotBytes;
-        if (j * k8KS + lane * 32 < K) {   // lanes past the end of a short last step idle
+        // lanes past the end of a short last step idle; a wide lane-chunk (scale -0)
+        // adds nothing here and is taken element by element below
+        const bool live = j * k8KS + lane * 32 < K;
+        const float scale = live ? Ss[j * 32 + lane] : 0.0f;
+        const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && __float_as_uint(scale) == 0x80000000u);
+        if (live) {
             uint4 lm[k8LaneVecs];
 #pragma unroll
             for (int q = 0; q < k8LaneVecs; ++q) lm[q] = limb_l[(j * k8LaneVecs + q) * 32];
-            const float scale = Ss[j * 32 + lane];
 #pragma unroll
             for (int r = 0; r < kRU; ++r) {
                 const uint4 *qp = reinterpret_cast<const uint4 *>(sl + r * k8KS) + 2 * lane;
                 acc[r] += lane_chunk_idot8(qp[0], qp[1], lm, scale);
+            }
+        }
+        for (uint32_t m = wm; m != 0; m &= m - 1) {   // wide lane-chunks, warp-uniform
+            const int l = __ffs(m) - 1;
+            const uint16_t *xv = reinterpret_cast<const uint16_t *>(
+                limbs + ((size_t)(j * k8LaneVecs + (lane >> 3)) * 32 + l) * 16);
+            const float xj = bf16_bits_to_f32(xv[lane & 7]);
+#pragma unroll
+            for (int r = 0; r < kRU; ++r) {
+                // lane t takes code t of the lane-chunk: x q in fp32 (exact), then a
+                // butterfly adds the 32 products in a fixed order
+                float p = xj * (float)reinterpret_cast<const int8_t *>(sl + r * k8KS)[l * 32 + lane];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xFFFFFFFFu, p, o);
+                if (lane == l) acc[r] += p;
             }
         }
         if (++j == nch) {
@@ -220,6 +246,8 @@ __global__ void __launch_bounds__(k8MaxWarps * 32, 1) qmm8_m1_stream_kernel(Qmm8
 // column and activation row; lanes take every 32nd k, add in K order, the same
 // shuffle tree joins them, the row scale multiplies the total.
 __global__ void qmm8_generic_kernel(Qmm8Args a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long ntask = (long long)a.M * a.seg.ncols;
@@ -258,8 +286,7 @@ static cudaError_t launch_q8(const Qmm8Args &a, int ri, cudaStream_t stream) {
     int blocks = num_sms();
     const int need = (units + W - 1) / W;
     if (need < blocks) blocks = need;
-    qmm8_m1_stream_kernel<RU><<<blocks, W * 32, L.total, stream>>>(a, units);
-    return cudaGetLastError();
+    return launch_pdl(qmm8_m1_stream_kernel<RU>, dim3(blocks), dim3(W * 32), L.total, stream, a, units);
 }
 
 cudaError_t launch_qmm8(const Qmm8Args &a, cudaStream_t stream) {
@@ -276,8 +303,7 @@ cudaError_t launch_qmm8(const Qmm8Args &a, cudaStream_t stream) {
     long long blocks = ((long long)a.M * a.seg.ncols + 7) / 8;
     if (blocks > num_sms() * 16) blocks = num_sms() * 16;
     if (blocks < 1) blocks = 1;
-    qmm8_generic_kernel<<<(int)blocks, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(qmm8_generic_kernel, dim3((int)blocks), dim3(256), 0, stream, a);
 }
 
 }  // namespace tf

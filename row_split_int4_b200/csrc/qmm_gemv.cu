@@ -9,10 +9,11 @@
 // bits -- PR #1433 review, "a different sk is a different fp32 order"):
 //   * K is cut into chunks of 1024; in chunk c lane l owns the 32 consecutive
 //     k in [1024c + 32l, +32), which lie inside group 16c + l/2.
-//   * The lane forms P = sum of q_k x_k over its 32 k with two fp32
-//     accumulators (even / odd k, ascending), P = P_even + P_odd, and adds
-//     s*P then b*X, X = the ascending fp32 sum of the same 32 x_k
-//     (w = s q + b, so x.w over the 32 k is s*P + b*X).
+//   * The lane forms sum of x_k w_k over its 32 k, w_k = s q_k + b in fp32,
+//     with two fp32 accumulators (even / odd k, ascending) added at the end,
+//     and adds that to its running sum.  (The streaming M = 1 kernels of
+//     qmm_stream.cu take the same lane-chunks, lanes and tree with exact
+//     integer dot products instead.)
 //   * The lane's running sum goes over the chunks in ascending c; the 32 lane
 //     sums are then added by a shfl_down tree (16, 8, 4, 2, 1) and lane 0's
 //     total is rounded to bf16.
@@ -45,7 +46,7 @@ __device__ __forceinline__ uint32_t ld_stream_u16(const uint16_t *p) {
 // M = 1.  x is staged once per CTA into shared memory as fp32, permuted so that
 // the float4 holding elements 4j..4j+3 of lane l's 32 in chunk c sits at
 // float4 index (c*8 + j)*32 + l: a warp's 128-bit reads are conflict-free.
-// Positions past K are zero.  The per-lane-chunk x sums X follow at the end.
+// Positions past K are zero.
 // Each warp walks its own contiguous range of row groups (kSlots rows each);
 // the (group, chunk) pairs form one sequence and the codes of step t+1 are
 // loaded while step t computes.
@@ -56,11 +57,12 @@ struct StepLoad {
 };
 
 __global__ void __launch_bounds__(kWarps * 32, 2) qmm_m1_kernel(QmmArgs a, int units) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(16) float smem[];
     const int K = a.K;
     const int nch = (K + kChunk - 1) / kChunk;
     float4 *xs = reinterpret_cast<float4 *>(smem);
-    float *Xs = smem + nch * kChunk;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // stage x (row 0) into the permuted fp32 layout
@@ -69,14 +71,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2) qmm_m1_kernel(QmmArgs a, int u
         if (k < K) v = bf16_bits_to_f32(a.x[k]);
         const int c = k / kChunk, r = k % kChunk, l = r / 32, e = r % 32;
         smem[(((c * 8 + e / 4) * 32 + l) << 2) + (e & 3)] = v;
-    }
-    __syncthreads();
-    for (int lc = tid; lc < nch * 32; lc += blockDim.x) {
-        const int c = lc / 32, l = lc % 32;
-        float4 xv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xv[j] = xs[(c * 8 + j) * 32 + l];
-        Xs[lc] = lane_chunk_xsum(xv);
     }
     __syncthreads();
 
@@ -149,13 +143,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) qmm_m1_kernel(QmmArgs a, int u
         float4 xv[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) xv[j] = xs[(c * 8 + j) * 32 + lane];
-        const float X = Xs[c * 32 + lane];
 #pragma unroll
-        for (int s = 0; s < kSlots; ++s) {
-            const float P = lane_chunk_dot(cur.q[s], xv);
-            acc[s] = fmaf(bf16_bits_to_f32(cur.s[s]), P, acc[s]);
-            acc[s] = fmaf(bf16_bits_to_f32(cur.b[s]), X, acc[s]);
-        }
+        for (int s = 0; s < kSlots; ++s)
+            acc[s] += lane_chunk_wdot(cur.q[s], xv, bf16_bits_to_f32(cur.s[s]), bf16_bits_to_f32(cur.b[s]));
 
         if (c == nch - 1) {
             // unit u complete: reduce and store
@@ -217,6 +207,8 @@ __device__ __forceinline__ void load_x_lane(const uint16_t *xrow, int k0, int K,
 }
 
 __global__ void __launch_bounds__(kWarps * 32) qmm_generic_kernel(QmmArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
     const int nw = gridDim.x * kWarps;
@@ -237,14 +229,12 @@ __global__ void __launch_bounds__(kWarps * 32) qmm_generic_kernel(QmmArgs a) {
                 if (kk >= K) continue;
                 const int g = kk / kGroup;
                 float4 xv[kMT][8];
-                float X[kMT];
 #pragma unroll
                 for (int i = 0; i < kMT; ++i) {
                     if (m0 + i < a.M) load_x_lane(a.x + (size_t)(m0 + i) * a.ldx, kk, K, xv[i]);
                     else
 #pragma unroll
                         for (int j = 0; j < 8; ++j) xv[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    X[i] = lane_chunk_xsum(xv[i]);
                 }
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -254,11 +244,7 @@ __global__ void __launch_bounds__(kWarps * 32) qmm_generic_kernel(QmmArgs a) {
                     const float s = bf16_bits_to_f32(a.scales[n * G + g]);
                     const float b = bf16_bits_to_f32(a.biases[n * G + g]);
 #pragma unroll
-                    for (int i = 0; i < kMT; ++i) {
-                        const float P = lane_chunk_dot(q, xv[i]);
-                        acc[r][i] = fmaf(s, P, acc[r][i]);
-                        acc[r][i] = fmaf(b, X[i], acc[r][i]);
-                    }
+                    for (int i = 0; i < kMT; ++i) acc[r][i] += lane_chunk_wdot(q, xv[i], s, b);
                 }
             }
 #pragma unroll
@@ -307,7 +293,7 @@ int num_sms() {
 
 size_t qmm_m1_smem_bytes(int K) {
     const int nch = (K + kChunk - 1) / kChunk;
-    return (size_t)nch * kChunk * sizeof(float) + (size_t)nch * 32 * sizeof(float);
+    return (size_t)nch * kChunk * sizeof(float);
 }
 
 constexpr size_t kM1SmemMax = 200 * 1024;
@@ -330,13 +316,11 @@ cudaError_t launch_qmm(const QmmArgs &a, cudaStream_t stream) {
         int blocks = num_sms() * blocks_per_sm;
         const int need = (units + kWarps - 1) / kWarps;
         if (need < blocks) blocks = need;
-        qmm_m1_kernel<<<blocks, kWarps * 32, smem, stream>>>(a, units);
-        return cudaGetLastError();
+        return launch_pdl(qmm_m1_kernel, dim3(blocks), dim3(kWarps * 32), smem, stream, a, units);
     }
     int blocks = (ncols + kWarps - 1) / kWarps;
     blocks = min(blocks, num_sms() * 8);
-    qmm_generic_kernel<<<blocks, kWarps * 32, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(qmm_generic_kernel, dim3(blocks), dim3(kWarps * 32), 0, stream, a);
 }
 
 }  // namespace tf

@@ -18,19 +18,32 @@
 //
 // Exact integer dot (per lane-chunk: the 32 x a lane meets in one 1,024-K chunk).
 // The 32 bf16 x are put in fixed point with the chunk's own exponent E (every
-// |x| < 2^E, E the smallest such over the chunk): F = RN(x * 2^(23-E)), |F| < 2^23, which is
-// exact for every x within 2^15 of the chunk's largest magnitude (smaller ones
-// are rounded to 2^(E-24), far below the bf16 resolution of any output).  F is
-// kept as three bytes, F = L2*2^16 + L1*2^8 + L0 (L2 signed), and
-//     P = sum q_k F_k = 2^16 sum q L2 + 2^8 sum q L1 + sum q L0
-// with three int32 dp4a accumulators that cannot overflow (32 * 15 * 255 < 2^17).
-// The lane then adds s * 2^(E-23) * P and b * X (X = the fp32 sum of the same 32
-// x) to its running sum; w = s q + b, so those two terms are the chunk's x.w.
+// |x| < 2^E, E the smallest such over the chunk): F = x * 2^(23-E), |F| < 2^23,
+// exact for every x within 2^15 of the chunk's largest magnitude.  F is kept as
+// three bytes, F = L2*2^16 + L1*2^8 + L0 (L2 signed), and with the code written
+// as q = (q - 8) + 8 and the weight as w = s (q - 8) + (b + 8 s),
+//     P' = sum (q - 8) F = 2^16 sum q L2 + 2^8 sum q L1 + sum q L0 - 8 sum F
+// comes from three int32 dp4a accumulators that cannot overflow (32 * 15 * 255 <
+// 2^17); |P'| < 2^31, so P' is exact in int32 and is rounded once to fp32.  The
+// lane adds s * 2^(E-23) * P' and (b + 8 s) * X, X = 2^(E-23) sum F = the exact
+// sum of the 32 x rounded once.  Taking the code about its middle keeps the two
+// terms near the size of their sum for the usual bias b ~ -8 s, where s q and b
+// alone would be large terms that cancel.
+// A lane-chunk holding a nonzero x more than 2^15 below its largest ("wide":
+// fixed point would round it) keeps its 32 raw x instead of limbs, and the warp
+// takes it element by element: lane j forms w_j = s q_j + b and x_j w_j in fp32,
+// a fixed butterfly adds the 32 products, and the owning lane adds the sum -- a
+// plain fp32 dot for that lane-chunk, whose value does not depend on how far
+// below the largest x the others lie.
 // A chunk holding NaN or +-Inf gets the scale NaN, so the row's result is NaN.
 //
-// Order of every operation depends on K alone (chunks ascending, per-lane
-// sums, the shuffle tree of qmm_gemv.cu), never on the rows a launch covers:
-// split == whole holds bit for bit.
+// Order of every operation depends on K alone, never on the rows a launch
+// covers, so split == whole holds bit for bit.  K is cut into slices of chunks
+// (slice_chunks: the whole K up to 8 chunks, else 4 chunks = 4,096 K, the last
+// one shorter); over a slice each lane adds its lane-chunks' terms in ascending
+// chunk order, the shuffle tree of qmm_gemv.cu joins the 32 lanes, and the row
+// total is the slices' sums added in ascending order.  A slice is the unit in
+// which the narrow-call kernel below shares a row's K among warps.
 //
 // Slot (kRU rows x kKS values of K):
 //   [codes of row 0 (kKS/2 B)] .. [codes of row kRU-1] [scales, kKS/32 B per row] [biases]
@@ -55,7 +68,7 @@ constexpr long long kSpinLimit = 1ll << 22;                  // bounded waits, s
 
 struct StreamLayout {
     int nch, warps;
-    size_t limb_off, X_off, scale_off, bar_off, ring_off, total;
+    size_t limb_off, sf_off, scale_off, bar_off, ring_off, total;
 };
 
 __host__ __device__ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -66,18 +79,19 @@ __host__ __device__ inline StreamLayout stream_layout(int K, int warps, int ru) 
     L.nch = (K + kChunk - 1) / kChunk;
     L.warps = warps;
     L.limb_off = 0;
-    L.X_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.X_off + (size_t)L.nch * 32 * 4, 128);
+    L.sf_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
+    L.scale_off = round_up(L.sf_off + (size_t)L.nch * 32 * 4, 128);
     L.bar_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
     L.ring_off = round_up(L.bar_off + (size_t)warps * stages_for(ru) * 8, 128);
     L.total = L.ring_off + (size_t)warps * stages_for(ru) * slot_bytes(ru);
     return L;
 }
 
-// sum over the lane's 32 codes of q_k * F_k, as a float.  limb[j] (j = limb*2 +
-// parity) holds in word w the limb bytes of x[8w+p], x[8w+p+2], x[8w+p+4], x[8w+p+6];
-// the even codes of word w are its low nibbles, the odd codes its high nibbles.
-__device__ __forceinline__ float lane_chunk_idot(const uint4 &q, const uint4 *limb) {
+// P' = sum over the lane's 32 codes of (q_k - 8) F_k, exact (see above); sf8 = 8 sum F.
+// limb[j] (j = limb*2 + parity) holds in word w the limb bytes of x[8w+p],
+// x[8w+p+2], x[8w+p+4], x[8w+p+6]; the even codes of word w are its low nibbles,
+// the odd codes its high nibbles.
+__device__ __forceinline__ int lane_chunk_pq(const uint4 &q, const uint4 *limb, uint32_t sf8) {
     int a0 = 0, a1 = 0, a2 = 0;
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
     const uint32_t *L = reinterpret_cast<const uint32_t *>(limb);
@@ -92,17 +106,64 @@ __device__ __forceinline__ float lane_chunk_idot(const uint4 &q, const uint4 *li
         a2 = dp4a_us(ue, L[4 * 4 + w], a2);
         a2 = dp4a_us(uo, L[5 * 4 + w], a2);
     }
-    return fmaf((float)a2, 65536.0f, fmaf((float)a1, 256.0f, (float)a0));
+    // modulo 2^32; the true value fits int32, so the wrap-around is exact
+    return (int)(((uint32_t)a2 << 16) + ((uint32_t)a1 << 8) + (uint32_t)a0 - sf8);
+}
+
+// What a lane needs of its lane-chunk c: limbs, the scale 2^(E-23) (-0 marks a
+// wide lane-chunk, NaN a non-finite x), X and 8 sum F.
+struct LaneChunk {
+    uint4 lm[6];
+    float scale, X;
+    uint32_t sf8;
+    bool wide;
+};
+__device__ __forceinline__ void load_lane_chunk(LaneChunk &t, const uint4 *limb_l, const int *SFs, const float *Ss,
+                                                int c, int lane) {
+#pragma unroll
+    for (int q = 0; q < 6; ++q) t.lm[q] = limb_l[(c * 6 + q) * 32];
+    const int sf = SFs[c * 32 + lane];
+    t.scale = Ss[c * 32 + lane];
+    t.X = __int2float_rn(sf) * t.scale;   // one rounding, then an exact power of two
+    t.sf8 = (uint32_t)sf << 3;
+    t.wide = __float_as_uint(t.scale) == 0x80000000u;
+}
+
+// acc += the lane's x.w over lane-chunk t for a row with codes qv, scale s, bias b
+// (a wide lane-chunk has scale and X zero here and adds nothing).
+__device__ __forceinline__ float lane_chunk_fma(float acc, const uint4 &qv, const LaneChunk &t, float s, float b) {
+    const int P = lane_chunk_pq(qv, t.lm, t.sf8);
+    acc = fmaf(s, __int2float_rn(P) * t.scale, acc);   // P' * 2^(E-23): exact power-of-two scaling
+    return fmaf(fmaf(8.0f, s, b), t.X, acc);            // b + 8 s
+}
+
+// Element `lane` of the wide lane-chunk (c, l), from the raw bf16 x it keeps in
+// place of its limbs (value j in 16-byte vector j / 8 of the lane-chunk).
+__device__ __forceinline__ float wide_x(const uint8_t *limbs, int c, int l, int lane) {
+    const uint16_t *v = reinterpret_cast<const uint16_t *>(limbs + ((size_t)(c * 6 + (lane >> 3)) * 32 + l) * 16);
+    return bf16_bits_to_f32(v[lane & 7]);
+}
+
+// The x.w of a wide lane-chunk for one row, lane j taking element j: word = code
+// word j / 8 of the lane-chunk, s and b its group's scale and bias.  w = s q + b
+// and x w in fp32, then a butterfly over the warp adds the 32 products (every
+// lane ends with the same sum, so the order is fixed).
+__device__ __forceinline__ float wide_dot(float xj, uint32_t word, int lane, float s, float b) {
+    const float q = (float)((word >> (4 * (lane & 7))) & 15u);
+    float p = xj * fmaf(s, q, b);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xFFFFFFFFu, p, o);
+    return p;
 }
 
 // Fixed-point limbs of x for every lane-chunk, on the bf16 fields alone: x = sign *
 // M * 2^(e-134), M = 128 + mantissa (e >= 1) or the mantissa (e = 0, subnormal, read
-// with e = 1).  With emax
-// the chunk's largest e, F = x * 2^(23-E), E = emax - 126, is sign * M * 2^(e - emax
-// + 15): a left shift when e >= emax - 15 (exact), else a right shift rounded to
-// nearest even.  Xs gets the fp32 sum of the chunk's 32 x, Ss the power of two
-// 2^(E-23) (NaN when the chunk holds a NaN or an infinity).
-__device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, float *Xs, float *Ss, int W,
+// with e = 1).  With emax the chunk's largest e, F = x * 2^(23-E), E = emax - 126,
+// is sign * M * 2^(e - emax + 15), a left shift when e >= emax - 15 (exact).  A
+// lane-chunk with a nonzero x below that is wide: its 32 raw x go where its limbs
+// would, its scale is -0 and its sum 0.  SFs gets sum F (|sum F| < 2^28), Ss the
+// power of two 2^(E-23) (NaN when the chunk holds a NaN or an infinity).
+__device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, int *SFs, float *Ss, int W,
                                            int warp, int lane) {
     // one thread per lane-chunk, all of it in registers: no cross-lane step, so
     // the whole CTA prepares up to W * 32 lane-chunks in one pass
@@ -144,6 +205,8 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
         for (int q = 0; q < 6; ++q)
 #pragma unroll
             for (int w = 0; w < 4; ++w) L[q][w] = 0u;
+        bool wide = false;
+        int sf = 0;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
@@ -151,98 +214,116 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             const int e = ef == 0 ? 1 : (int)ef;
             const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
             const int sh = e - emax + 15;
-            int F;
-            if (sh >= 0) {
-                F = M << sh;
-            } else if (sh > -9) {
-                const int d = -sh;
-                F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
-            } else {
-                F = 0;
-            }
+            wide = wide || (sh < 0 && M != 0);
+            int F = sh >= 0 ? M << sh : 0;
             if (h & 0x8000u) F = -F;
-            if (bad) F = 0;
+            sf += F;
             // value t of the lane-chunk: word t >> 3, byte (t & 7) >> 1 of limb vector 2 limb + (t & 1)
             const int w = t >> 3, p = t & 1, sft = 8 * ((t & 7) >> 1);
             L[0 + p][w] |= (uint32_t)(F & 0xFF) << sft;
             L[2 + p][w] |= (uint32_t)((F >> 8) & 0xFF) << sft;
             L[4 + p][w] |= (uint32_t)((F >> 16) & 0xFF) << sft;
         }
+        wide = wide && !bad;
         uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
+        if (wide) {
 #pragma unroll
-        for (int q = 0; q < 6; ++q) dst[q * 32] = make_uint4(L[q][0], L[q][1], L[q][2], L[q][3]);
-        // sum of the 32 x in the pairing of a five-step warp shuffle tree
-        float sx[16];
+            for (int q = 0; q < 4; ++q) dst[q * 32] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            sx[i] = bf16_bits_to_f32(hv[i >> 1] >> (16 * (i & 1)) & 0xFFFFu) +
-                    bf16_bits_to_f32(hv[(i + 16) >> 1] >> (16 * (i & 1)) & 0xFFFFu);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1)
-#pragma unroll
-            for (int i = 0; i < o; ++i) sx[i] += sx[i + o];
-        Xs[lc] = sx[0];
+            for (int q = 0; q < 6; ++q) dst[q * 32] = make_uint4(L[q][0], L[q][1], L[q][2], L[q][3]);
+        }
+        SFs[lc] = bad || wide ? 0 : sf;
         // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
-        Ss[lc] = bad ? __int_as_float(0x7FC00000) : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
+        Ss[lc] = bad ? __int_as_float(0x7FC00000)
+                     : (wide ? __int_as_float(0x80000000)
+                             : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149)));
     }
 }
 
-// Fused head: every warp publishes the largest argmax key of the rows it wrote;
-// the last CTA to finish (a fence, then a ticket: the usual last-block pattern)
-// reduces all of them into the argmax word and clears the ticket counter.
-__device__ __forceinline__ void fused_head_tail(const QmmArgs &a, uint64_t best, int W, int tid, int warp, int lane) {
+// Fused head: every warp of the grid publishes the largest argmax key of the rows
+// it wrote (0 when it wrote none); argmax_keys_kernel turns them into the word.
+__device__ __forceinline__ void fused_head_keys(const QmmArgs &a, uint64_t best, int W, int warp, int lane) {
     if (lane == 0) a.cand[(long long)blockIdx.x * W + warp] = best;
-    __threadfence();
+}
+
+// The word of one slice from the qmm grid's ncand warp keys: max over them (the
+// argmax order is the keys' unsigned order, so any tree gives the same key), the
+// winning value read back from the logits.  One CTA.
+__global__ void __launch_bounds__(1024) argmax_keys_kernel(const uint64_t *cand, int ncand, const uint16_t *logits,
+                                                           uint32_t id_base, uint64_t *word) {
+    pdl_trigger();
+    pdl_wait();
+    uint64_t v = 0;
+    for (int i = threadIdx.x; i < ncand; i += blockDim.x) v = umax64(v, cand[i]);
+    v = warp_max64(v);
+    __shared__ uint64_t red[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
     __syncthreads();
-    __shared__ unsigned int ticket;
-    if (tid == 0) ticket = atomicAdd(a.done, 1u);
-    __syncthreads();
-    if (ticket == gridDim.x - 1) {
-        __threadfence();
-        const int ncand = (int)(gridDim.x * W);
-        uint64_t v = 0;
-        for (int i = tid; i < ncand; i += blockDim.x) v = umax64(v, ((volatile uint64_t *)a.cand)[i]);
+    if (warp == 0) {
+        v = lane < (int)(blockDim.x >> 5) ? red[lane] : 0ull;
         v = warp_max64(v);
-        __shared__ uint64_t red[32];
-        if (lane == 0) red[warp] = v;
-        __syncthreads();
-        if (warp == 0) {
-            v = lane < W ? red[lane] : 0ull;
-            v = warp_max64(v);
-            if (lane == 0) {
-                *a.word = word_of_key(v, a.y, a.id_base);
-                *a.done = 0u;
-            }
-        }
+        if (lane == 0) *word = word_of_key(v, logits, id_base);
     }
+}
+
+// Chunks per K-slice (see the reduction order above).
+__host__ __device__ constexpr int slice_chunks(int nch) { return nch <= 8 ? nch : 4; }
+__device__ __forceinline__ bool slice_end(int c, int sc, int nch) { return (c + 1) % sc == 0 || c + 1 == nch; }
+// At the end of a slice: the 32 lanes' sums of the slice by the tree into lane 0,
+// added to the row's total (lane 0's tot; the first slice starts it).
+__device__ __forceinline__ void slice_fold(float &acc, float &tot, int c, int sc) {
+    const float v = warp_sum_to_lane0(acc);
+    tot = c < sc ? v : tot + v;
+    acc = 0.0f;
 }
 
 // acc[r] += the x.w of unit row r over the chunks of one slot: chunk c0 + cc sits
 // at position cc of the slot.  A lane whose 32 values start at or past kend (K
-// covered by the slot) stops there.  Full slots pass compile-time nc and kend, so
-// their bounds fold away.
+// covered by the slot) adds nothing there.  Full slots pass compile-time nc and
+// kend, so their bounds fold away.
 template <int kRU>
-__device__ __forceinline__ void slot_dot(float (&acc)[kRU], const uint8_t *sl, const uint4 *limb_l, const float *Xs,
-                                         const float *Ss, int c0, int nc, int kend, int lane) {
+__device__ __forceinline__ void slot_dot(float (&acc)[kRU], float (&tot)[kRU], const uint8_t *sl, const uint8_t *limbs,
+                                         const int *SFs, const float *Ss, int c0, int nc, int kend, int nch, int sc,
+                                         int lane) {
     const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
-    const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kRU * kSlotQ) + (lane >> 1);
+    const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kRU * kSlotQ);
+    const uint16_t *sc16 = sc0 + (lane >> 1);
+    const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
 #pragma unroll
     for (int cc = 0; cc < kKS / kChunk; ++cc) {
-        if (cc >= nc || cc * kChunk + lane * 32 >= kend) break;
+        if (cc >= nc) break;
         const int c = c0 + cc;
-        uint4 lm[6];
+        const bool live = cc * kChunk + lane * 32 < kend;
+        LaneChunk t;
+        load_lane_chunk(t, limb_l, SFs, Ss, c, lane);
+        const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && t.wide);
+        if (live) {
 #pragma unroll
-        for (int q = 0; q < 6; ++q) lm[q] = limb_l[(c * 6 + q) * 32];
-        const float X = Xs[c * 32 + lane];
-        const float scale = Ss[c * 32 + lane];
+            for (int r = 0; r < kRU; ++r) {
+                const uint4 qv = ql[(r * kSlotQ + cc * (kChunk / 2)) / 16];
+                const float s = bf16_bits_to_f32(sc16[r * (kKS / kGroup) + cc * 16]);
+                const float b = bf16_bits_to_f32(sc16[kRU * (kKS / kGroup) + r * (kKS / kGroup) + cc * 16]);
+                acc[r] = lane_chunk_fma(acc[r], qv, t, s, b);
+            }
+        }
+        for (uint32_t m = wm; m != 0; m &= m - 1) {   // wide lane-chunks, warp-uniform
+            const int l = __ffs(m) - 1;
+            const float xj = wide_x(limbs, c, l, lane);
 #pragma unroll
-        for (int r = 0; r < kRU; ++r) {
-            const uint4 qv = ql[(r * kSlotQ + cc * (kChunk / 2)) / 16];
-            const float s = bf16_bits_to_f32(sc16[r * (kKS / kGroup) + cc * 16]);
-            const float b = bf16_bits_to_f32(sc16[kRU * (kKS / kGroup) + r * (kKS / kGroup) + cc * 16]);
-            const float P = lane_chunk_idot(qv, lm);
-            acc[r] = fmaf(s, P * scale, acc[r]);   // P * 2^(E-23): exact power-of-two scaling
-            acc[r] = fmaf(b, X, acc[r]);
+            for (int r = 0; r < kRU; ++r) {
+                const uint32_t word =
+                    reinterpret_cast<const uint32_t *>(sl)[((r * kSlotQ + cc * (kChunk / 2)) / 16 + l) * 4 + (lane >> 3)];
+                const float s = bf16_bits_to_f32(sc0[r * (kKS / kGroup) + cc * 16 + (l >> 1)]);
+                const float b = bf16_bits_to_f32(sc0[kRU * (kKS / kGroup) + r * (kKS / kGroup) + cc * 16 + (l >> 1)]);
+                const float d = wide_dot(xj, word, lane, s, b);
+                if (lane == l) acc[r] += d;
+            }
+        }
+        if (slice_end(c, sc, nch)) {
+#pragma unroll
+            for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot[r], c, sc);
         }
     }
 }
@@ -260,7 +341,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     const int G = K / kGroup;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *limbs = smem + L.limb_off;
-    float *Xs = reinterpret_cast<float *>(smem + L.X_off);
+    int *SFs = reinterpret_cast<int *>(smem + L.sf_off);
     float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
     uint8_t *ring = smem + L.ring_off + (size_t)warp * kStages * kSlotBytes;
     const uint32_t ring_s = smem_addr(ring);
@@ -327,6 +408,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
         fence_mbar_init();
     }
     __syncwarp();
+    // While the kernel before this one may still run: the warp's first ring of
+    // weights into L2 (never written by the library's kernels; an L2 prefetch
+    // cannot see stale data in any case).
+    {
+        int pu = u0, pj = 0;
+        const uint8_t *psrc = csrc;
+        for (int i = 0; i < kStages && i < steps; ++i) {
+            if (psrc != nullptr)
+                l2_prefetch(psrc + (size_t)pj * piece_full, pj == nsl - 1 ? piece_last : piece_full);
+            if (++pj == nsl) {
+                pj = 0;
+                if (++pu >= u1) break;
+                const int row = copier ? unit_row(pu, my_r) : -1;
+                psrc = row >= 0 ? gbase + (size_t)row * grow : nullptr;
+            }
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
     // Wide units send only their first slot's copies before the limb preparation:
     // with every warp queueing its whole ring at once the copy queue fills and the
     // issuing lanes wait, which would hold the preparation back; the rest follow
@@ -334,17 +434,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     constexpr int kPreStages = kRU >= 4 ? 1 : kStages;
     while (issued < kPreStages && issued < steps) issue_next();
 
-    prep_limbs(a.x, K, nch, limbs, Xs, Ss, W, warp, lane);
+    prep_limbs(a.x, K, nch, limbs, SFs, Ss, W, warp, lane);
     __syncthreads();
     while (issued < kStages && issued < steps) issue_next();
 
-    float acc[kRU];
+    float acc[kRU], tot[kRU];
 #pragma unroll
-    for (int r = 0; r < kRU; ++r) acc[r] = 0.0f;
+    for (int r = 0; r < kRU; ++r) acc[r] = tot[r] = 0.0f;
+    const int sc = slice_chunks(nch);
     uint64_t best = 0;   // fused head: the largest argmax key of the rows this warp wrote
     int slot = 0;
     uint32_t par = 0;
-    const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
     const int nc_last = (len_last + kChunk - 1) / kChunk;
 
     for (int u = u0; u < u1; ++u) {
@@ -353,21 +453,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
             failed = failed || !ok;
             const uint8_t *sl = ring + slot * kSlotBytes;
             if (j + 1 < nsl)
-                slot_dot<kRU>(acc, sl, limb_l, Xs, Ss, j * (kKS / kChunk), kKS / kChunk, kKS, lane);
+                slot_dot<kRU>(acc, tot, sl, limbs, SFs, Ss, j * (kKS / kChunk), kKS / kChunk, kKS, nch, sc, lane);
             else
-                slot_dot<kRU>(acc, sl, limb_l, Xs, Ss, j * (kKS / kChunk), nc_last, len_last, lane);
+                slot_dot<kRU>(acc, tot, sl, limbs, SFs, Ss, j * (kKS / kChunk), nc_last, len_last, nch, sc, lane);
             if (++slot == kStages) {
                 slot = 0;
                 par ^= 1u;
             }
             __syncwarp();
             if (issued < steps && !failed) issue_next();
-        }
-        float tot[kRU];
-#pragma unroll
-        for (int r = 0; r < kRU; ++r) {
-            tot[r] = warp_sum_to_lane0(acc[r]);
-            acc[r] = 0.0f;
         }
         if (lane == 0) {
             if (a.glu) {
@@ -398,7 +492,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     if (failed) {
         for (int s2 = 0; s2 < kStages; ++s2) wait_slot(bar0 + 8 * s2, 0, 1024);
     }
-    if (a.cand) fused_head_tail(a, best, W, tid, warp, lane);
+    if (a.cand) fused_head_keys(a, best, W, warp, lane);
 }
 
 // ---------------------------------------------------------- tile ring --
@@ -434,7 +528,7 @@ constexpr int kTMaxStages = 6;
 
 struct TileLayout {
     int nch, stages;
-    size_t limb_off, X_off, scale_off, full_off, empty_off, hdr_off, ctl_off, ring_off, total;
+    size_t limb_off, sf_off, scale_off, full_off, empty_off, hdr_off, ctl_off, ring_off, total;
 };
 
 __host__ __device__ inline TileLayout tile_layout(int K, int stages) {
@@ -442,8 +536,8 @@ __host__ __device__ inline TileLayout tile_layout(int K, int stages) {
     L.nch = (K + kChunk - 1) / kChunk;
     L.stages = stages;
     L.limb_off = 0;
-    L.X_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.X_off + (size_t)L.nch * 32 * 4, 128);
+    L.sf_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
+    L.scale_off = round_up(L.sf_off + (size_t)L.nch * 32 * 4, 128);
     L.full_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
     L.empty_off = L.full_off + (size_t)kTGroups * stages * 8;
     L.hdr_off = L.empty_off + (size_t)kTGroups * stages * 8;    // (tile, chunk) of each slot
@@ -492,7 +586,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const bool producer = warp >= kTWarps;
     const int grp = producer ? warp - kTWarps : warp / kTGroupWarps, w_in = warp % kTGroupWarps;
     uint8_t *limbs = smem + L.limb_off;
-    float *Xs = reinterpret_cast<float *>(smem + L.X_off);
+    int *SFs = reinterpret_cast<int *>(smem + L.sf_off);
     float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
     int2 *hdr = reinterpret_cast<int2 *>(smem + L.hdr_off) + grp * S;
     int *claim = reinterpret_cast<int *>(smem + L.ctl_off);
@@ -590,12 +684,33 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
     };
 
+    // While the kernel before this one may still run, each producer asks for the
+    // first ring's worth of one of the CTA's first four tiles (the four the groups
+    // claim first) to be brought into L2; weights are never written by a kernel
+    // of the library, and an L2 prefetch cannot see stale data in any case.
+    if (producer && lane == 0 && t0 + grp < t1) {
+        int r_a, r_b, col, ncol;
+        tile_rows(t0 + grp, r_a, r_b, col, ncol);
+        for (int c = 0; c < S && c < nsl; ++c) {
+            const int cq = c * (Sh::q / Sh::qelem), cs = c * (Sh::sb / 2);
+            l2_prefetch_2d(&qmap, cq, r_a);
+            l2_prefetch_2d(&smap, cs, r_a);
+            l2_prefetch_2d(&bmap, cs, r_a);
+            if (kGlu) {
+                l2_prefetch_2d(&qmap, cq, r_b);
+                l2_prefetch_2d(&smap, cs, r_b);
+                l2_prefetch_2d(&bmap, cs, r_b);
+            }
+        }
+    }
+    pdl_wait();
+    pdl_trigger();
     // the whole ring goes out before the limb preparation (one tile-chunk a slot);
     // all warps prepare the limbs, then the producers keep the rings full
     if (producer && lane == 0)
         for (int i = 0; i < S; ++i) issue_next();
     __syncwarp();
-    prep_limbs(a.x, K, nch, limbs, Xs, Ss, kTWarps + kTGroups, warp, lane);
+    prep_limbs(a.x, K, nch, limbs, SFs, Ss, kTWarps + kTGroups, warp, lane);
     __syncthreads();
     if (producer) {
         if (lane == 0)
@@ -603,9 +718,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
         __syncwarp();
     }
 
-    float acc[kWR];
+    float acc[kWR], tot[kWR];
 #pragma unroll
-    for (int r = 0; r < kWR; ++r) acc[r] = 0.0f;
+    for (int r = 0; r < kWR; ++r) acc[r] = tot[r] = 0.0f;
+    const int sc = slice_chunks(nch);
     uint64_t best = 0;
     int slot = 0;
     uint32_t par = 0;
@@ -621,26 +737,45 @@ __global__ void __launch_bounds__(kTThreads, 1)
         if (h.x < 0) break;
         const uint8_t *sl = ring + slot * kTSlotBytes;
         const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
-        const uint16_t *sc16 = reinterpret_cast<const uint16_t *>(sl + kRows * Sh::q) + (lane >> 1);
+        const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kRows * Sh::q);
+        const uint16_t *sc16 = sc0 + (lane >> 1);
 #pragma unroll
         for (int cc = 0; cc < kCps; ++cc) {
             const int c = h.y * kCps + cc;
-            // chunks past K, and lanes past the end of a short last chunk, add nothing
-            if (c >= nch || lane * 32 >= K - c * kChunk) break;
-            uint4 lm[6];
+            if (c >= nch) break;   // chunks past K add nothing
+            // nor do lanes past the end of a short last chunk
+            const bool live = lane * 32 < K - c * kChunk;
+            LaneChunk t;
+            load_lane_chunk(t, limb_l, SFs, Ss, c, lane);
+            const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && t.wide);
+            if (live) {
 #pragma unroll
-            for (int q = 0; q < 6; ++q) lm[q] = limb_l[(c * 6 + q) * 32];
-            const float X = Xs[c * 32 + lane];
-            const float scale = Ss[c * 32 + lane];
+                for (int r = 0; r < kWR; ++r) {
+                    const int R = tile_row<kGlu, kWR>(w_in, r);
+                    const uint4 qv = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
+                    const float s = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+                    const float b = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+                    acc[r] = lane_chunk_fma(acc[r], qv, t, s, b);
+                }
+            }
+            for (uint32_t m = wm; m != 0; m &= m - 1) {   // wide lane-chunks, warp-uniform
+                const int l = __ffs(m) - 1;
+                const float xj = wide_x(limbs, c, l, lane);
 #pragma unroll
-            for (int r = 0; r < kWR; ++r) {
-                const int R = tile_row<kGlu, kWR>(w_in, r);
-                const uint4 qv = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
-                const float s = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
-                const float b = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
-                const float P = lane_chunk_idot(qv, lm);
-                acc[r] = fmaf(s, P * scale, acc[r]);   // P * 2^(E-23): exact power-of-two scaling
-                acc[r] = fmaf(b, X, acc[r]);
+                for (int r = 0; r < kWR; ++r) {
+                    const int R = tile_row<kGlu, kWR>(w_in, r);
+                    const uint32_t word = reinterpret_cast<const uint32_t *>(
+                        sl)[(R * (Sh::q / 16) + cc * (kChunk / 32) + l) * 4 + (lane >> 3)];
+                    const float s = bf16_bits_to_f32(sc0[R * (Sh::sb / 2) + cc * (kChunk / 64) + (l >> 1)]);
+                    const float b =
+                        bf16_bits_to_f32(sc0[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64) + (l >> 1)]);
+                    const float d = wide_dot(xj, word, lane, s, b);
+                    if (lane == l) acc[r] += d;
+                }
+            }
+            if (slice_end(c, sc, nch)) {
+#pragma unroll
+                for (int r = 0; r < kWR; ++r) slice_fold(acc[r], tot[r], c, sc);
             }
         }
         __syncwarp();
@@ -650,12 +785,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
             par ^= 1u;
         }
         if (h.y == nsl - 1) {
-            float tot[kWR];
-#pragma unroll
-            for (int r = 0; r < kWR; ++r) {
-                tot[r] = warp_sum_to_lane0(acc[r]);
-                acc[r] = 0.0f;
-            }
             if (lane == 0) {
                 int r_a, r_b, col, ncol;
                 tile_rows(h.x, r_a, r_b, col, ncol);
@@ -700,7 +829,173 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
         best = cand_key((uint16_t)TF_NAN_BF16, 0u);
     }
-    if (a.cand) fused_head_tail(a, best, kTWarps + kTGroups, tid, warp, lane);
+    if (a.cand) fused_head_keys(a, best, kTWarps + kTGroups, warp, lane);
+}
+
+// ---------------------------------------------------------- narrow calls --
+// A call with a long K (more than 8 chunks) and too few rows for the 16-row tile
+// ring -- down's 2,560-row halves at K = 17,408 -- has about one row per warp of
+// the GPU: a warp per row at the full K would run two rounds on a few warps
+// while the rest idle.  Here each CTA owns a contiguous run of output columns
+// and its warps share the (column, K-slice) pairs of that run, round robin.  A
+// pair is one row over one slice (up to 4,096 K: 2 KB of codes and 128 B each of
+// scales and biases), streamed through the warp's own ring by three 1-D bulk
+// copies (one lane each); the warp leaves the slice's tree sum in shared memory,
+// and once every pair is done each column's slice sums are added in ascending
+// order.  That is the reduction order of every M = 1 kernel (see the top of this
+// file), so the bits are theirs.
+constexpr int kSWarps = 16;
+constexpr int kSStages = 4;
+constexpr int kSItemQ = 4 * kChunk / 2;          // code bytes of one row-slice
+constexpr int kSItemS = 4 * kChunk / 32;         // scale (or bias) bytes of one row-slice
+constexpr int kSSlot = kSItemQ + 2 * kSItemS;    // 2,304
+
+struct SplitLayout {
+    int nch, nsl;
+    size_t limb_off, sf_off, scale_off, part_off, bar_off, ring_off, total;
+};
+
+__host__ __device__ inline SplitLayout split_layout(int K, int maxcols) {
+    SplitLayout L;
+    L.nch = (K + kChunk - 1) / kChunk;
+    L.nsl = (L.nch + 3) / 4;
+    L.limb_off = 0;
+    L.sf_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
+    L.scale_off = round_up(L.sf_off + (size_t)L.nch * 32 * 4, 128);
+    L.part_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
+    L.bar_off = round_up(L.part_off + (size_t)maxcols * L.nsl * 4, 128);
+    L.ring_off = round_up(L.bar_off + (size_t)kSWarps * kSStages * 8, 128);
+    L.total = L.ring_off + (size_t)kSWarps * kSStages * kSSlot;
+    return L;
+}
+
+__global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a, int maxcols) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const SplitLayout L = split_layout(a.K, maxcols);
+    const int K = a.K, nch = L.nch, nsl = L.nsl;
+    const int G = K / kGroup;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t *limbs = smem + L.limb_off;
+    int *SFs = reinterpret_cast<int *>(smem + L.sf_off);
+    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
+    float *part = reinterpret_cast<float *>(smem + L.part_off);
+    uint8_t *ring = smem + L.ring_off + (size_t)warp * kSStages * kSSlot;
+    const uint32_t ring_s = smem_addr(ring);
+    const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kSStages * 8);
+
+    // this CTA's columns and the warp's (column, slice) pairs: i = warp + t * kSWarps
+    const int c0 = (int)((long long)blockIdx.x * a.seg.ncols / gridDim.x);
+    const int c1 = (int)((long long)(blockIdx.x + 1) * a.seg.ncols / gridDim.x);
+    const int nitems = (c1 - c0) * nsl;
+    const int my_items = nitems > warp ? (nitems - warp + kSWarps - 1) / kSWarps : 0;
+
+    // lane 0 copies the codes of a pair, lane 1 its scales, lane 2 its biases
+    auto piece = [&](int t, const uint8_t *&src, uint32_t &bytes, uint32_t &dst_off, uint32_t &tx) {
+        const int i = warp + t * kSWarps;
+        const int col = c0 + i / nsl, j = i % nsl;
+        const int len = min(4 * kChunk, K - j * 4 * kChunk);   // K of the slice (a multiple of 512)
+        const size_t row = (size_t)seg_row(a.seg, col, 0, 0);
+        tx = (uint32_t)(len / 2 + len / 16);
+        if (lane == 0) {
+            src = a.wq + row * (size_t)(K / 2) + (size_t)j * kSItemQ;
+            bytes = (uint32_t)(len / 2);
+            dst_off = 0;
+        } else {
+            const uint16_t *base = lane == 1 ? a.scales : a.biases;
+            src = reinterpret_cast<const uint8_t *>(base + row * (size_t)G + (size_t)j * (4 * kChunk / kGroup));
+            bytes = (uint32_t)(len / 32);
+            dst_off = lane == 1 ? kSItemQ : kSItemQ + kSItemS;
+        }
+    };
+    auto issue = [&](int t) {
+        const int slot = t % kSStages;
+        const uint32_t bar = bar0 + 8 * slot;
+        const uint8_t *src = nullptr;
+        uint32_t bytes = 0, dst_off = 0, tx = 0;
+        piece(t, src, bytes, dst_off, tx);
+        if (lane == 0) mbar_expect_tx(bar, tx);
+        __syncwarp();
+        if (lane < 3) bulk_g2s(ring_s + slot * kSSlot + dst_off, src, bytes, bar);
+    };
+
+    if (lane == 0) {
+        for (int st = 0; st < kSStages; ++st) mbar_init(bar0 + 8 * st, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    // While the kernel before this one may still run: the warp's first pairs into
+    // L2 (weights are never written by the library's kernels; an L2 prefetch cannot
+    // see stale data in any case).
+    if (lane < 3)
+        for (int t = 0; t < kSStages && t < my_items; ++t) {
+            const uint8_t *src = nullptr;
+            uint32_t bytes = 0, dst_off = 0, tx = 0;
+            piece(t, src, bytes, dst_off, tx);
+            l2_prefetch(src, bytes);
+        }
+    pdl_wait();
+    pdl_trigger();
+    for (int t = 0; t < kSStages && t < my_items; ++t) issue(t);
+    prep_limbs(a.x, K, nch, limbs, SFs, Ss, kSWarps, warp, lane);
+    __syncthreads();
+
+    const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
+    bool failed = false;
+    for (int t = 0; t < my_items; ++t) {
+        const int slot = t % kSStages;
+        const bool ok = __all_sync(0xFFFFFFFFu, wait_slot(bar0 + 8 * slot, (uint32_t)((t / kSStages) & 1),
+                                                          failed ? 64 : kSpinLimit));
+        failed = failed || !ok;
+        const int i = warp + t * kSWarps;
+        const int col = c0 + i / nsl, j = i % nsl;
+        const int ch = min(4, nch - 4 * j);
+        const uint8_t *sl = ring + slot * kSSlot;
+        const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kSItemQ);
+        float acc = 0.0f;
+        for (int cc = 0; cc < ch; ++cc) {
+            const int c = 4 * j + cc;
+            const bool live = lane * 32 < K - c * kChunk;   // lanes past the end of a short last chunk add nothing
+            LaneChunk lc;
+            load_lane_chunk(lc, limb_l, SFs, Ss, c, lane);
+            const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && lc.wide);
+            if (live) {
+                const uint4 qv = reinterpret_cast<const uint4 *>(sl)[cc * 32 + lane];
+                const float sv = bf16_bits_to_f32(sc0[cc * 16 + (lane >> 1)]);
+                const float bv = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (lane >> 1)]);
+                acc = lane_chunk_fma(acc, qv, lc, sv, bv);
+            }
+            for (uint32_t m = wm; m != 0; m &= m - 1) {   // wide lane-chunks, warp-uniform
+                const int l = __ffs(m) - 1;
+                const float xj = wide_x(limbs, c, l, lane);
+                const uint32_t word = reinterpret_cast<const uint32_t *>(sl)[(cc * 32 + l) * 4 + (lane >> 3)];
+                const float sv = bf16_bits_to_f32(sc0[cc * 16 + (l >> 1)]);
+                const float bv = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (l >> 1)]);
+                const float d = wide_dot(xj, word, lane, sv, bv);
+                if (lane == l) acc += d;
+            }
+        }
+        const float v = warp_sum_to_lane0(acc);
+        if (lane == 0) part[(col - c0) * nsl + j] = failed ? __int_as_float(0x7FC00000) : v;
+        __syncwarp();
+        if (t + kSStages < my_items && !failed) issue(t + kSStages);
+    }
+    if (failed)   // copies still in flight get a bounded chance to land before exit
+        for (int st = 0; st < kSStages; ++st) wait_slot(bar0 + 8 * st, 0, 1024);
+    __syncthreads();
+
+    // each column: its slice sums in ascending order
+    uint64_t best = 0;
+    for (int q = tid; q < c1 - c0; q += blockDim.x) {
+        float tot = part[q * nsl];
+        for (int j = 1; j < nsl; ++j) tot += part[q * nsl + j];
+        const uint16_t h = f32_to_bf16_rne(tot);
+        a.y[c0 + q] = h;
+        if (a.cand) best = umax64(best, cand_key(h, a.id_base + (uint32_t)(c0 + q)));
+    }
+    if (a.cand) {
+        best = warp_max64(best);
+        fused_head_keys(a, best, kSWarps, warp, lane);
+    }
 }
 
 // The widest warp count whose shared memory fits 227 KB with 1 KB left for the
@@ -722,7 +1017,7 @@ bool qmm_m1_stream_eligible(const QmmArgs &a) {
 static size_t g_stream_smem_set[64][3];
 
 template <int RU>
-static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream) {
+static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream, int *ncand) {
     const int W = stream_warps(a.K, RU);
     const StreamLayout L = stream_layout(a.K, W, RU);
     int dev = 0;
@@ -737,8 +1032,8 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream) {
     int blocks = num_sms();
     const int need = (units + W - 1) / W;
     if (need < blocks) blocks = need;
-    qmm_m1_stream_kernel<RU><<<blocks, W * 32, L.total, stream>>>(a, units);
-    return cudaGetLastError();
+    if (ncand) *ncand = blocks * W;
+    return launch_pdl(qmm_m1_stream_kernel<RU>, dim3(blocks), dim3(W * 32), L.total, stream, a, units);
 }
 
 // ---------------------------------------------------------- tile ring host --
@@ -782,7 +1077,7 @@ static int tile_ring_shape(const QmmArgs &a) {
 static bool g_tile_smem_set[64][2][2];
 
 template <bool kGlu, int kWR>
-static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream) {
+static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream, int *ncand) {
     using Sh = TileShape<kWR>;
     const int S = tile_stages(a.K);
     const TileLayout L = tile_layout(a.K, S);
@@ -823,25 +1118,58 @@ static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream) {
         g_tile_smem_set[dev][kGlu ? 1 : 0][kWR == 4 ? 1 : 0] = true;
     }
     const int blocks = plan.ntiles < num_sms() ? plan.ntiles : num_sms();
-    qmm_m1_tile_kernel<kGlu, kWR><<<blocks, kTThreads, L.total, stream>>>(a, plan, qmap, smap, bmap, S);
-    return cudaGetLastError();
+    if (ncand) *ncand = blocks * (kTWarps + kTGroups);
+    return launch_pdl(qmm_m1_tile_kernel<kGlu, kWR>, dim3(blocks), dim3(kTThreads), L.total, stream, a, plan, qmap, smap,
+                      bmap, S);
 }
 
 // Calls with enough tiles take the tile ring.  Otherwise rows per unit only change
 // how often a lane reuses its activation limbs, never a row's arithmetic, so the
 // choice may follow N: four rows while every warp of the grid still gets two
 // units, fewer when the slice is narrow.
-cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream) {
-    switch (tile_ring_shape(a)) {
-        case 4: return a.glu ? launch_tile<true, 4>(a, stream) : launch_tile<false, 4>(a, stream);
-        case 1: return launch_tile<false, 1>(a, stream);
-        default: break;
+// The narrow-call kernel: M = 1, no GLU, K longer than 8 chunks, and its layout
+// fits (the rings beside the limbs and the slice sums of a CTA's columns).
+static int split_maxcols(const QmmArgs &a) {
+    const int blocks = a.seg.ncols < num_sms() ? a.seg.ncols : num_sms();
+    return blocks > 0 ? (a.seg.ncols + blocks - 1) / blocks : 0;
+}
+static bool split_eligible(const QmmArgs &a) {
+    if (a.glu || (a.K + kChunk - 1) / kChunk <= 8) return false;
+    return split_layout(a.K, split_maxcols(a)).total <= 226 * 1024;
+}
+
+static bool g_split_smem_set[64];
+
+static cudaError_t launch_split(const QmmArgs &a, cudaStream_t stream, int *ncand) {
+    const int maxcols = split_maxcols(a);
+    const SplitLayout L = split_layout(a.K, maxcols);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!g_split_smem_set[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(qmm_m1_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+        if (e != cudaSuccess) return e;
+        g_split_smem_set[dev] = true;
     }
+    const int blocks = a.seg.ncols < num_sms() ? a.seg.ncols : num_sms();
+    if (ncand) *ncand = blocks * kSWarps;
+    return launch_pdl(qmm_m1_split_kernel, dim3(blocks), dim3(kSWarps * 32), L.total, stream, a, maxcols);
+}
+
+cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream, int *ncand) {
+    const int shape = tile_ring_shape(a);
+    if (shape == 4) return a.glu ? launch_tile<true, 4>(a, stream, ncand) : launch_tile<false, 4>(a, stream, ncand);
+    if (split_eligible(a)) return launch_split(a, stream, ncand);
+    if (shape == 1) return launch_tile<false, 1>(a, stream, ncand);
     const long long warps = (long long)num_sms() * stream_warps(a.K, 4);
     const long long rows = a.glu ? 2ll * a.seg.ncols : a.seg.ncols;
-    if (rows >= 8 * warps) return launch_ru<4>(a, 0, stream);
-    if (rows >= 2 * warps || a.glu) return launch_ru<2>(a, 1, stream);
-    return launch_ru<1>(a, 2, stream);
+    if (rows >= 8 * warps) return launch_ru<4>(a, 0, stream, ncand);
+    if (rows >= 2 * warps || a.glu) return launch_ru<2>(a, 1, stream, ncand);
+    return launch_ru<1>(a, 2, stream, ncand);
+}
+
+cudaError_t launch_argmax_keys(const uint64_t *cand, int ncand, const uint16_t *logits, uint32_t id_base, uint64_t *word,
+                               cudaStream_t stream) {
+    return launch_pdl(argmax_keys_kernel, dim3(1), dim3(1024), 0, stream, cand, ncand, logits, id_base, word);
 }
 
 int qmm_m1_stream_max_cand() { return num_sms() * kMaxWarps; }

@@ -1,14 +1,16 @@
 // qmm_tc.cu -- prompt-chunk qmm (M = 2..128 activation rows) on the 5th-generation
 // tensor cores.
 //
-// The weights enter the tensor core as their 4-bit codes, held exactly in bf16
-// as 128 + q (128..143), so one group of 64 values gives
-// D_g = sum_{k in g} (128 + q_k) x_k per weight row and activation row, with the
+// The weights enter the tensor core as their 4-bit codes taken about their
+// middle, q - 8 (-8..7, exact in bf16), so one group of 64 values gives
+// D_g = sum_{k in g} (q_k - 8) x_k per weight row and activation row, with the
 // fp32 sums in tensor memory.  The group's scale and bias are applied on the CUDA
 // cores:
-//     y += s_g * D_g + (b_g - 128 s_g) * X_g,        X_g = sum_{k in g} x_k,
+//     y += s_g * D_g + (b_g + 8 s_g) * X_g,        X_g = sum_{k in g} x_k,
 // which is sum_{k in g} x_k (s_g q_k + b_g) -- the affine format's dot product,
-// with no rounded copy of the weights anywhere (b_g - 128 s_g is exact in fp32).
+// with no rounded copy of the weights anywhere.  With the usual bias b ~ -8 s
+// both terms stay near the size of their sum, and a large x whose weight is
+// zero (q = 8, b = -8 s) adds exactly nothing to either.
 // Per output the fp32 sum runs over the groups in ascending order, an order fixed
 // by K alone.
 //
@@ -251,17 +253,19 @@ __device__ __forceinline__ void tc_st<32>(uint32_t taddr, const uint32_t *v) {
         : "memory");
 }
 
-// Codes 2j and 2j+1 of a packed word as the bf16 pair (128 + q_2j, 128 + q_2j+1),
+// Codes 2j and 2j+1 of a packed word as the bf16 pair (q_2j - 8, q_2j+1 - 8),
 // exactly (code 2j in the low half).  w holds code i at bits 4i, ws = w >> 4.
 // Byte j of w has code 2j in its low nibble, byte j of ws has code 2j+1 there;
 // prmt puts them at bits 0 and 16, the mask keeps the nibbles and ORs in the
-// bf16 exponent of 128.  The offset 128 is taken out with the bias term.
+// bf16 exponent of 128, which makes each half 128 + q; one bf16x2 subtraction of
+// 136 leaves q - 8 (exact: every value involved is an integer below 2^8).
 template <int j>
 __device__ __forceinline__ uint32_t tc_code_pair(uint32_t w, uint32_t ws) {
     constexpr uint32_t sel = j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12);
-    uint32_t p;
+    uint32_t p, r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(p) : "r"(w), "r"(ws), "n"(sel));
-    return (p & 0x000F000Fu) | 0x43004300u;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"((p & 0x000F000Fu) | 0x43004300u), "r"(0x43084308u));
+    return r;
 }
 
 // acc + lo(w) + hi(w) for a bf16 pair w, each add fp32 += bf16 (Blackwell's
@@ -304,6 +308,8 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     volatile int *fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     const int ks = plan.ks;
     const int rank = (int)tc_cluster_rank();
     const int tile = blockIdx.x / ks;
@@ -559,8 +565,8 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             break;                                                                                                  \
         }                                                                                                           \
         tc_fence_after();                                                                                           \
-        /* D holds sum (128 + q) x: y += s D + (b - 128 s) X; b - 128 s is exact in fp32 */                      \
-        const float sf = tc_pick_bf16<J>(s8), bf = fmaf(-128.0f, sf, tc_pick_bf16<J>(b8));                          \
+        /* D holds sum (q - 8) x: y += s D + (b + 8 s) X */                                                       \
+        const float sf = tc_pick_bf16<J>(s8), bf = fmaf(8.0f, sf, tc_pick_bf16<J>(b8));                             \
         const float *xg = xb_h + xs * kTcMaxN;                                                                      \
         _Pragma("unroll") for (int c = 0; c < NT; c += CH) {                                                        \
             uint32_t d[CH];                                                                                         \
@@ -696,13 +702,15 @@ static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const 
     cfg.blockDim = dim3(tc_threads(N));
     cfg.dynamicSmemBytes = tc_smem_bytes(N);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)plan.ks;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, qmm_tc_kernel<N>, a, xmap, cmap, plan);
 }
 

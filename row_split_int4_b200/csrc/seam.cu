@@ -11,6 +11,8 @@ namespace tf {
 // One thread per 8 bf16 (16 bytes) of the output; every part's width and
 // offset and the row pitches are multiples of 8, the pointers 16-byte aligned.
 __global__ void gather_vec_kernel(GatherArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int total = a.off[a.nparts];
     const int per_row = total / 8;
     const long long n = (long long)a.M * per_row;
@@ -32,6 +34,8 @@ __global__ void gather_vec_kernel(GatherArgs a) {
 
 // Element-wise form for pitches or widths that are not multiples of 8.
 __global__ void gather_scalar_kernel(GatherArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int total = a.off[a.nparts];
     const long long n = (long long)a.M * total;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
@@ -52,17 +56,16 @@ cudaError_t launch_gather(const GatherArgs &a, bool vec, cudaStream_t stream) {
     if (total == 0) return cudaSuccess;
     long long blocks = (total + 255) / 256;
     if (blocks > kNumSMs * 16) blocks = kNumSMs * 16;
-    if (vec)
-        gather_vec_kernel<<<(int)blocks, 256, 0, stream>>>(a);
-    else
-        gather_scalar_kernel<<<(int)blocks, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    if (vec) return launch_pdl(gather_vec_kernel, dim3((int)blocks), dim3(256), 0, stream, a);
+    return launch_pdl(gather_scalar_kernel, dim3((int)blocks), dim3(256), 0, stream, a);
 }
 
 // ---------------------------------------------------------------- argmax --
 constexpr int kArgmaxThreads = 256;
 
 __global__ void __launch_bounds__(kArgmaxThreads) argmax_partial_kernel(ArgmaxArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.y;
     const int b = blockIdx.x;
     const uint16_t *row = a.logits + (long long)m * a.ld;
@@ -97,6 +100,8 @@ __global__ void __launch_bounds__(kArgmaxThreads) argmax_partial_kernel(ArgmaxAr
 
 // One warp per row: max over the row's partial keys, then the word.
 __global__ void argmax_final_kernel(ArgmaxArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (m >= a.M) return;
     const int lane = threadIdx.x & 31;
@@ -124,11 +129,9 @@ cudaError_t launch_argmax(ArgmaxArgs a, cudaStream_t stream) {
     span = (span + 7) / 8 * 8;
     a.span = span;
     dim3 grid(a.blocks_per_row, a.M);
-    argmax_partial_kernel<<<grid, kArgmaxThreads, 0, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(argmax_partial_kernel, grid, dim3(kArgmaxThreads), 0, stream, a);
     if (e != cudaSuccess) return e;
-    argmax_final_kernel<<<(a.M + 7) / 8, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(argmax_final_kernel, dim3((a.M + 7) / 8), dim3(256), 0, stream, a);
 }
 
 // ------------------------------------------------------------- top two --
@@ -160,6 +163,8 @@ __device__ __forceinline__ void warp_top2(uint64_t &k1, uint64_t &k2) {
 }
 
 __global__ void __launch_bounds__(kArgmaxThreads) top2_partial_kernel(ArgmaxArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.y;
     const int b = blockIdx.x;
     const uint16_t *row = a.logits + (long long)m * a.ld;
@@ -204,6 +209,8 @@ __global__ void __launch_bounds__(kArgmaxThreads) top2_partial_kernel(ArgmaxArgs
 // A flagged row gives its flagged word twice; an empty second place gives
 // TF_TOP2_NONE.
 __global__ void top2_final_kernel(ArgmaxArgs a) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (m >= a.M) return;
     const int lane = threadIdx.x & 31;
@@ -232,11 +239,9 @@ cudaError_t launch_top2(ArgmaxArgs a, cudaStream_t stream) {
     span = (span + 7) / 8 * 8;
     a.span = span;
     dim3 grid(a.blocks_per_row, a.M);
-    top2_partial_kernel<<<grid, kArgmaxThreads, 0, stream>>>(a);
-    cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(top2_partial_kernel, grid, dim3(kArgmaxThreads), 0, stream, a);
     if (e != cudaSuccess) return e;
-    top2_final_kernel<<<(a.M + 7) / 8, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(top2_final_kernel, dim3((a.M + 7) / 8), dim3(256), 0, stream, a);
 }
 
 // One thread per row: the lowest part whose winner is flagged gives its flagged
@@ -248,6 +253,8 @@ __device__ __forceinline__ uint64_t key_of_word(uint64_t w) {
     return cand_key((uint32_t)(w & 0xFFFFFFFFull) >> 16, (uint32_t)(w >> 32));
 }
 __global__ void top2_merge_kernel(const uint64_t *words2, int nparts, int M, uint64_t *out2) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x * blockDim.x + threadIdx.x;
     if (m >= M) return;
     for (int p = 0; p < nparts; ++p) {
@@ -278,14 +285,16 @@ __global__ void top2_merge_kernel(const uint64_t *words2, int nparts, int M, uin
 }
 
 cudaError_t launch_top2_merge(const uint64_t *words2, int nparts, int M, uint64_t *out2, cudaStream_t stream) {
-    top2_merge_kernel<<<(M + 127) / 128, 128, 0, stream>>>(words2, nparts, M, out2);
-    return cudaGetLastError();
+    return launch_pdl(top2_merge_kernel, dim3((M + 127) / 128), dim3(128), 0, stream, words2, nparts, M, out2);
+
 }
 
 // ------------------------------------------------------------------ pick --
 // One thread per row: any flagged id word -> the sentinel; otherwise the larger
 // value, the lower id on equal values (fp32 compare: +0 == -0).
 __global__ void pick_kernel(const uint64_t *words, int nparts, int M, uint32_t *ids) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x * blockDim.x + threadIdx.x;
     if (m >= M) return;
     bool flagged = false;
@@ -305,8 +314,8 @@ __global__ void pick_kernel(const uint64_t *words, int nparts, int M, uint32_t *
 }
 
 cudaError_t launch_pick(const uint64_t *words, int nparts, int M, uint32_t *ids, cudaStream_t stream) {
-    pick_kernel<<<(M + 127) / 128, 128, 0, stream>>>(words, nparts, M, ids);
-    return cudaGetLastError();
+    return launch_pdl(pick_kernel, dim3((M + 127) / 128), dim3(128), 0, stream, words, nparts, M, ids);
+
 }
 
 }  // namespace tf

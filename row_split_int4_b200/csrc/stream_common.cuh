@@ -36,6 +36,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int c
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
+// Bring bytes of global memory into L2 without waiting for them (no shared
+// memory, no barrier): the 1-D form for `bytes` (a multiple of 16) at a 16-byte
+// aligned address, and the 2-D tile of a tensor map at (c0, c1).
+__device__ __forceinline__ void l2_prefetch(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void l2_prefetch_2d(const void *map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

@@ -14,6 +14,8 @@ namespace tf {
 // h[m][j] = fp32(h[m][j] + y[m][j]): one rounding, the IEEE fp32 addition.
 // Vector path: eight elements a thread (two float4 of h, one uint4 of y).
 __global__ void residual_add_vec_kernel(float *h, long long ld_h, const uint16_t *y, long long ld_y, int M, int n) {
+    pdl_trigger();
+    pdl_wait();
     const int n8 = n / 8;
     const long long total = (long long)M * n8;
     for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < total; v += (long long)gridDim.x * blockDim.x) {
@@ -42,6 +44,8 @@ __global__ void residual_add_vec_kernel(float *h, long long ld_h, const uint16_t
 }
 
 __global__ void residual_add_scalar_kernel(float *h, long long ld_h, const uint16_t *y, long long ld_y, int M, int n) {
+    pdl_trigger();
+    pdl_wait();
     const long long total = (long long)M * n;
     for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < total; v += (long long)gridDim.x * blockDim.x) {
         const int m = (int)(v / n), j = (int)(v % n);
@@ -56,17 +60,16 @@ cudaError_t launch_residual_add(float *h, long long ld_h, const uint16_t *y, lon
     const long long cap = (long long)num_sms() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    if (vec)
-        residual_add_vec_kernel<<<(int)blocks, 256, 0, stream>>>(h, ld_h, y, ld_y, M, n);
-    else
-        residual_add_scalar_kernel<<<(int)blocks, 256, 0, stream>>>(h, ld_h, y, ld_y, M, n);
-    return cudaGetLastError();
+    if (vec) return launch_pdl(residual_add_vec_kernel, dim3((int)blocks), dim3(256), 0, stream, h, ld_h, y, ld_y, M, n);
+    return launch_pdl(residual_add_scalar_kernel, dim3((int)blocks), dim3(256), 0, stream, h, ld_h, y, ld_y, M, n);
 }
 
 // out[m][:H] = table[ids[m]][:H] for ids below the bound, else the bf16 NaN.
 // One CTA per output row (grid-strided), 16-byte vectors when aligned.
 __global__ void embed_rows_kernel(const uint16_t *table, long long ld_table, uint32_t bound, int H, const uint32_t *ids,
                                   int M, uint16_t *out, long long ld_out, int vec) {
+    pdl_trigger();
+    pdl_wait();
     for (int m = blockIdx.x; m < M; m += gridDim.x) {
         const uint32_t id = ids[m];
         uint16_t *dst = out + m * ld_out;
@@ -90,8 +93,7 @@ cudaError_t launch_embed_rows(const uint16_t *table, long long ld_table, uint32_
                               int M, uint16_t *out, long long ld_out, bool vec, cudaStream_t stream) {
     int blocks = M < num_sms() * 8 ? M : num_sms() * 8;
     if (blocks < 1) blocks = 1;
-    embed_rows_kernel<<<blocks, 256, 0, stream>>>(table, ld_table, bound, H, ids, M, out, ld_out, vec ? 1 : 0);
-    return cudaGetLastError();
+    return launch_pdl(embed_rows_kernel, dim3(blocks), dim3(256), 0, stream, table, ld_table, bound, H, ids, M, out, ld_out, vec ? 1 : 0);
 }
 
 }  // namespace tf

@@ -4,6 +4,7 @@
 // call by status before anything is enqueued (TensorFold PR #1434 review
 // thread: refuse by name before the backend moves any state; fail closed).
 #include <climits>
+#include <cstdlib>
 #include <cstring>
 
 #include "tf_common.cuh"
@@ -22,6 +23,14 @@ tf_status cuda_status(cudaError_t e) {
 }
 
 cudaError_t last_cuda_error() { return g_last_cuda; }
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("TF_PDL");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
 
 }  // namespace tf
 
@@ -134,8 +143,6 @@ static tf_status qmm_args(const void *x, int M, int K, int ldx, const uint8_t *w
     a.n_whole = N_whole;
     a.cand = nullptr;
     a.id_base = 0;
-    a.done = nullptr;
-    a.word = nullptr;
     return TF_OK;
 }
 
@@ -190,8 +197,8 @@ tf_status tf_qmm8_rows(const void *x, int M, int K, int ldx, const int8_t *q8, c
 
 size_t tf_qmm_argmax_scratch_bytes(int M, int nrows) {
     if (M <= 0 || nrows <= 0) return 0;
-    // fused: one key per warp of the grid, then the finish counter
-    const size_t fused = (size_t)qmm_m1_stream_max_cand() * sizeof(uint64_t) + 16;
+    // fused: one key per warp of the grid
+    const size_t fused = (size_t)qmm_m1_stream_max_cand() * sizeof(uint64_t);
     const size_t plain = tf_argmax_scratch_bytes(M, nrows);
     return fused > plain ? fused : plain;
 }
@@ -211,15 +218,14 @@ tf_status tf_qmm_argmax_rows(const void *x, int M, int K, int ldx, const uint8_t
     if (scratch_bytes < tf_qmm_argmax_scratch_bytes(M, seg.nrows)) return TF_E_ARG;
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (M == 1 && qmm_m1_stream_eligible(a)) {
-        // fused: the qmm warps leave their best keys in scratch and the kernel's last
-        // CTA turns them into the word; the finish counter starts at zero
+        // fused: the qmm warps leave their best keys in scratch, one small kernel
+        // turns them into the word
         a.cand = static_cast<uint64_t *>(scratch);
         a.id_base = id_base;
-        a.done = reinterpret_cast<unsigned int *>(a.cand + qmm_m1_stream_max_cand());
-        a.word = words;
-        const tf_status z = cuda_status(cudaMemsetAsync(a.done, 0, sizeof(unsigned int), s));
-        if (z != TF_OK) return z;
-        return cuda_status(launch_qmm_m1_stream(a, s));
+        int ncand = 0;
+        const tf_status q = cuda_status(launch_qmm_m1_stream(a, s, &ncand));
+        if (q != TF_OK) return q;
+        return cuda_status(launch_argmax_keys(a.cand, ncand, a.y, id_base, words, s));
     }
     // otherwise the two steps: the rows, then the argmax over them
     const tf_status q = cuda_status(launch_qmm(a, s));

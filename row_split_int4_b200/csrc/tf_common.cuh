@@ -81,4 +81,41 @@ __host__ __forceinline__ bool aligned(const void *p, uintptr_t a) {
     return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialization: it may be scheduled while the kernel before it on the stream is
+// still running, once every block of that kernel has called pdl_trigger() (or
+// exited).  pdl_wait() blocks the calling thread until the kernels before it
+// have finished and their writes are visible.  Each kernel calls pdl_wait()
+// before it reads any array it was given or writes any output, with one
+// exception: it may ask for weights to be brought into L2 first (a prefetch
+// reads L2, which every write reaches, so it can never see stale data).  Each
+// qmm kernel calls pdl_trigger() once its own pdl_wait() has returned, so that
+// the next one queues behind it but no further; the short kernels between them
+// (gather, argmax, pick, ...) call it first thing, so that the qmm after them
+// can take each SM as soon as the qmm before them leaves it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// false when the environment sets TF_PDL=0: launches then keep the plain stream
+// order (the kernels' pdl_wait/pdl_trigger do nothing)
+bool pdl_enabled();
+
+// kernel<<<grid, block, smem, stream>>>(args...) with programmatic stream serialization
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace tf

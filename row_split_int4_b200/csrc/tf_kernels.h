@@ -32,12 +32,9 @@ struct QmmArgs {
     int n_whole;   // rows of the whole matrix (the call may cover only some of them)
     // fused head (M = 1 stream kernel only): when cand is set, every warp of the grid
     // writes the largest argmax key of the rows it wrote (ids id_base + column) to
-    // cand[warp of the grid] (0 when it wrote none); the last CTA to finish, counted
-    // on *done (zero at launch, zero again at exit), reduces them into *word
+    // cand[warp of the grid] (0 when it wrote none); launch_argmax_keys reduces them
     uint64_t *cand;
     uint32_t id_base;
-    unsigned int *done;
-    uint64_t *word;
 };
 
 // The int8 head: codes [N][K] int8, one bf16 scale per row.
@@ -85,7 +82,10 @@ cudaError_t launch_pick(const uint64_t *words, int nparts, int M, uint32_t *ids,
 bool qmm_m1_stream_eligible(const QmmArgs &a);
 bool qmm_tc_eligible(const QmmArgs &a);
 cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream);
-cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream);
+// *ncand (when not null) receives the number of warp keys the launch writes to a.cand
+cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream, int *ncand = nullptr);
+cudaError_t launch_argmax_keys(const uint64_t *cand, int ncand, const uint16_t *logits, uint32_t id_base, uint64_t *word,
+                               cudaStream_t stream);
 int qmm_m1_stream_max_cand();   // an upper bound of the warps of any stream launch
 
 int argmax_blocks_per_row(int M, int n);

@@ -227,3 +227,63 @@ def apply_plants(logits_bits: np.ndarray, plants, bump_bits: int | None = None) 
         elif p.kind == "allequal":
             row[:] = p.value_bits
     return logits_bits
+
+
+# ------------------------------------------------------------ wide-range inputs
+# Activations whose 32-value runs (the 32 consecutive k starting at a multiple of
+# 32) each hold one large value and 31 small ones, and weights that give the
+# large values a weight of exactly zero, so that the output is made of the small
+# values alone.  A kernel that keeps the small values only to the precision of
+# the run's largest one, or that lets the large value's cancelled product swamp
+# them, misses the fp32 accuracy the method asks for.
+
+def wide_positions(K: int, seed: int = 0, tag: int = 11) -> np.ndarray:
+    """One position per 32-value run of K: the k of its large value."""
+    assert K % 32 == 0
+    rng = np.random.default_rng([seed, tag])
+    return np.arange(0, K, 32) + rng.integers(0, 32, size=K // 32)
+
+
+def make_x_wide(M: int, K: int, big_exp: int = 10, small_exp=(-14, -10), seed: int = 0, tag: int = 12,
+                positions: np.ndarray | None = None) -> np.ndarray:
+    """[M, K] bf16 bits: at every position of ``positions`` (default
+    ``wide_positions(K, seed)``) +-2^big_exp; elsewhere +-2^u * (1 + f) with u
+    uniform over the integers of [small_exp[0], small_exp[1]] and f uniform in
+    [0, 1), random signs."""
+    rng = np.random.default_rng([seed, tag])
+    pos = wide_positions(K, seed) if positions is None else positions
+    u = rng.integers(small_exp[0], small_exp[1] + 1, size=(M, K))
+    f = rng.uniform(0.0, 1.0, size=(M, K))
+    sgn = np.where(rng.integers(0, 2, size=(M, K)) == 1, -1.0, 1.0)
+    v = sgn * np.ldexp(1.0 + f, u)
+    big_sgn = np.where(rng.integers(0, 2, size=(M, len(pos))) == 1, -1.0, 1.0)
+    v[:, pos] = big_sgn * 2.0 ** big_exp
+    return to_bf16_bits(v.astype(np.float32))
+
+
+def with_zero_weights(w: QWeights, positions: np.ndarray, offset: int = 8) -> QWeights:
+    """A copy of ``w`` whose weights at columns ``positions`` are exactly zero in
+    every row: code ``offset`` there and, in every group holding such a column,
+    bias = -offset * scale (exact in bf16 for offset 8, a power of two; for
+    other offsets the scale is rounded to 4 significant bits first, so that
+    offset * scale still fits bf16)."""
+    q = np.empty((w.N, w.K), dtype=np.uint8)
+    q[:, 0::2] = w.wq & 0x0F
+    q[:, 1::2] = w.wq >> 4
+    q[:, positions] = offset
+    sc = w.scales.copy()
+    bi = w.biases.copy()
+    groups = np.unique(np.asarray(positions) // GROUP)
+    if offset & (offset - 1):
+        sc[:, groups] &= 0xFFF0   # 4 significant bits: offset * scale is exact
+    bi[:, groups] = to_bf16_bits(np.float32(-offset) * bf16_bits_to_f32(sc[:, groups]))
+    assert np.array_equal(bf16_bits_to_f32(bi[:, groups]).astype(np.float64),
+                          -offset * bf16_bits_to_f32(sc[:, groups]).astype(np.float64))
+    return QWeights(pack_nibbles(q), sc, bi)
+
+
+def with_zero_weights8(w: Q8Weights, positions: np.ndarray) -> Q8Weights:
+    """A copy of the int8 matrix with code 0 at columns ``positions``."""
+    q8 = w.q8.copy()
+    q8[:, positions] = 0
+    return Q8Weights(q8, w.scales.copy())

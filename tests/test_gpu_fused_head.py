@@ -2,8 +2,8 @@
 one call (TensorFold PR #1433 step-1 body: each rank computes its half of the
 lm_head, then pair_argmax over it).
 
-At M = 1 the qmm warps keep the best argmax key of the rows they write and the
-kernel's last CTA to finish combines them.  The contract is bit-for-bit equality with
+At M = 1 the qmm warps keep the best argmax key of the rows they write and a
+one-CTA kernel combines the keys into the word.  The contract is bit-for-bit equality with
 the two separate calls (tf_qmm_rows, then tf_argmax_rows on its logits), which
 these tests check on natural weights, on weights that make an exact tie across
 the halves, a NaN row and an overflowing row, at full lm_head-half size, and
@@ -132,3 +132,69 @@ def test_fused_lm_head_half_full_size(tf):
         torch.cuda.synchronize()
         assert bits_equal(lf, lu)
         assert torch.equal(wf, wu)
+
+
+@pytest.fixture(scope="module")
+def whole_head():
+    w = synth.make_weights(synth.VOCAB, synth.HIDDEN, seed=14, tag=synth.TAG_HEAD)
+    return w, DevWeights(w)
+
+
+@pytest.mark.parametrize("kind", ["natural", "tie", "nan", "inf"])
+def test_fused_full_head_planted(tf, orc, whole_head, kind):
+    """Both 124,160-row halves of the 248,320-row head on the tile ring, with a
+    planted exact tie across the halves (the top row copied into the other half),
+    a NaN row in half 0 or an overflowing row in half 1: each half's word equals
+    the oracle's scan of the GPU's own logits, and the pick of the two words is
+    the lower id of the tie, or the sentinel."""
+    w, W = whole_head
+    V, K = synth.VOCAB, synth.HIDDEN
+    h = V // 2
+    x = dev(synth.make_x(1, K, seed=14, tag=5))
+    saved = []
+
+    def plant(row, wq=None, sc=None, bi=None):
+        saved.append((row, W.wq[row].clone(), W.scales[row].clone(), W.biases[row].clone()))
+        if wq is not None:
+            W.wq[row] = wq
+        if sc is not None:
+            W.scales[row] = sc
+        if bi is not None:
+            W.biases[row] = bi
+
+    try:
+        expect = None
+        if kind == "tie":
+            lg, _ = unfused(tf, x, W, (0, V), 0)
+            f = lg.float()[0]
+            top = int(torch.argmax(torch.where(torch.isfinite(f), f, torch.full_like(f, -float("inf")))))
+            other = top + h + 5 if top < h else top - h + 5
+            plant(other, W.wq[top].clone(), W.scales[top].clone(), W.biases[top].clone())
+            expect = min(top, other)
+        elif kind == "nan":   # every group scale NaN (0x7FC0): the logit is NaN
+            plant(1234, sc=torch.full_like(W.scales[1234].view(torch.int16), 0x7FC0).view(torch.bfloat16))
+        elif kind == "inf":   # codes 15, scale and bias the largest finite bf16 (0x7F7F): the row overflows
+            r = h + 4321
+            big = torch.full_like(W.scales[r].view(torch.int16), 0x7F7F).view(torch.bfloat16)
+            plant(r, wq=torch.full_like(W.wq[r], 0xFF), sc=big, bi=big.clone())
+        torch.cuda.synchronize()
+        words = torch.empty(2, 1, dtype=torch.int64, device="cuda")
+        for p in range(2):
+            seg = tf.tf_split_rows(V, 2, p)
+            lf, wf = fused(tf, x, W, seg, seg[0])
+            torch.cuda.synchronize()
+            assert np.array_equal(host_bits(wf), orc.argmax_rows(host_bits(lf), seg[0])), (kind, p)
+            words[p] = wf
+        ids = pick(tf, words)
+        if kind in ("nan", "inf"):
+            assert ids[0] == tf.TF_PICK_FAILED
+            flagged = int(host_bits(words)[0 if kind == "nan" else 1, 0]) >> 32
+            assert flagged & 0x80000000
+        else:
+            assert ids[0] != tf.TF_PICK_FAILED
+        if expect is not None:
+            assert ids[0] == expect, (ids[0], expect)
+    finally:
+        for row, a, b, c in reversed(saved):
+            W.wq[row], W.scales[row], W.biases[row] = a, b, c
+        torch.cuda.synchronize()

@@ -1,9 +1,12 @@
 """PairDecode on the GPU kernels, as a one-rank NCCL group (every call here gets
 one GPU): with one rank the seams' all-gathers return the rank's own rows, so
 the step must give exactly the one-GPU whole path -- the fused gate-up with the
-GLU, down, the head, argmax and pick -- bit for bit.  This checks the step's
-composition (shares, buffers, calls); the exchange between two ranks is checked
-on CPU ranks in test_pair_seam.py."""
+GLU, down, the head, argmax and pick -- bit for bit.  Each stage of the step is
+also held to the oracle: the gate and up rows and the down and head outputs
+within 2 bf16 ulps of the fp64 oracle on the GPU stage's own inputs, the GLU
+frame against the oracle's GLU of the GPU's gate and up rows, the word and the
+id bit for bit against the oracle's scan and pick of the GPU's logits.  The
+exchange between two ranks is checked on CPU ranks in test_pair_seam.py."""
 import os
 import socket
 from datetime import timedelta
@@ -13,7 +16,7 @@ import pytest
 import torch
 
 import synth
-from gpu_util import DevWeights, bits_equal, dev, empty_bf16, host_bits, need_gpu
+from gpu_util import DevWeights, bits_equal, check_values, dev, empty_bf16, host_bits, need_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -24,17 +27,19 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_pair_decode_one_rank_equals_whole():
+def test_pair_decode_one_rank_equals_whole(orc):
     need_gpu()
     import torch.distributed as dist
     import row_split_int4_b200 as tf
     from row_split_int4_b200.pair import PairDecode, PairSeam
 
     H, F, V = 1024, 2048, 4096
-    wgu = DevWeights(synth.make_weights(2 * F, H, seed=41, tag=synth.TAG_W))
-    wd = DevWeights(synth.make_weights(H, F, seed=41, tag=synth.TAG_W2))
-    wlm = DevWeights(synth.make_weights(V, H, seed=41, tag=synth.TAG_HEAD))
-    x = dev(synth.make_x(1, H, seed=41))
+    hgu = synth.make_weights(2 * F, H, seed=41, tag=synth.TAG_W)
+    hd = synth.make_weights(H, F, seed=41, tag=synth.TAG_W2)
+    hlm = synth.make_weights(V, H, seed=41, tag=synth.TAG_HEAD)
+    wgu, wd, wlm = DevWeights(hgu), DevWeights(hd), DevWeights(hlm)
+    xb = synth.make_x(1, H, seed=41)
+    x = dev(xb)
 
     # the one-GPU whole path
     act = empty_bf16(1, F)
@@ -60,3 +65,20 @@ def test_pair_decode_one_rank_equals_whole():
         assert host_bits(ids)[0] == int(host_bits(word)[0]) >> 32
     finally:
         dist.destroy_process_group()
+
+    # every stage against the oracle, on the GPU stage's own inputs
+    g, u = empty_bf16(1, F), empty_bf16(1, F)
+    tf.tf_qmm_rows(x, *wgu.t(), [(0, F)], g)
+    tf.tf_qmm_rows(x, *wgu.t(), [(F, F)], u)
+    torch.cuda.synchronize()
+    for t, rows, what in ((g, np.arange(F), "gate"), (u, np.arange(F, 2 * F), "up")):
+        yo, y64, ad = orc.qmm_rows(xb, *hgu.astuple(), rows, want_f64=True)
+        check_values(host_bits(t), yo, y64, ad, H, what)
+    check_values(host_bits(dec.act), orc.glu(host_bits(g), host_bits(u)), what="GLU frame")
+    yo, y64, ad = orc.qmm_rows(host_bits(dec.act), *hd.astuple(), np.arange(H), want_f64=True)
+    check_values(host_bits(dec.y), yo, y64, ad, F, "down")
+    yo, y64, ad = orc.qmm_rows(host_bits(dec.y), *hlm.astuple(), np.arange(V), want_f64=True)
+    check_values(host_bits(dec.logits), yo, y64, ad, H, "head logits")
+    o_word = orc.argmax_rows(host_bits(dec.logits), 0)
+    assert np.array_equal(host_bits(word), o_word)
+    assert np.array_equal(host_bits(ids), orc.pick(o_word[None, :]))

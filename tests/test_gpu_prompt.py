@@ -4,8 +4,10 @@
   and down (17,408 -> 5,120); M=512 requested and capped into four 128-row
   chunks; each chunk's activated half frame fits 128 * 8,704 * 2 bytes.
 * M in {1,2,4,8,16,32,64,128} over the four shapes (lm_head with argmax and
-  pick).  Values are checked on sampled columns (all m); ids bit for bit
-  against the oracle's argmax/pick on the GPU's own logits.
+  pick).  Values are checked on sampled columns (all m): 4,096 random columns
+  plus every position of the first and the last 128-row tile and the rows on
+  either side of the half boundary; ids bit for bit against the oracle's
+  argmax/pick on the GPU's own logits.
 """
 import os
 
@@ -19,7 +21,8 @@ import head_pipeline as HP
 
 pytestmark = pytest.mark.gpu
 NT = os.cpu_count() or 1
-SAMPLE = 192
+SAMPLE = 4096
+TILE = 128   # rows of one tensor-core tile
 
 
 @pytest.fixture(scope="module")
@@ -46,9 +49,19 @@ def W_head():
     return w, DevWeights(w)
 
 
-def sampled_check(orc, x_bits, w, y_bits, cols, K, what, seed=0):
+def sample_cols(n, seed=0):
+    """4,096 random output columns of n, plus every position of the first and the
+    last 128-row tile (a wrong row inside a tile shows there) and the two columns
+    either side of the middle (the half boundary)."""
     rng = np.random.default_rng(seed)
-    pick = np.sort(rng.choice(len(cols), min(SAMPLE, len(cols)), replace=False))
+    pick = rng.choice(n, min(SAMPLE, n), replace=False)
+    forced = np.concatenate([np.arange(min(TILE, n)), np.arange(max(0, n - TILE), n),
+                             [max(0, n // 2 - 1), n // 2]])
+    return np.unique(np.concatenate([pick, forced]))
+
+
+def sampled_check(orc, x_bits, w, y_bits, cols, K, what, seed=0):
+    pick = sample_cols(len(cols), seed)
     yo, y64, ad = orc.qmm_rows(x_bits, *w.astuple(), np.asarray(cols)[pick], nthreads=NT, want_f64=True)
     return check_values(y_bits[:, pick], yo, y64, ad, K, what)
 
@@ -120,6 +133,11 @@ def test_prompt_chunk_m128(tf, orc, W):
     sampled_check(orc, xb[:128], wgu, host_bits(g), np.arange(F), H, "gate M=128")
     check_values(a_bits[:128], orc.glu(host_bits(g), host_bits(u)), what="GLU stage M=128")
     sampled_check(orc, a_bits, wd, host_bits(y_down), np.arange(H), F, "down M=128")
+    # one 128-row chunk of attn_out and of down at full width
+    yo, y64, ad = orc.qmm_rows(xb[:128], *wa.astuple(), np.arange(H), nthreads=NT, want_f64=True)
+    check_values(host_bits(y_attn)[:128], yo, y64, ad, H, "attn_out M=128, every column")
+    yo, y64, ad = orc.qmm_rows(a_bits[:128], *wd.astuple(), np.arange(H), nthreads=NT, want_f64=True)
+    check_values(host_bits(y_down)[:128], yo, y64, ad, F, "down M=128, every column")
 
 
 SHAPES = ["attn_out", "gate_up", "down"]

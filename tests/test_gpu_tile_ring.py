@@ -87,3 +87,33 @@ def test_tile_ring_glu_odd_columns(tf, orc):
     check_values(host_bits(whole), orc.glu(host_bits(g), host_bits(u)), what="GLU stage, tile ring")
     sampled(orc, x, w, host_bits(g), np.arange(F), K, "gate rows")
     sampled(orc, x, w, host_bits(u), np.arange(F, 2 * F), K, "up rows", seed=2)
+
+
+def test_long_k_routes_agree(tf, orc):
+    """K = 17,408 (17 chunks: slices of 4, 4, 4, 4 and 1 chunks).  The whole
+    9,600-row matrix runs on the 16-row tile ring, which folds each slice's tree
+    sum into the row inside the warp; a 2,560-row slice and a short one run on the
+    narrow-call kernel, whose warps share the (row, slice) pairs and add the
+    slice sums afterwards; a GLU call over 4,800 columns takes the tile ring and
+    a 100-column one the per-warp ring.  Every route must give the same bits for
+    the same row, and values within the V bar of the oracle."""
+    N, K = 9600, 17408
+    w = synth.make_weights(N, K, seed=41, tag=synth.TAG_W2)
+    W = DevWeights(w)
+    x = synth.make_x(1, K, seed=41)
+    xt = dev(x)
+    whole = qmm(tf, xt, W, [(0, N)])
+    torch.cuda.synchronize()
+    sampled(orc, x, w, host_bits(whole), np.arange(N), K, "K=17,408 whole (tile ring)")
+    for segs in ([(0, 2560)], [(7040, 2560)], [(5000, 37), (100, 3)]):
+        y = qmm(tf, xt, W, segs)
+        cols = columns_of(segs)
+        torch.cuda.synchronize()
+        assert bits_equal(y, whole[:, torch.as_tensor(cols, device="cuda")]), segs
+    F = N // 2
+    glu_whole = qmm(tf, xt, W, [(0, F), (F, F)], epi=tf.TF_EPI_GLU)
+    glu_small = qmm(tf, xt, W, [(200, 100), (F + 200, 100)], epi=tf.TF_EPI_GLU)
+    torch.cuda.synchronize()
+    assert bits_equal(glu_small, glu_whole[:, 200:300])
+    check_values(host_bits(glu_whole), orc.glu(host_bits(whole)[:, :F], host_bits(whole)[:, F:]),
+                 what="GLU stage at K = 17,408")

@@ -87,3 +87,53 @@ def test_static_scratch_refuses_oversize(tf):
     w = torch.zeros(1, dtype=torch.int64, device="cuda")
     st = tf.lib.tf_argmax_rows_static(ctypes.c_void_p(lg.data_ptr()), M, n, n, 0, ctypes.c_void_p(w.data_ptr()), None)
     assert st == tf.TF_E_ARG
+
+
+_RESET_CHILD = r"""
+import ctypes, sys
+import numpy as np
+lib = ctypes.CDLL(sys.argv[1])
+rt = ctypes.CDLL("libcudart.so.12")   # the runtime instance libtf.so is linked against
+lib.tf_argmax_rows_static.restype = ctypes.c_int
+M, n = 3, 5000
+rng = np.random.default_rng(5)
+host = (rng.standard_normal((M, n)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+def once():
+    d_l, d_w = ctypes.c_void_p(), ctypes.c_void_p()
+    assert rt.cudaMalloc(ctypes.byref(d_l), ctypes.c_size_t(M * n * 2)) == 0
+    assert rt.cudaMalloc(ctypes.byref(d_w), ctypes.c_size_t(M * 8)) == 0
+    assert rt.cudaMemcpy(d_l, host.ctypes.data_as(ctypes.c_void_p), ctypes.c_size_t(M * n * 2), 1) == 0
+    st = lib.tf_argmax_rows_static(d_l, M, n, n, ctypes.c_uint32(0), d_w, None)
+    assert rt.cudaDeviceSynchronize() == 0
+    out = np.zeros(M, dtype=np.uint64)
+    assert rt.cudaMemcpy(out.ctypes.data_as(ctypes.c_void_p), d_w, ctypes.c_size_t(M * 8), 2) == 0
+    rt.cudaFree(d_l)
+    rt.cudaFree(d_w)
+    return st, out
+
+st1, w1 = once()
+assert rt.cudaDeviceReset() == 0   # a new primary context, the library's module loaded again
+st2, w2 = once()
+np.save(sys.argv[2], np.stack([w1, w2]))
+print(st1, st2)
+"""
+
+
+def test_static_scratch_after_context_reset(tf, orc, tmp_path):
+    """After cudaDeviceReset the next call looks its array's address up again in the
+    new context (run in a child process that uses only the CUDA runtime, so the
+    reset touches no other state of this process)."""
+    import os
+    import subprocess
+    import sys
+    out = tmp_path / "words.npy"
+    r = subprocess.run([sys.executable, "-c", _RESET_CHILD, os.path.abspath(tf.LIB_PATH), str(out)],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.split() == ["0", "0"], r.stdout
+    words = np.load(out)
+    rng = np.random.default_rng(5)
+    host = (rng.standard_normal((3, 5000)).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    want = orc.argmax_rows(host, 0)
+    assert np.array_equal(words[0], want) and np.array_equal(words[1], want)
