@@ -531,14 +531,16 @@ struct TileLayout {
     size_t limb_off, sf_off, scale_off, full_off, empty_off, hdr_off, ctl_off, ring_off, total;
 };
 
-__host__ __device__ inline TileLayout tile_layout(int K, int stages) {
+// Shared memory of the tile ring for K, `stages` slots per group and M activation
+// rows (limbs, sums and scales of every row, row m at offset m times one row's).
+__host__ __device__ inline TileLayout tile_layout(int K, int stages, int M = 1) {
     TileLayout L;
     L.nch = (K + kChunk - 1) / kChunk;
     L.stages = stages;
     L.limb_off = 0;
-    L.sf_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.sf_off + (size_t)L.nch * 32 * 4, 128);
-    L.full_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
+    L.sf_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
+    L.scale_off = round_up(L.sf_off + (size_t)M * L.nch * 32 * 4, 128);
+    L.full_off = round_up(L.scale_off + (size_t)M * L.nch * 32 * 4, 128);
     L.empty_off = L.full_off + (size_t)kTGroups * stages * 8;
     L.hdr_off = L.empty_off + (size_t)kTGroups * stages * 8;    // (tile, chunk) of each slot
     L.ctl_off = L.hdr_off + (size_t)kTGroups * stages * 8;      // claim counter, abort flag
@@ -571,12 +573,12 @@ __device__ __forceinline__ int tile_row(int w, int r) {
     return kGlu ? (r & 1) * (2 * kWR) + (kWR / 2) * w + (r >> 1) : kWR * w + r;
 }
 
-template <bool kGlu, int kWR>
+template <bool kGlu, int kWR, int kM>
 __global__ void __launch_bounds__(kTThreads, 1)
     qmm_m1_tile_kernel(QmmArgs a, TilePlan plan, const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap bmap, int S) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const TileLayout L = tile_layout(a.K, S);
+    const TileLayout L = tile_layout(a.K, S, kM);
     using Sh = TileShape<kWR>;
     static_assert(!kGlu || kWR >= 2, "a GLU column needs its gate and up rows in one warp");
     constexpr int kRows = Sh::rows, kCps = Sh::cps;
@@ -710,7 +712,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
     if (producer && lane == 0)
         for (int i = 0; i < S; ++i) issue_next();
     __syncwarp();
-    prep_limbs(a.x, K, nch, limbs, SFs, Ss, kTWarps + kTGroups, warp, lane);
+    const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
+#pragma unroll
+    for (int m = 0; m < kM; ++m)
+        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, SFs + m * lc_n, Ss + m * lc_n,
+                   kTWarps + kTGroups, warp, lane);
     __syncthreads();
     if (producer) {
         if (lane == 0)
@@ -718,9 +724,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
         __syncwarp();
     }
 
-    float acc[kWR], tot[kWR];
+    float acc[kWR][kM], tot[kWR][kM];
 #pragma unroll
-    for (int r = 0; r < kWR; ++r) acc[r] = tot[r] = 0.0f;
+    for (int r = 0; r < kWR; ++r)
+#pragma unroll
+        for (int m = 0; m < kM; ++m) acc[r][m] = tot[r][m] = 0.0f;
     const int sc = slice_chunks(nch);
     uint64_t best = 0;
     int slot = 0;
@@ -745,37 +753,46 @@ __global__ void __launch_bounds__(kTThreads, 1)
             if (c >= nch) break;   // chunks past K add nothing
             // nor do lanes past the end of a short last chunk
             const bool live = lane * 32 < K - c * kChunk;
-            LaneChunk t;
-            load_lane_chunk(t, limb_l, SFs, Ss, c, lane);
-            const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && t.wide);
-            if (live) {
+            // the warp's rows: codes, scale and bias, shared by the activation rows
+            uint4 qv[kWR];
+            float sv[kWR], bv[kWR];
 #pragma unroll
-                for (int r = 0; r < kWR; ++r) {
-                    const int R = tile_row<kGlu, kWR>(w_in, r);
-                    const uint4 qv = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
-                    const float s = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
-                    const float b = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
-                    acc[r] = lane_chunk_fma(acc[r], qv, t, s, b);
-                }
+            for (int r = 0; r < kWR; ++r) {
+                const int R = tile_row<kGlu, kWR>(w_in, r);
+                qv[r] = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
+                sv[r] = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+                bv[r] = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
             }
-            for (uint32_t m = wm; m != 0; m &= m - 1) {   // wide lane-chunks, warp-uniform
-                const int l = __ffs(m) - 1;
-                const float xj = wide_x(limbs, c, l, lane);
 #pragma unroll
-                for (int r = 0; r < kWR; ++r) {
-                    const int R = tile_row<kGlu, kWR>(w_in, r);
-                    const uint32_t word = reinterpret_cast<const uint32_t *>(
-                        sl)[(R * (Sh::q / 16) + cc * (kChunk / 32) + l) * 4 + (lane >> 3)];
-                    const float s = bf16_bits_to_f32(sc0[R * (Sh::sb / 2) + cc * (kChunk / 64) + (l >> 1)]);
-                    const float b =
-                        bf16_bits_to_f32(sc0[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64) + (l >> 1)]);
-                    const float d = wide_dot(xj, word, lane, s, b);
-                    if (lane == l) acc[r] += d;
+            for (int m = 0; m < kM; ++m) {
+                LaneChunk t;
+                load_lane_chunk(t, limb_l + m * lc_n * (kLimbBytes / 16), SFs + m * lc_n, Ss + m * lc_n, c, lane);
+                const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && t.wide);
+                if (live) {
+#pragma unroll
+                    for (int r = 0; r < kWR; ++r) acc[r][m] = lane_chunk_fma(acc[r][m], qv[r], t, sv[r], bv[r]);
+                }
+                for (uint32_t mm = wm; mm != 0; mm &= mm - 1) {   // wide lane-chunks, warp-uniform
+                    const int l = __ffs(mm) - 1;
+                    const float xj = wide_x(limbs + m * lc_n * kLimbBytes, c, l, lane);
+#pragma unroll
+                    for (int r = 0; r < kWR; ++r) {
+                        const int R = tile_row<kGlu, kWR>(w_in, r);
+                        const uint32_t word = reinterpret_cast<const uint32_t *>(
+                            sl)[(R * (Sh::q / 16) + cc * (kChunk / 32) + l) * 4 + (lane >> 3)];
+                        const float s = bf16_bits_to_f32(sc0[R * (Sh::sb / 2) + cc * (kChunk / 64) + (l >> 1)]);
+                        const float b =
+                            bf16_bits_to_f32(sc0[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64) + (l >> 1)]);
+                        const float d = wide_dot(xj, word, lane, s, b);
+                        if (lane == l) acc[r][m] += d;
+                    }
                 }
             }
             if (slice_end(c, sc, nch)) {
 #pragma unroll
-                for (int r = 0; r < kWR; ++r) slice_fold(acc[r], tot[r], c, sc);
+                for (int r = 0; r < kWR; ++r)
+#pragma unroll
+                    for (int m = 0; m < kM; ++m) slice_fold(acc[r][m], tot[r][m], c, sc);
             }
         }
         __syncwarp();
@@ -788,24 +805,28 @@ __global__ void __launch_bounds__(kTThreads, 1)
             if (lane == 0) {
                 int r_a, r_b, col, ncol;
                 tile_rows(h.x, r_a, r_b, col, ncol);
-                if (kGlu) {
 #pragma unroll
-                    for (int p = 0; p < kWR / 2; ++p) {
-                        const int cj = (kWR / 2) * w_in + p;
-                        if (cj < ncol) {
-                            const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p]));
-                            const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1]));
-                            a.y[col + cj] = f32_to_bf16_rne(glu_f32(g, uu));
+                for (int m = 0; m < kM; ++m) {
+                    uint16_t *ym = a.y + (size_t)m * a.ldy;
+                    if (kGlu) {
+#pragma unroll
+                        for (int p = 0; p < kWR / 2; ++p) {
+                            const int cj = (kWR / 2) * w_in + p;
+                            if (cj < ncol) {
+                                const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p][m]));
+                                const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1][m]));
+                                ym[col + cj] = f32_to_bf16_rne(glu_f32(g, uu));
+                            }
                         }
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int r = 0; r < kWR; ++r) {
-                        const int cj = kWR * w_in + r;
-                        if (cj < ncol) {
-                            const uint16_t hv = f32_to_bf16_rne(tot[r]);
-                            a.y[col + cj] = hv;
-                            if (a.cand) best = umax64(best, cand_key(hv, a.id_base + (uint32_t)(col + cj)));
+                        for (int r = 0; r < kWR; ++r) {
+                            const int cj = kWR * w_in + r;
+                            if (cj < ncol) {
+                                const uint16_t hv = f32_to_bf16_rne(tot[r][m]);
+                                ym[col + cj] = hv;
+                                if (kM == 1 && a.cand) best = umax64(best, cand_key(hv, a.id_base + (uint32_t)(col + cj)));
+                            }
                         }
                     }
                 }
@@ -820,7 +841,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
         for (int t = t0; t < t1; ++t) {
             int r_a, r_b, col, ncol;
             tile_rows(t, r_a, r_b, col, ncol);
-            for (int i = tid; i < ncol; i += blockDim.x) a.y[col + i] = (uint16_t)TF_NAN_BF16;
+            for (int i = tid; i < kM * ncol; i += blockDim.x)
+                a.y[(size_t)(i / ncol) * a.ldy + col + i % ncol] = (uint16_t)TF_NAN_BF16;
         }
         if (producer && lane == 0)
             for (int s2 = 0; s2 < S && s2 < nissued; ++s2) {
@@ -845,7 +867,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 // order.  That is the reduction order of every M = 1 kernel (see the top of this
 // file), so the bits are theirs.
 constexpr int kSWarps = 16;
-constexpr int kSStages = 4;
+constexpr int kSMaxStages = 4;
 constexpr int kSItemQ = 4 * kChunk / 2;          // code bytes of one row-slice
 constexpr int kSItemS = 4 * kChunk / 32;         // scale (or bias) bytes of one row-slice
 constexpr int kSSlot = kSItemQ + 2 * kSItemS;    // 2,304
@@ -855,23 +877,25 @@ struct SplitLayout {
     size_t limb_off, sf_off, scale_off, part_off, bar_off, ring_off, total;
 };
 
-__host__ __device__ inline SplitLayout split_layout(int K, int maxcols) {
+// M activation rows (limbs, sums and scales of each), `stages` slots per warp.
+__host__ __device__ inline SplitLayout split_layout(int K, int maxcols, int M, int stages) {
     SplitLayout L;
     L.nch = (K + kChunk - 1) / kChunk;
     L.nsl = (L.nch + 3) / 4;
     L.limb_off = 0;
-    L.sf_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.sf_off + (size_t)L.nch * 32 * 4, 128);
-    L.part_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
-    L.bar_off = round_up(L.part_off + (size_t)maxcols * L.nsl * 4, 128);
-    L.ring_off = round_up(L.bar_off + (size_t)kSWarps * kSStages * 8, 128);
-    L.total = L.ring_off + (size_t)kSWarps * kSStages * kSSlot;
+    L.sf_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
+    L.scale_off = round_up(L.sf_off + (size_t)M * L.nch * 32 * 4, 128);
+    L.part_off = round_up(L.scale_off + (size_t)M * L.nch * 32 * 4, 128);
+    L.bar_off = round_up(L.part_off + (size_t)maxcols * L.nsl * M * 4, 128);
+    L.ring_off = round_up(L.bar_off + (size_t)kSWarps * kSMaxStages * 8, 128);
+    L.total = L.ring_off + (size_t)kSWarps * stages * kSSlot;
     return L;
 }
 
-__global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a, int maxcols) {
+template <int kM>
+__global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a, int maxcols, int kSStages) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const SplitLayout L = split_layout(a.K, maxcols);
+    const SplitLayout L = split_layout(a.K, maxcols, kM, kSStages);
     const int K = a.K, nch = L.nch, nsl = L.nsl;
     const int G = K / kGroup;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -881,7 +905,7 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     float *part = reinterpret_cast<float *>(smem + L.part_off);
     uint8_t *ring = smem + L.ring_off + (size_t)warp * kSStages * kSSlot;
     const uint32_t ring_s = smem_addr(ring);
-    const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kSStages * 8);
+    const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kSMaxStages * 8);
 
     // this CTA's columns and the warp's (column, slice) pairs: i = warp + t * kSWarps
     const int c0 = (int)((long long)blockIdx.x * a.seg.ncols / gridDim.x);
@@ -936,7 +960,11 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     pdl_wait();
     pdl_trigger();
     for (int t = 0; t < kSStages && t < my_items; ++t) issue(t);
-    prep_limbs(a.x, K, nch, limbs, SFs, Ss, kSWarps, warp, lane);
+    const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
+#pragma unroll
+    for (int m = 0; m < kM; ++m)
+        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, SFs + m * lc_n, Ss + m * lc_n,
+                   kSWarps, warp, lane);
     __syncthreads();
 
     const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
@@ -951,31 +979,37 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
         const int ch = min(4, nch - 4 * j);
         const uint8_t *sl = ring + slot * kSSlot;
         const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kSItemQ);
-        float acc = 0.0f;
+        float acc[kM];
+#pragma unroll
+        for (int m = 0; m < kM; ++m) acc[m] = 0.0f;
         for (int cc = 0; cc < ch; ++cc) {
             const int c = 4 * j + cc;
             const bool live = lane * 32 < K - c * kChunk;   // lanes past the end of a short last chunk add nothing
-            LaneChunk lc;
-            load_lane_chunk(lc, limb_l, SFs, Ss, c, lane);
-            const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && lc.wide);
-            if (live) {
-                const uint4 qv = reinterpret_cast<const uint4 *>(sl)[cc * 32 + lane];
-                const float sv = bf16_bits_to_f32(sc0[cc * 16 + (lane >> 1)]);
-                const float bv = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (lane >> 1)]);
-                acc = lane_chunk_fma(acc, qv, lc, sv, bv);
-            }
-            for (uint32_t m = wm; m != 0; m &= m - 1) {   // wide lane-chunks, warp-uniform
-                const int l = __ffs(m) - 1;
-                const float xj = wide_x(limbs, c, l, lane);
-                const uint32_t word = reinterpret_cast<const uint32_t *>(sl)[(cc * 32 + l) * 4 + (lane >> 3)];
-                const float sv = bf16_bits_to_f32(sc0[cc * 16 + (l >> 1)]);
-                const float bv = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (l >> 1)]);
-                const float d = wide_dot(xj, word, lane, sv, bv);
-                if (lane == l) acc += d;
+            const uint4 qv = reinterpret_cast<const uint4 *>(sl)[cc * 32 + lane];
+            const float sv = bf16_bits_to_f32(sc0[cc * 16 + (lane >> 1)]);
+            const float bv = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (lane >> 1)]);
+#pragma unroll
+            for (int m = 0; m < kM; ++m) {
+                LaneChunk lc;
+                load_lane_chunk(lc, limb_l + m * lc_n * (kLimbBytes / 16), SFs + m * lc_n, Ss + m * lc_n, c, lane);
+                const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && lc.wide);
+                if (live) acc[m] = lane_chunk_fma(acc[m], qv, lc, sv, bv);
+                for (uint32_t mm = wm; mm != 0; mm &= mm - 1) {   // wide lane-chunks, warp-uniform
+                    const int l = __ffs(mm) - 1;
+                    const float xj = wide_x(limbs + m * lc_n * kLimbBytes, c, l, lane);
+                    const uint32_t word = reinterpret_cast<const uint32_t *>(sl)[(cc * 32 + l) * 4 + (lane >> 3)];
+                    const float s = bf16_bits_to_f32(sc0[cc * 16 + (l >> 1)]);
+                    const float b = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (l >> 1)]);
+                    const float d = wide_dot(xj, word, lane, s, b);
+                    if (lane == l) acc[m] += d;
+                }
             }
         }
-        const float v = warp_sum_to_lane0(acc);
-        if (lane == 0) part[(col - c0) * nsl + j] = failed ? __int_as_float(0x7FC00000) : v;
+#pragma unroll
+        for (int m = 0; m < kM; ++m) {
+            const float v = warp_sum_to_lane0(acc[m]);
+            if (lane == 0) part[((col - c0) * nsl + j) * kM + m] = failed ? __int_as_float(0x7FC00000) : v;
+        }
         __syncwarp();
         if (t + kSStages < my_items && !failed) issue(t + kSStages);
     }
@@ -983,16 +1017,17 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
         for (int st = 0; st < kSStages; ++st) wait_slot(bar0 + 8 * st, 0, 1024);
     __syncthreads();
 
-    // each column: its slice sums in ascending order
+    // each column and activation row: its slice sums in ascending order
     uint64_t best = 0;
-    for (int q = tid; q < c1 - c0; q += blockDim.x) {
-        float tot = part[q * nsl];
-        for (int j = 1; j < nsl; ++j) tot += part[q * nsl + j];
+    for (int qm = tid; qm < (c1 - c0) * kM; qm += blockDim.x) {
+        const int q = qm / kM, m = qm % kM;
+        float tot = part[q * nsl * kM + m];
+        for (int j = 1; j < nsl; ++j) tot += part[(q * nsl + j) * kM + m];
         const uint16_t h = f32_to_bf16_rne(tot);
-        a.y[c0 + q] = h;
-        if (a.cand) best = umax64(best, cand_key(h, a.id_base + (uint32_t)(c0 + q)));
+        a.y[(size_t)m * a.ldy + c0 + q] = h;
+        if (kM == 1 && a.cand) best = umax64(best, cand_key(h, a.id_base + (uint32_t)(c0 + q)));
     }
-    if (a.cand) {
+    if (kM == 1 && a.cand) {
         best = warp_max64(best);
         fused_head_keys(a, best, kSWarps, warp, lane);
     }
@@ -1006,12 +1041,16 @@ static int stream_warps(int K, int ru) {
     return 0;
 }
 
+static bool stream_multi_eligible(const QmmArgs &a);
+
 // K % 512 == 0 (every slot piece is a multiple of 16 B) and 16-byte aligned
-// code, scale and bias arrays: the bulk copies' requirements.
+// code, scale and bias arrays: the bulk copies' requirements.  One activation
+// row, or two to four where their limbs leave room for the rings.
 bool qmm_m1_stream_eligible(const QmmArgs &a) {
-    if (a.M != 1 || a.K % 512 != 0) return false;
+    if (a.K % 512 != 0) return false;
     if (!aligned(a.scales, 16) || !aligned(a.biases, 16) || !aligned(a.wq, 16)) return false;
-    return stream_warps(a.K, 4) > 0;
+    if (a.M == 1) return stream_warps(a.K, 4) > 0;
+    return stream_multi_eligible(a);
 }
 
 static size_t g_stream_smem_set[64][3];
@@ -1037,9 +1076,9 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream, int 
 }
 
 // ---------------------------------------------------------- tile ring host --
-static int tile_stages(int K) {
+static int tile_stages(int K, int M) {
     for (int st = kTMaxStages; st >= 2; --st)
-        if (tile_layout(K, st).total <= 226 * 1024) return st;
+        if (tile_layout(K, st, M).total <= 226 * 1024) return st;
     return 0;
 }
 
@@ -1068,19 +1107,18 @@ static TilePlan tile_plan(const QmmArgs &a, int rows) {
 // slot holds one chunk -- and the per-warp ring measured faster there.)  Returns the
 // rows per compute warp of the tile shape, 0 for the per-warp kernel.
 static int tile_ring_shape(const QmmArgs &a) {
-    if (!encode_tiled_fn() || tile_stages(a.K) < 2) return 0;
+    if (!encode_tiled_fn() || tile_stages(a.K, 1) < 2) return 0;
     if (tile_plan(a, TileShape<4>::rows).ntiles >= 4 * num_sms()) return 4;
     if (!a.glu && a.K >= 8192 && tile_plan(a, TileShape<1>::rows).ntiles >= 2 * num_sms()) return 1;
     return 0;
 }
 
-static bool g_tile_smem_set[64][2][2];
-
-template <bool kGlu, int kWR>
+template <bool kGlu, int kWR, int kM>
 static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream, int *ncand) {
+    static bool smem_set[64];
     using Sh = TileShape<kWR>;
-    const int S = tile_stages(a.K);
-    const TileLayout L = tile_layout(a.K, S);
+    const int S = tile_stages(a.K, kM);
+    const TileLayout L = tile_layout(a.K, S, kM);
     const TilePlan plan = tile_plan(a, Sh::rows);
     auto enc = encode_tiled_fn();
     const cuuint32_t box_rows = kGlu ? (cuuint32_t)(Sh::rows / 2) : (cuuint32_t)Sh::rows;
@@ -1111,55 +1149,97 @@ static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream, int *ncand
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (!g_tile_smem_set[dev][kGlu ? 1 : 0][kWR == 4 ? 1 : 0]) {
+    if (!smem_set[dev]) {
         cudaError_t e =
-            cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu, kWR>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+            cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu, kWR, kM>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
         if (e != cudaSuccess) return e;
-        g_tile_smem_set[dev][kGlu ? 1 : 0][kWR == 4 ? 1 : 0] = true;
+        smem_set[dev] = true;
     }
     const int blocks = plan.ntiles < num_sms() ? plan.ntiles : num_sms();
     if (ncand) *ncand = blocks * (kTWarps + kTGroups);
-    return launch_pdl(qmm_m1_tile_kernel<kGlu, kWR>, dim3(blocks), dim3(kTThreads), L.total, stream, a, plan, qmap, smap,
-                      bmap, S);
+    return launch_pdl(qmm_m1_tile_kernel<kGlu, kWR, kM>, dim3(blocks), dim3(kTThreads), L.total, stream, a, plan, qmap,
+                      smap, bmap, S);
 }
 
 // Calls with enough tiles take the tile ring.  Otherwise rows per unit only change
 // how often a lane reuses its activation limbs, never a row's arithmetic, so the
 // choice may follow N: four rows while every warp of the grid still gets two
 // units, fewer when the slice is narrow.
-// The narrow-call kernel: M = 1, no GLU, K longer than 8 chunks, and its layout
-// fits (the rings beside the limbs and the slice sums of a CTA's columns).
+// The narrow-call kernel: no GLU, K longer than 8 chunks, and its layout fits (the
+// rings beside the limbs and the slice sums of a CTA's columns): four slots a
+// warp for one activation row, two for two.
 static int split_maxcols(const QmmArgs &a) {
     const int blocks = a.seg.ncols < num_sms() ? a.seg.ncols : num_sms();
     return blocks > 0 ? (a.seg.ncols + blocks - 1) / blocks : 0;
 }
-static bool split_eligible(const QmmArgs &a) {
-    if (a.glu || (a.K + kChunk - 1) / kChunk <= 8) return false;
-    return split_layout(a.K, split_maxcols(a)).total <= 226 * 1024;
+static int split_stages(const QmmArgs &a) {
+    if (a.glu || (a.K + kChunk - 1) / kChunk <= 8 || a.M > 2) return 0;
+    const int want = a.M == 1 ? kSMaxStages : 2;
+    return split_layout(a.K, split_maxcols(a), a.M, want).total <= 226 * 1024 ? want : 0;
 }
 
-static bool g_split_smem_set[64];
-
+template <int kM>
 static cudaError_t launch_split(const QmmArgs &a, cudaStream_t stream, int *ncand) {
-    const int maxcols = split_maxcols(a);
-    const SplitLayout L = split_layout(a.K, maxcols);
+    static bool smem_set[64];
+    const int maxcols = split_maxcols(a), S = split_stages(a);
+    const SplitLayout L = split_layout(a.K, maxcols, kM, S);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    if (!g_split_smem_set[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(qmm_m1_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+    if (!smem_set[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(qmm_m1_split_kernel<kM>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
         if (e != cudaSuccess) return e;
-        g_split_smem_set[dev] = true;
+        smem_set[dev] = true;
     }
     const int blocks = a.seg.ncols < num_sms() ? a.seg.ncols : num_sms();
     if (ncand) *ncand = blocks * kSWarps;
-    return launch_pdl(qmm_m1_split_kernel, dim3(blocks), dim3(kSWarps * 32), L.total, stream, a, maxcols);
+    return launch_pdl(qmm_m1_split_kernel<kM>, dim3(blocks), dim3(kSWarps * 32), L.total, stream, a, maxcols, S);
+}
+
+// 2 to 4 activation rows on the streaming kernels: each row takes exactly the
+// arithmetic it takes alone (the same lane-chunks, order and tree), so its bits
+// equal those of an M = 1 call; the codes, scales and biases of a tile are read
+// once for all the rows.  Long-K calls take the narrow-call kernel (two rows at
+// most: the limbs of more leave too little room for its rings); the others the
+// tile ring with as many rows per warp as still give every group a tile
+// (four rows by 16 for two activation rows, two by 8 for three or four).
+static int multi_tile_shape(const QmmArgs &a) {
+    if (!encode_tiled_fn() || tile_stages(a.K, a.M) < 2) return 0;
+    const int big = a.M == 2 ? 4 : 2;
+    if (tile_plan(a, 4 * big).ntiles >= 4 * num_sms() || a.glu) return big;
+    return 1;
+}
+
+static bool stream_multi_eligible(const QmmArgs &a) {
+    if (a.M < 2 || a.M > 4) return false;
+    if (!a.glu && (a.K + kChunk - 1) / kChunk > 8) return split_stages(a) > 0;
+    return multi_tile_shape(a) > 0;
+}
+
+template <int kM>
+static cudaError_t launch_multi(const QmmArgs &a, cudaStream_t stream) {
+    if (!a.glu && (a.K + kChunk - 1) / kChunk > 8) {
+        if (kM == 2) return launch_split<2>(a, stream, nullptr);
+        return cudaErrorInvalidValue;
+    }
+    constexpr int kBig = kM == 2 ? 4 : 2;
+    if (multi_tile_shape(a) == kBig)
+        return a.glu ? launch_tile<true, kBig, kM>(a, stream, nullptr) : launch_tile<false, kBig, kM>(a, stream, nullptr);
+    return launch_tile<false, 1, kM>(a, stream, nullptr);
 }
 
 cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream, int *ncand) {
+    switch (a.M) {
+        case 2: return launch_multi<2>(a, stream);
+        case 3: return launch_multi<3>(a, stream);
+        case 4: return launch_multi<4>(a, stream);
+        default: break;
+    }
     const int shape = tile_ring_shape(a);
-    if (shape == 4) return a.glu ? launch_tile<true, 4>(a, stream, ncand) : launch_tile<false, 4>(a, stream, ncand);
-    if (split_eligible(a)) return launch_split(a, stream, ncand);
-    if (shape == 1) return launch_tile<false, 1>(a, stream, ncand);
+    if (shape == 4)
+        return a.glu ? launch_tile<true, 4, 1>(a, stream, ncand) : launch_tile<false, 4, 1>(a, stream, ncand);
+    if (split_stages(a) > 0) return launch_split<1>(a, stream, ncand);
+    if (shape == 1) return launch_tile<false, 1, 1>(a, stream, ncand);
     const long long warps = (long long)num_sms() * stream_warps(a.K, 4);
     const long long rows = a.glu ? 2ll * a.seg.ncols : a.seg.ncols;
     if (rows >= 8 * warps) return launch_ru<4>(a, 0, stream, ncand);

@@ -268,6 +268,17 @@ __device__ __forceinline__ uint32_t tc_code_pair(uint32_t w, uint32_t ws) {
     return r;
 }
 
+// Two outputs' fold, a_i = fma(b, X_i, fma(s, D_i, a_i)), as two packed fp32x2
+// FMAs: each half is the IEEE fma of its own operands, so the bits are those of
+// four scalar fmaf in the same order, at half the instructions.
+__device__ __forceinline__ void tc_fold2(float &a0, float &a1, float s, float d0, float d1, float b, float x0, float x1) {
+    asm("{\n .reg .b64 A, S, D, B, X;\n mov.b64 A, {%0, %1};\n mov.b64 S, {%2, %2};\n mov.b64 D, {%3, %4};\n"
+        " mov.b64 B, {%5, %5};\n mov.b64 X, {%6, %7};\n fma.rn.f32x2 A, S, D, A;\n fma.rn.f32x2 A, B, X, A;\n"
+        " mov.b64 {%0, %1}, A;\n}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(s), "f"(d0), "f"(d1), "f"(b), "f"(x0), "f"(x1));
+}
+
 // acc + lo(w) + hi(w) for a bf16 pair w, each add fp32 += bf16 (Blackwell's
 // mixed-precision add: the bf16 operand is widened exactly, one rounding per add).
 __device__ __forceinline__ float tc_add_bf16x2(float acc, uint32_t w) {
@@ -574,10 +585,10 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             tc_wait_ld();                                                                                           \
             _Pragma("unroll") for (int j = 0; j < CH; j += 4) {                                                     \
                 const float4 xv = *reinterpret_cast<const float4 *>(xg + c + j);                                    \
-                acc[c + j + 0] = fmaf(bf, xv.x, fmaf(sf, __uint_as_float(d[j + 0]), acc[c + j + 0]));               \
-                acc[c + j + 1] = fmaf(bf, xv.y, fmaf(sf, __uint_as_float(d[j + 1]), acc[c + j + 1]));               \
-                acc[c + j + 2] = fmaf(bf, xv.z, fmaf(sf, __uint_as_float(d[j + 2]), acc[c + j + 2]));               \
-                acc[c + j + 3] = fmaf(bf, xv.w, fmaf(sf, __uint_as_float(d[j + 3]), acc[c + j + 3]));               \
+                tc_fold2(acc[c + j + 0], acc[c + j + 1], sf, __uint_as_float(d[j + 0]), __uint_as_float(d[j + 1]),  \
+                         bf, xv.x, xv.y);                                                                           \
+                tc_fold2(acc[c + j + 2], acc[c + j + 3], sf, __uint_as_float(d[j + 2]), __uint_as_float(d[j + 3]),  \
+                         bf, xv.z, xv.w);                                                                           \
             }                                                                                                       \
         }                                                                                                           \
         tc_fence_before();                                                                                          \

@@ -117,3 +117,45 @@ def test_long_k_routes_agree(tf, orc):
     assert bits_equal(glu_small, glu_whole[:, 200:300])
     check_values(host_bits(glu_whole), orc.glu(host_bits(whole)[:, :F], host_bits(whole)[:, F:]),
                  what="GLU stage at K = 17,408")
+
+
+@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("shape", ["head", "glu", "narrow", "long_k"])
+def test_few_rows_equal_one_row_calls(tf, orc, M, shape):
+    """Two to four activation rows on the streaming kernels: every row's outputs
+    are bit for bit those of a call with that row alone, and within the V bar of
+    the oracle on sampled columns.  Shapes: 12,000 rows at K = 5,120 (the tile
+    ring's 16-row or 8-row tiles), a GLU call over 4,800 columns, 2,560 rows at
+    K = 5,120 (4-row x 4,096-K tiles) and 2,560 rows at K = 17,408 (the narrow-call
+    kernel for two rows, the tensor cores above)."""
+    K, N, segs, epi = {
+        "head": (5120, 12000, [(0, 12000)], 0),
+        "glu": (5120, 9600, [(0, 4800), (4800, 4800)], 1),
+        "narrow": (5120, 2560, [(0, 2560)], 0),
+        "long_k": (17408, 2560, [(0, 2560)], 0),
+    }[shape]
+    w = synth.make_weights(N, K, seed=50 + M, tag=synth.TAG_W2)
+    W = DevWeights(w)
+    x = synth.make_x(M, K, seed=60 + M)
+    xt = dev(x)
+    ncols = segs[0][1] if epi else sum(n for _, n in segs)
+    y = empty_bf16(M, ncols)
+    tf.tf_qmm_rows(xt, *W.t(), segs, y, epi=epi)
+    ones = []
+    for m in range(M):
+        o = empty_bf16(1, ncols)
+        tf.tf_qmm_rows(xt[m:m + 1], *W.t(), segs, o, epi=epi)
+        ones.append(o)
+    torch.cuda.synchronize()
+    if not (shape == "long_k" and M > 2):   # 3 and 4 long-K rows run on the tensor cores
+        assert bits_equal(y, torch.cat(ones)), (shape, M)
+    if epi:
+        g = empty_bf16(M, ncols)
+        u = empty_bf16(M, ncols)
+        tf.tf_qmm_rows(xt, *W.t(), [segs[0]], g)
+        tf.tf_qmm_rows(xt, *W.t(), [segs[1]], u)
+        torch.cuda.synchronize()
+        check_values(host_bits(y), orc.glu(host_bits(g), host_bits(u)), what=f"GLU M={M}")
+        sampled(orc, x, w, host_bits(g), np.arange(segs[0][0], segs[0][0] + ncols), K, f"gate M={M}")
+    else:
+        sampled(orc, x, w, host_bits(y), columns_of(segs), K, f"{shape} M={M}")

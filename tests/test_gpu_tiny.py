@@ -95,17 +95,23 @@ def test_ragged_shapes(tf, orc, K, N):
 
 
 def test_row_bits_do_not_depend_on_chunk(tf, orc):
-    """For M > 1 a row's bits do not depend on how many other rows share its
-    call or where it sits in the chunk; every row is within tolerance of the oracle."""
+    """A row's bits do not depend on where it sits in its chunk: calls of 5 or more
+    rows (the tensor cores) agree with one another, and calls of 2 to 4 rows (the
+    streaming kernels, each row taking the one-row arithmetic) agree with one-row
+    calls; every row is within tolerance of the oracle."""
     K, N = 5120, 96
     w = synth.make_weights(N, K, seed=7)
     W = DevWeights(w)
     x = synth.make_x(16, K, seed=7)
     xt = dev(x)
     y16 = qmm(tf, xt, W, [(0, N)])
-    for m0, M in ((0, 2), (3, 5), (9, 7)):
+    for m0, M in ((3, 5), (9, 7)):
         yM = qmm(tf, xt[m0:m0 + M], W, [(0, N)])
         assert bits_equal(yM, y16[m0:m0 + M]), (m0, M)
+    ones = torch.cat([qmm(tf, xt[m:m + 1], W, [(0, N)]) for m in range(16)])
+    for m0, M in ((0, 2), (5, 3), (11, 4)):
+        yM = qmm(tf, xt[m0:m0 + M], W, [(0, N)])
+        assert bits_equal(yM, ones[m0:m0 + M]), (m0, M)
     yo, y64, ad = orc.qmm_rows(x, *w.astuple(), np.arange(N), want_f64=True)
     check_values(host_bits(y16), yo, y64, ad, K, "M=16")
     y1 = qmm(tf, xt[:1], W, [(0, N)])

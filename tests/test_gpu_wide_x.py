@@ -17,10 +17,10 @@ Variants:
   offset7  as window, but the zero weights are code 7 with bias -7 * scale, so
            any split of w into a code part and a bias part leaves two large
            terms that cancel.
-Each runs through every route of tf_qmm_rows: the M = 1 tile ring (16-row and
-4-row tiles, with and without the fused GLU), the per-warp ring, the fp32 M = 1
-kernel (K not a multiple of 512), the tensor-core kernel (M >= 2) and the
-general kernel; and through tf_qmm8_rows.
+Each runs through every route of tf_qmm_rows: the M = 1 tile ring (with and
+without the fused GLU), the narrow-call kernel, the per-warp ring, the fp32 M = 1
+kernel (K not a multiple of 512), three rows on the streaming kernels, the
+tensor-core kernel (M >= 5) and the general kernel; and through tf_qmm8_rows.
 """
 import os
 
@@ -44,12 +44,13 @@ VARIANTS = {   # name: (small exponent range, code of the zero weights or None f
 # name: (M, K, whole rows, segments, epilogue) -- the route each one takes is in its comment
 ROUTES = {
     "tile16": (1, 5120, 9600, [(0, 9600)], 0),                 # tile ring, 600 16-row tiles
-    "tile4": (1, 17408, 2560, [(0, 2560)], 0),                 # tile ring, 4-row x 4,096-K tiles
+    "split": (1, 17408, 2560, [(0, 2560)], 0),                 # narrow-call kernel, (row, K-slice) pairs
     "tile_glu": (1, 5120, 9600, [(0, 4800), (4800, 4800)], 1),  # tile ring, 8-column GLU tiles
     "warp": (1, 5120, 512, [(0, 512)], 0),                     # per-warp ring
     "warp_glu": (1, 5120, 512, [(0, 256), (256, 256)], 1),     # per-warp ring, GLU
     "m1_fp32": (1, 1088, 512, [(0, 512)], 0),                  # K % 512 != 0: the fp32 M = 1 kernel
-    "tc": (4, 5120, 512, [(0, 512)], 0),                       # tensor cores
+    "rows3": (3, 5120, 512, [(0, 512)], 0),                    # three rows on the streaming kernels
+    "tc": (8, 5120, 512, [(0, 512)], 0),                       # tensor cores
     "tc_glu": (16, 5120, 512, [(0, 256), (256, 256)], 1),      # tensor cores, GLU
     "generic": (3, 1088, 512, [(0, 512)], 0),                  # K % 512 != 0, M > 1: general kernel
 }
