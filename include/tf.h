@@ -104,10 +104,15 @@ typedef enum {
  *     w[n,k]  = s[n, k/64] * q[n,k] + b[n, k/64]
  *     out[m,n] = bf16_RNE( sum_{k<K} x[m,k] * w[n,k] )   (fp32 accumulation)
  * for every row n of the segments, in segment order.  The summation order
- * depends on K alone -- never on the segments, their order, N_whole or M's
+ * depends on K alone -- never on the segments, their order, N_whole or a row's
  * position in a chunk -- so a row computed in a slice has the same bits as the
  * same row computed in the whole matrix (PR #1433 review: "a different sk is
- * a different fp32 order").
+ * a different fp32 order").  With M <= 4 (and K % 512 == 0, 16-byte aligned
+ * weights) each activation row's outputs are bit for bit those of a call with
+ * that row alone; calls of 5 or more rows run on the tensor cores, whose rows
+ * agree with one another but not bit for bit with the M <= 4 calls (both meet
+ * the same 2-ulp bar).  Accuracy holds for any activations: a 32-value run
+ * whose values span more than 2^15 is summed as a plain fp32 dot.
  *
  *   x       bf16 [M][ldx] activations.  16-byte aligned, ldx % 8 == 0, ldx >= K.
  *   M       rows of x, 0 <= M <= TF_BATCH_ROWS (M == 0: nothing is enqueued).

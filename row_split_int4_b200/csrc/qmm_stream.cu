@@ -68,7 +68,7 @@ constexpr long long kSpinLimit = 1ll << 22;                  // bounded waits, s
 
 struct StreamLayout {
     int nch, warps;
-    size_t limb_off, sf_off, scale_off, bar_off, ring_off, total;
+    size_t limb_off, cst_off, wm_off, tot_off, bar_off, ring_off, total;
 };
 
 __host__ __device__ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -79,9 +79,10 @@ __host__ __device__ inline StreamLayout stream_layout(int K, int warps, int ru) 
     L.nch = (K + kChunk - 1) / kChunk;
     L.warps = warps;
     L.limb_off = 0;
-    L.sf_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.sf_off + (size_t)L.nch * 32 * 4, 128);
-    L.bar_off = round_up(L.scale_off + (size_t)L.nch * 32 * 4, 128);
+    L.cst_off = round_up(L.limb_off + (size_t)L.nch * 32 * kLimbBytes, 128);
+    L.wm_off = L.cst_off + (size_t)L.nch * 32 * 16;
+    L.tot_off = round_up(L.wm_off + (size_t)L.nch * 4, 16);
+    L.bar_off = round_up(L.tot_off + (size_t)warps * 4 * 4, 128);
     L.ring_off = round_up(L.bar_off + (size_t)warps * stages_for(ru) * 8, 128);
     L.total = L.ring_off + (size_t)warps * stages_for(ru) * slot_bytes(ru);
     return L;
@@ -110,27 +111,26 @@ __device__ __forceinline__ int lane_chunk_pq(const uint4 &q, const uint4 *limb, 
     return (int)(((uint32_t)a2 << 16) + ((uint32_t)a1 << 8) + (uint32_t)a0 - sf8);
 }
 
-// What a lane needs of its lane-chunk c: limbs, the scale 2^(E-23) (-0 marks a
-// wide lane-chunk, NaN a non-finite x), X and 8 sum F.
+// What a lane needs of its lane-chunk c: limbs and the constants the limb
+// preparation left in cst (the scale 2^(E-23), X and 8 sum F as one 16-byte
+// vector; all three zero for a lane-chunk taken in fp32, NaN scale for a
+// non-finite x).
 struct LaneChunk {
     uint4 lm[6];
     float scale, X;
     uint32_t sf8;
-    bool wide;
 };
-__device__ __forceinline__ void load_lane_chunk(LaneChunk &t, const uint4 *limb_l, const int *SFs, const float *Ss,
-                                                int c, int lane) {
+__device__ __forceinline__ void load_lane_chunk(LaneChunk &t, const uint4 *limb_l, const uint4 *cst, int c, int lane) {
 #pragma unroll
     for (int q = 0; q < 6; ++q) t.lm[q] = limb_l[(c * 6 + q) * 32];
-    const int sf = SFs[c * 32 + lane];
-    t.scale = Ss[c * 32 + lane];
-    t.X = __int2float_rn(sf) * t.scale;   // one rounding, then an exact power of two
-    t.sf8 = (uint32_t)sf << 3;
-    t.wide = __float_as_uint(t.scale) == 0x80000000u;
+    const uint4 v = cst[c * 32 + lane];
+    t.scale = __uint_as_float(v.x);
+    t.X = __uint_as_float(v.y);
+    t.sf8 = v.z;
 }
 
 // acc += the lane's x.w over lane-chunk t for a row with codes qv, scale s, bias b
-// (a wide lane-chunk has scale and X zero here and adds nothing).
+// (a lane-chunk taken in fp32 has scale and X zero here and adds nothing).
 __device__ __forceinline__ float lane_chunk_fma(float acc, const uint4 &qv, const LaneChunk &t, float s, float b) {
     const int P = lane_chunk_pq(qv, t.lm, t.sf8);
     acc = fmaf(s, __int2float_rn(P) * t.scale, acc);   // P' * 2^(E-23): exact power-of-two scaling
@@ -159,14 +159,20 @@ __device__ __forceinline__ float wide_dot(float xj, uint32_t word, int lane, flo
 // Fixed-point limbs of x for every lane-chunk, on the bf16 fields alone: x = sign *
 // M * 2^(e-134), M = 128 + mantissa (e >= 1) or the mantissa (e = 0, subnormal, read
 // with e = 1).  With emax the chunk's largest e, F = x * 2^(23-E), E = emax - 126,
-// is sign * M * 2^(e - emax + 15), a left shift when e >= emax - 15 (exact).  A
-// lane-chunk with a nonzero x below that is wide: its 32 raw x go where its limbs
-// would, its scale is -0 and its sum 0.  SFs gets sum F (|sum F| < 2^28), Ss the
-// power of two 2^(E-23) (NaN when the chunk holds a NaN or an infinity).
-__device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, int *SFs, float *Ss, int W,
-                                           int warp, int lane) {
-    // one thread per lane-chunk, all of it in registers: no cross-lane step, so
-    // the whole CTA prepares up to W * 32 lane-chunks in one pass
+// is sign * M * 2^(e - emax + 15), a left shift when e >= emax - 15 (exact).
+// A lane-chunk goes to the fp32 pass (its 32 raw x where its limbs would be, its
+// constants zero, its bit set in wmask[c]) when a nonzero x lies more than 2^15
+// below the largest (fixed point would round it), or when the largest exceeds
+// every other nonzero magnitude by 2^4 or more: a lone outlier, whose product
+// with a zero weight the integer form would carry as two large terms that
+// cancel.  cst gets (2^(E-23), X = 2^(E-23) sum F, 8 sum F, 0) per lane-chunk
+// (|sum F| < 2^28; the scale NaN when the chunk holds a NaN or an infinity).
+// Each warp's 32 lanes take the 32 lane-chunks of one chunk, so a ballot gives
+// the chunk's mask.
+__device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, uint4 *cst, uint32_t *wmask,
+                                           int W, int warp, int lane) {
+    // one thread per lane-chunk, all of it in registers: no cross-lane step but
+    // the ballot, so the whole CTA prepares up to W * 32 lane-chunks in one pass
     const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
     for (int lc = warp * 32 + lane; lc < nch * 32; lc += W * 32) {
         const int c = lc >> 5, l = lc & 31;
@@ -191,21 +197,23 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             }
         }
         bool bad = false;
-        int emax = 0;
+        int emax = 0, e2 = 0;   // the largest and second largest e of a nonzero x (0: none)
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
             const uint32_t ef = (h >> 7) & 0xFFu;
             bad = bad || ef == 0xFFu;
-            const int e = ef == 0 ? 1 : (int)ef;
-            if ((h & 0x7FFFu) != 0) emax = max(emax, e);   // M != 0
+            const int e = (h & 0x7FFFu) == 0 ? 0 : (ef == 0 ? 1 : (int)ef);   // M != 0
+            e2 = max(e2, min(e, emax));
+            emax = max(emax, e);
         }
         uint32_t L[6][4];
 #pragma unroll
         for (int q = 0; q < 6; ++q)
 #pragma unroll
             for (int w = 0; w < 4; ++w) L[q][w] = 0u;
-        bool wide = false;
+        // a nonzero x below emax - 15 would be rounded; emax - e2 >= 5 is a lone outlier
+        bool fallback = e2 > 0 && emax - e2 >= 5;
         int sf = 0;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
@@ -214,7 +222,7 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             const int e = ef == 0 ? 1 : (int)ef;
             const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
             const int sh = e - emax + 15;
-            wide = wide || (sh < 0 && M != 0);
+            fallback = fallback || (sh < 0 && M != 0);
             int F = sh >= 0 ? M << sh : 0;
             if (h & 0x8000u) F = -F;
             sf += F;
@@ -224,20 +232,24 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             L[2 + p][w] |= (uint32_t)((F >> 8) & 0xFF) << sft;
             L[4 + p][w] |= (uint32_t)((F >> 16) & 0xFF) << sft;
         }
-        wide = wide && !bad;
+        fallback = fallback && !bad;
         uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
-        if (wide) {
+        if (fallback) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[q * 32] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+            cst[lc] = make_uint4(0u, 0u, 0u, 0u);
         } else {
 #pragma unroll
             for (int q = 0; q < 6; ++q) dst[q * 32] = make_uint4(L[q][0], L[q][1], L[q][2], L[q][3]);
+            // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
+            const float scale = bad ? __int_as_float(0x7FC00000)
+                                    : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
+            const int sfv = bad ? 0 : sf;
+            cst[lc] = make_uint4(__float_as_uint(scale), __float_as_uint(__int2float_rn(sfv) * scale),
+                                 (uint32_t)sfv << 3, 0u);
         }
-        SFs[lc] = bad || wide ? 0 : sf;
-        // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
-        Ss[lc] = bad ? __int_as_float(0x7FC00000)
-                     : (wide ? __int_as_float(0x80000000)
-                             : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149)));
+        const uint32_t wb = __ballot_sync(0xFFFFFFFFu, fallback);
+        if (l == 0) wmask[c] = wb;
     }
 }
 
@@ -270,12 +282,16 @@ __global__ void __launch_bounds__(1024) argmax_keys_kernel(const uint64_t *cand,
 
 // Chunks per K-slice (see the reduction order above).
 __host__ __device__ constexpr int slice_chunks(int nch) { return nch <= 8 ? nch : 4; }
-__device__ __forceinline__ bool slice_end(int c, int sc, int nch) { return (c + 1) % sc == 0 || c + 1 == nch; }
+__device__ __forceinline__ bool slice_end(int c, int sc, int nch) {
+    return c + 1 == nch || (sc == 4 && (c & 3) == 3);   // sc is nch or 4
+}
 // At the end of a slice: the 32 lanes' sums of the slice by the tree into lane 0,
-// added to the row's total (lane 0's tot; the first slice starts it).
-__device__ __forceinline__ void slice_fold(float &acc, float &tot, int c, int sc) {
+// which adds them to the row's total (the first slice starts it).  The totals
+// live in shared memory, one float per row of the warp, read by lane 0 alone:
+// registers are the kernels' scarce resource.
+__device__ __forceinline__ void slice_fold(float &acc, float *tot, int c, int sc, int lane) {
     const float v = warp_sum_to_lane0(acc);
-    tot = c < sc ? v : tot + v;
+    if (lane == 0) *tot = c < sc ? v : *tot + v;
     acc = 0.0f;
 }
 
@@ -284,8 +300,8 @@ __device__ __forceinline__ void slice_fold(float &acc, float &tot, int c, int sc
 // covered by the slot) adds nothing there.  Full slots pass compile-time nc and
 // kend, so their bounds fold away.
 template <int kRU>
-__device__ __forceinline__ void slot_dot(float (&acc)[kRU], float (&tot)[kRU], const uint8_t *sl, const uint8_t *limbs,
-                                         const int *SFs, const float *Ss, int c0, int nc, int kend, int nch, int sc,
+__device__ __forceinline__ void slot_dot(float (&acc)[kRU], float *tot, const uint8_t *sl, const uint8_t *limbs,
+                                         const uint4 *cst, const uint32_t *wms, int c0, int nc, int kend, int nch, int sc,
                                          int lane) {
     const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
     const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kRU * kSlotQ);
@@ -297,8 +313,8 @@ __device__ __forceinline__ void slot_dot(float (&acc)[kRU], float (&tot)[kRU], c
         const int c = c0 + cc;
         const bool live = cc * kChunk + lane * 32 < kend;
         LaneChunk t;
-        load_lane_chunk(t, limb_l, SFs, Ss, c, lane);
-        const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && t.wide);
+        load_lane_chunk(t, limb_l, cst, c, lane);
+        const uint32_t wm = wms[c];
         if (live) {
 #pragma unroll
             for (int r = 0; r < kRU; ++r) {
@@ -323,7 +339,7 @@ __device__ __forceinline__ void slot_dot(float (&acc)[kRU], float (&tot)[kRU], c
         }
         if (slice_end(c, sc, nch)) {
 #pragma unroll
-            for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot[r], c, sc);
+            for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot + r, c, sc, lane);
         }
     }
 }
@@ -341,8 +357,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     const int G = K / kGroup;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *limbs = smem + L.limb_off;
-    int *SFs = reinterpret_cast<int *>(smem + L.sf_off);
-    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
+    uint4 *csts = reinterpret_cast<uint4 *>(smem + L.cst_off);
+    uint32_t *wms = reinterpret_cast<uint32_t *>(smem + L.wm_off);
     uint8_t *ring = smem + L.ring_off + (size_t)warp * kStages * kSlotBytes;
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kStages * 8);
@@ -434,13 +450,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
     constexpr int kPreStages = kRU >= 4 ? 1 : kStages;
     while (issued < kPreStages && issued < steps) issue_next();
 
-    prep_limbs(a.x, K, nch, limbs, SFs, Ss, W, warp, lane);
+    prep_limbs(a.x, K, nch, limbs, csts, wms, W, warp, lane);
     __syncthreads();
     while (issued < kStages && issued < steps) issue_next();
 
-    float acc[kRU], tot[kRU];
+    float acc[kRU];
 #pragma unroll
-    for (int r = 0; r < kRU; ++r) acc[r] = tot[r] = 0.0f;
+    for (int r = 0; r < kRU; ++r) acc[r] = 0.0f;
+    float *tot = reinterpret_cast<float *>(smem + L.tot_off) + warp * 4;   // lane 0's row totals
     const int sc = slice_chunks(nch);
     uint64_t best = 0;   // fused head: the largest argmax key of the rows this warp wrote
     int slot = 0;
@@ -453,9 +470,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
             failed = failed || !ok;
             const uint8_t *sl = ring + slot * kSlotBytes;
             if (j + 1 < nsl)
-                slot_dot<kRU>(acc, tot, sl, limbs, SFs, Ss, j * (kKS / kChunk), kKS / kChunk, kKS, nch, sc, lane);
+                slot_dot<kRU>(acc, tot, sl, limbs, csts, wms, j * (kKS / kChunk), kKS / kChunk, kKS, nch, sc, lane);
             else
-                slot_dot<kRU>(acc, tot, sl, limbs, SFs, Ss, j * (kKS / kChunk), nc_last, len_last, nch, sc, lane);
+                slot_dot<kRU>(acc, tot, sl, limbs, csts, wms, j * (kKS / kChunk), nc_last, len_last, nch, sc, lane);
             if (++slot == kStages) {
                 slot = 0;
                 par ^= 1u;
@@ -528,7 +545,7 @@ constexpr int kTMaxStages = 6;
 
 struct TileLayout {
     int nch, stages;
-    size_t limb_off, sf_off, scale_off, full_off, empty_off, hdr_off, ctl_off, ring_off, total;
+    size_t limb_off, cst_off, wm_off, full_off, empty_off, hdr_off, ctl_off, tot_off, ring_off, total;
 };
 
 // Shared memory of the tile ring for K, `stages` slots per group and M activation
@@ -538,13 +555,14 @@ __host__ __device__ inline TileLayout tile_layout(int K, int stages, int M = 1) 
     L.nch = (K + kChunk - 1) / kChunk;
     L.stages = stages;
     L.limb_off = 0;
-    L.sf_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.sf_off + (size_t)M * L.nch * 32 * 4, 128);
-    L.full_off = round_up(L.scale_off + (size_t)M * L.nch * 32 * 4, 128);
+    L.cst_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
+    L.wm_off = L.cst_off + (size_t)M * L.nch * 32 * 16;
+    L.full_off = round_up(L.wm_off + (size_t)M * L.nch * 4, 128);
     L.empty_off = L.full_off + (size_t)kTGroups * stages * 8;
     L.hdr_off = L.empty_off + (size_t)kTGroups * stages * 8;    // (tile, chunk) of each slot
     L.ctl_off = L.hdr_off + (size_t)kTGroups * stages * 8;      // claim counter, abort flag
-    L.ring_off = round_up(L.ctl_off + 16, 128);
+    L.tot_off = L.ctl_off + 16;                                   // row totals: 8 floats per compute warp
+    L.ring_off = round_up(L.tot_off + (size_t)kTWarps * 8 * 4, 128);
     L.total = L.ring_off + (size_t)kTGroups * stages * kTSlotBytes;
     return L;
 }
@@ -588,8 +606,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const bool producer = warp >= kTWarps;
     const int grp = producer ? warp - kTWarps : warp / kTGroupWarps, w_in = warp % kTGroupWarps;
     uint8_t *limbs = smem + L.limb_off;
-    int *SFs = reinterpret_cast<int *>(smem + L.sf_off);
-    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
+    uint4 *csts = reinterpret_cast<uint4 *>(smem + L.cst_off);
+    uint32_t *wms = reinterpret_cast<uint32_t *>(smem + L.wm_off);
     int2 *hdr = reinterpret_cast<int2 *>(smem + L.hdr_off) + grp * S;
     int *claim = reinterpret_cast<int *>(smem + L.ctl_off);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.ctl_off) + 1;
@@ -715,7 +733,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
 #pragma unroll
     for (int m = 0; m < kM; ++m)
-        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, SFs + m * lc_n, Ss + m * lc_n,
+        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, csts + m * lc_n, wms + m * nch,
                    kTWarps + kTGroups, warp, lane);
     __syncthreads();
     if (producer) {
@@ -724,11 +742,13 @@ __global__ void __launch_bounds__(kTThreads, 1)
         __syncwarp();
     }
 
-    float acc[kWR][kM], tot[kWR][kM];
+    static_assert(kWR * kM <= 8, "row totals: 8 floats per warp");
+    float acc[kWR][kM];
 #pragma unroll
     for (int r = 0; r < kWR; ++r)
 #pragma unroll
-        for (int m = 0; m < kM; ++m) acc[r][m] = tot[r][m] = 0.0f;
+        for (int m = 0; m < kM; ++m) acc[r][m] = 0.0f;
+    float *tot = reinterpret_cast<float *>(smem + L.tot_off) + (producer ? 0 : warp * 8);   // lane 0's, [r][m]
     const int sc = slice_chunks(nch);
     uint64_t best = 0;
     int slot = 0;
@@ -753,24 +773,32 @@ __global__ void __launch_bounds__(kTThreads, 1)
             if (c >= nch) break;   // chunks past K add nothing
             // nor do lanes past the end of a short last chunk
             const bool live = lane * 32 < K - c * kChunk;
-            // the warp's rows: codes, scale and bias, shared by the activation rows
-            uint4 qv[kWR];
-            float sv[kWR], bv[kWR];
-#pragma unroll
-            for (int r = 0; r < kWR; ++r) {
+            // the warp's rows: codes, scale and bias (read once per activation row
+            // for one row, kept in registers across the rows for more)
+            constexpr int kQ = kM == 1 ? 1 : kWR;
+            uint4 qv[kQ];
+            float sv[kQ], bv[kQ];
+            auto row_operands = [&](int r, uint4 &q, float &sr, float &br) {
                 const int R = tile_row<kGlu, kWR>(w_in, r);
-                qv[r] = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
-                sv[r] = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
-                bv[r] = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+                q = ql[R * (Sh::q / 16) + cc * (kChunk / 32)];
+                sr = bf16_bits_to_f32(sc16[R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+                br = bf16_bits_to_f32(sc16[kRows * (Sh::sb / 2) + R * (Sh::sb / 2) + cc * (kChunk / 64)]);
+            };
+            if (kM > 1) {
+#pragma unroll
+                for (int r = 0; r < kWR; ++r) row_operands(r, qv[r % kQ], sv[r % kQ], bv[r % kQ]);
             }
 #pragma unroll
             for (int m = 0; m < kM; ++m) {
                 LaneChunk t;
-                load_lane_chunk(t, limb_l + m * lc_n * (kLimbBytes / 16), SFs + m * lc_n, Ss + m * lc_n, c, lane);
-                const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && t.wide);
+                load_lane_chunk(t, limb_l + m * lc_n * (kLimbBytes / 16), csts + m * lc_n, c, lane);
+                const uint32_t wm = wms[m * nch + c];
                 if (live) {
 #pragma unroll
-                    for (int r = 0; r < kWR; ++r) acc[r][m] = lane_chunk_fma(acc[r][m], qv[r], t, sv[r], bv[r]);
+                    for (int r = 0; r < kWR; ++r) {
+                        if (kM == 1) row_operands(r, qv[0], sv[0], bv[0]);
+                        acc[r][m] = lane_chunk_fma(acc[r][m], qv[r % kQ], t, sv[r % kQ], bv[r % kQ]);
+                    }
                 }
                 for (uint32_t mm = wm; mm != 0; mm &= mm - 1) {   // wide lane-chunks, warp-uniform
                     const int l = __ffs(mm) - 1;
@@ -792,7 +820,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
                 for (int r = 0; r < kWR; ++r)
 #pragma unroll
-                    for (int m = 0; m < kM; ++m) slice_fold(acc[r][m], tot[r][m], c, sc);
+                    for (int m = 0; m < kM; ++m) slice_fold(acc[r][m], tot + r * kM + m, c, sc, lane);
             }
         }
         __syncwarp();
@@ -813,8 +841,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
                         for (int p = 0; p < kWR / 2; ++p) {
                             const int cj = (kWR / 2) * w_in + p;
                             if (cj < ncol) {
-                                const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p][m]));
-                                const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[2 * p + 1][m]));
+                                const float g = bf16_bits_to_f32(f32_to_bf16_rne(tot[(2 * p) * kM + m]));
+                                const float uu = bf16_bits_to_f32(f32_to_bf16_rne(tot[(2 * p + 1) * kM + m]));
                                 ym[col + cj] = f32_to_bf16_rne(glu_f32(g, uu));
                             }
                         }
@@ -823,7 +851,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
                         for (int r = 0; r < kWR; ++r) {
                             const int cj = kWR * w_in + r;
                             if (cj < ncol) {
-                                const uint16_t hv = f32_to_bf16_rne(tot[r][m]);
+                                const uint16_t hv = f32_to_bf16_rne(tot[r * kM + m]);
                                 ym[col + cj] = hv;
                                 if (kM == 1 && a.cand) best = umax64(best, cand_key(hv, a.id_base + (uint32_t)(col + cj)));
                             }
@@ -874,7 +902,7 @@ constexpr int kSSlot = kSItemQ + 2 * kSItemS;    // 2,304
 
 struct SplitLayout {
     int nch, nsl;
-    size_t limb_off, sf_off, scale_off, part_off, bar_off, ring_off, total;
+    size_t limb_off, cst_off, wm_off, part_off, bar_off, ring_off, total;
 };
 
 // M activation rows (limbs, sums and scales of each), `stages` slots per warp.
@@ -883,9 +911,9 @@ __host__ __device__ inline SplitLayout split_layout(int K, int maxcols, int M, i
     L.nch = (K + kChunk - 1) / kChunk;
     L.nsl = (L.nch + 3) / 4;
     L.limb_off = 0;
-    L.sf_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
-    L.scale_off = round_up(L.sf_off + (size_t)M * L.nch * 32 * 4, 128);
-    L.part_off = round_up(L.scale_off + (size_t)M * L.nch * 32 * 4, 128);
+    L.cst_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
+    L.wm_off = L.cst_off + (size_t)M * L.nch * 32 * 16;
+    L.part_off = round_up(L.wm_off + (size_t)M * L.nch * 4, 128);
     L.bar_off = round_up(L.part_off + (size_t)maxcols * L.nsl * M * 4, 128);
     L.ring_off = round_up(L.bar_off + (size_t)kSWarps * kSMaxStages * 8, 128);
     L.total = L.ring_off + (size_t)kSWarps * stages * kSSlot;
@@ -900,8 +928,8 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     const int G = K / kGroup;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *limbs = smem + L.limb_off;
-    int *SFs = reinterpret_cast<int *>(smem + L.sf_off);
-    float *Ss = reinterpret_cast<float *>(smem + L.scale_off);
+    uint4 *csts = reinterpret_cast<uint4 *>(smem + L.cst_off);
+    uint32_t *wms = reinterpret_cast<uint32_t *>(smem + L.wm_off);
     float *part = reinterpret_cast<float *>(smem + L.part_off);
     uint8_t *ring = smem + L.ring_off + (size_t)warp * kSStages * kSSlot;
     const uint32_t ring_s = smem_addr(ring);
@@ -963,7 +991,7 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
 #pragma unroll
     for (int m = 0; m < kM; ++m)
-        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, SFs + m * lc_n, Ss + m * lc_n,
+        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, csts + m * lc_n, wms + m * nch,
                    kSWarps, warp, lane);
     __syncthreads();
 
@@ -991,8 +1019,8 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
 #pragma unroll
             for (int m = 0; m < kM; ++m) {
                 LaneChunk lc;
-                load_lane_chunk(lc, limb_l + m * lc_n * (kLimbBytes / 16), SFs + m * lc_n, Ss + m * lc_n, c, lane);
-                const uint32_t wm = __ballot_sync(0xFFFFFFFFu, live && lc.wide);
+                load_lane_chunk(lc, limb_l + m * lc_n * (kLimbBytes / 16), csts + m * lc_n, c, lane);
+                const uint32_t wm = wms[m * nch + c];
                 if (live) acc[m] = lane_chunk_fma(acc[m], qv, lc, sv, bv);
                 for (uint32_t mm = wm; mm != 0; mm &= mm - 1) {   // wide lane-chunks, warp-uniform
                     const int l = __ffs(mm) - 1;
