@@ -238,17 +238,44 @@ class DecodeStep:
         tf.tf_gather_rows(self.y, self.y_h, [self.H // 2] * 2, window_bytes=self.window, stream=stream)
         if head_events is not None:
             head_events[0].record(stream)
+        self.run_head(stream)
+        if head_events is not None:
+            head_events[1].record(stream)
+
+    def run_head(self, stream):
+        """Per half the fused lm_head qmm and argmax word, then the pick."""
+        tf = self.tf
         for h in range(2):
             r0, n = self.head_rows[h]
             tf.tf_qmm_argmax_rows(self.x_head, *self.Wlm, (r0, n), r0, self.logits[h], self.words[h],
                                   self.head_scratch[h], stream=stream)
         tf.tf_pick(self.words, self.ids, stream=stream)
-        if head_events is not None:
-            head_events[1].record(stream)
 
     def lm_head_half(self, h, stream):
         """One half of the lm_head qmm alone: the kernel the fused head runs."""
         self.tf.tf_qmm_rows(self.x_head, *self.Wlm, [self.head_rows[h]], self.logits[h], stream=stream)
+
+
+def capture_graphs(torch, step):
+    """CUDA graphs of the decode step, of its head (both fused halves and the pick)
+    and of each lm_head half's qmm alone, captured on a side stream after one
+    eager pass there."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step.run(side)
+    torch.cuda.current_stream().wait_stream(side)
+    out = {"step": torch.cuda.CUDAGraph(), "head": torch.cuda.CUDAGraph(),
+           "lm": [torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()]}
+    with torch.cuda.graph(out["step"]):
+        step.run(torch.cuda.current_stream())
+    with torch.cuda.graph(out["head"]):
+        step.run_head(torch.cuda.current_stream())
+    for h in range(2):
+        with torch.cuda.graph(out["lm"][h]):
+            step.lm_head_half(h, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    return out
 
 
 def make_host_weights(synth, seed=0):
@@ -422,10 +449,19 @@ def run_kernel(args):
     x = torch.randn(args.M, K, device="cuda", generator=g).to(torch.bfloat16)
     cols = segs[0][1] if epi else sum(n for _, n in segs)
     y = torch.empty(args.M, cols, dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        tf.tf_qmm_rows(x, wq, sc, bi, segs, y, epi=epi, stream=torch.cuda.current_stream())
+    call()
+    if not args.no_graph:   # one call in a CUDA graph: a replay has no host work per kernel
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        call = g.replay
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.reps)]
     for a, b in ev:
         a.record()
-        tf.tf_qmm_rows(x, wq, sc, bi, segs, y, epi=epi)
+        call()
         b.record()
     torch.cuda.synchronize()
     us = [a.elapsed_time(b) * 1e3 for a, b in ev]
@@ -504,12 +540,23 @@ def run_sweep(args):
             for r in range(max(3, args.warmup)):
                 rep(r)
             torch.cuda.synchronize()
+            run = rep
+            if not args.no_graph:   # one CUDA graph per weight replica, replayed in turn
+                gs = []
+                for r in range(nrep):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        stream = torch.cuda.current_stream()
+                        rep(r)
+                    gs.append(g)
+                stream = torch.cuda.current_stream()
+                run = lambda r: gs[r % nrep].replay()   # noqa: E731
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             sampler = ClockSampler(0)
             with sampler:
                 e0.record(stream)
                 for r in range(args.reps):
-                    rep(r)
+                    run(r)
                 e1.record(stream)
                 torch.cuda.synchronize()
             us = e0.elapsed_time(e1) * 1e3 / args.reps
@@ -545,6 +592,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every call from the host (no CUDA graph)")
     ap.add_argument("--sweep", action="store_true", help="per-point sweep over M and the four shapes")
     ap.add_argument("--reps", type=int, default=1000)
     ap.add_argument("--kernel", choices=sorted(KERNELS) + list(ADJACENT),
@@ -597,6 +645,23 @@ def main():
     def ev_pair():
         return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
+    # The step, the head and one lm_head half, each captured once into a CUDA graph
+    # (the same library calls; a replay launches the same kernels with no host
+    # work per kernel), so that host launch costs do not starve the GPU.
+    graphs, graph_error = None, ""
+    if not args.no_graph:
+        try:
+            graphs = capture_graphs(torch, step)
+        except Exception as e:  # noqa: BLE001
+            graphs = None
+            graph_error = str(e)[:200]
+
+    def run_step():
+        if graphs:
+            graphs["step"].replay()
+        else:
+            step.run(stream)
+
     t0, t1 = ev_pair()
     sampler = ClockSampler(local)
     barrier()
@@ -604,20 +669,29 @@ def main():
         # 1. the whole step, K times back to back
         t0.record(stream)
         for i in range(K):
-            step.run(stream)
+            run_step()
         t1.record(stream)
         barrier()
         elapsed_ms = t0.elapsed_time(t1)
         # 2. the head chain of each step (both halves' qmm + argmax word, the pick)
         hd_ev = [ev_pair() for _ in range(K)]
         for i in range(K):
-            step.run(stream, head_events=hd_ev[i])
+            if graphs:
+                run_step()   # keeps the head's inputs in their place in the step's stream of work
+                hd_ev[i][0].record(stream)
+                graphs["head"].replay()
+                hd_ev[i][1].record(stream)
+            else:
+                step.run(stream, head_events=hd_ev[i])
         barrier()
         # 3. one lm_head half's qmm alone, halves alternating
         lm_ev = [ev_pair() for _ in range(K)]
         for i in range(K):
             lm_ev[i][0].record(stream)
-            step.lm_head_half(i % 2, stream)
+            if graphs:
+                graphs["lm"][i % 2].replay()
+            else:
+                step.lm_head_half(i % 2, stream)
             lm_ev[i][1].record(stream)
         barrier()
     lm_ms = [a.elapsed_time(b) for (a, b) in lm_ev]
@@ -674,7 +748,10 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "one GPU, two row halves",
                        "timed_regions": "value: K steps between two events; head: event pair per step around "
                                         "both fused halves and the pick; roofline: K lone lm_head-half qmm "
-                                        "launches, each in an event pair"},
+                                        "launches, each in an event pair",
+                       "launch": ("each timed region replays CUDA graphs of the library calls"
+                                  if graphs else "every call launched from the host" +
+                                  (f" (graph capture failed: {graph_error})" if not args.no_graph else ""))},
             "step_hbm_frac": {"measured": round(value / peak, 4), "spec_8000": round(value / SPEC_HBM_GBS, 4),
                               "peak_kind": peak_kind},
             "lm_head_argmax_us_per_token": round(statistics.fmean(head_ms) * 1e3, 2),

@@ -111,8 +111,9 @@ typedef enum {
  * weights) each activation row's outputs are bit for bit those of a call with
  * that row alone; calls of 5 or more rows run on the tensor cores, whose rows
  * agree with one another but not bit for bit with the M <= 4 calls (both meet
- * the same 2-ulp bar).  Accuracy holds for any activations: a 32-value run
- * whose values span more than 2^15 is summed as a plain fp32 dot.
+ * the same 2-ulp bar).  A 32-value run of x dominated by one or two outliers
+ * (no third value within 2^4 of its largest) is summed as a plain fp32 dot,
+ * so an outlier whose weight is zero adds exactly nothing.
  *
  *   x       bf16 [M][ldx] activations.  16-byte aligned, ldx % 8 == 0, ldx >= K.
  *   M       rows of x, 0 <= M <= TF_BATCH_ROWS (M == 0: nothing is enqueued).

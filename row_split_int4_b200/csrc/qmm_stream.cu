@@ -16,25 +16,27 @@
 //     the activations by dp4a, 4 products and their sum per instruction, in exact
 //     integer arithmetic.
 //
-// Exact integer dot (per lane-chunk: the 32 x a lane meets in one 1,024-K chunk).
+// Integer dot (per lane-chunk: the 32 x a lane meets in one 1,024-K chunk).
 // The 32 bf16 x are put in fixed point with the chunk's own exponent E (every
 // |x| < 2^E, E the smallest such over the chunk): F = x * 2^(23-E), |F| < 2^23,
-// exact for every x within 2^15 of the chunk's largest magnitude.  F is kept as
+// exact for every x within 2^15 of the chunk's largest magnitude and rounded to
+// nearest even below (an error under 2^-23 of the largest |x|).  F is kept as
 // three bytes, F = L2*2^16 + L1*2^8 + L0 (L2 signed), and with the code written
 // as q = (q - 8) + 8 and the weight as w = s (q - 8) + (b + 8 s),
 //     P' = sum (q - 8) F = 2^16 sum q L2 + 2^8 sum q L1 + sum q L0 - 8 sum F
 // comes from three int32 dp4a accumulators that cannot overflow (32 * 15 * 255 <
 // 2^17); |P'| < 2^31, so P' is exact in int32 and is rounded once to fp32.  The
-// lane adds s * 2^(E-23) * P' and (b + 8 s) * X, X = 2^(E-23) sum F = the exact
-// sum of the 32 x rounded once.  Taking the code about its middle keeps the two
-// terms near the size of their sum for the usual bias b ~ -8 s, where s q and b
-// alone would be large terms that cancel.
-// A lane-chunk holding a nonzero x more than 2^15 below its largest ("wide":
-// fixed point would round it) keeps its 32 raw x instead of limbs, and the warp
-// takes it element by element: lane j forms w_j = s q_j + b and x_j w_j in fp32,
-// a fixed butterfly adds the 32 products, and the owning lane adds the sum -- a
-// plain fp32 dot for that lane-chunk, whose value does not depend on how far
-// below the largest x the others lie.
+// lane adds s * 2^(E-23) * P' and (b + 8 s) * X, X = 2^(E-23) sum F = the sum of
+// the 32 x rounded once.  Taking the code about its middle keeps the two terms
+// near the size of their sum for the usual bias b ~ -8 s, where s q and b alone
+// would be large terms that cancel.
+// A lane-chunk dominated by one or two outliers (at most two nonzero x within
+// 2^4 of its largest, and smaller nonzero x beside them) keeps its 32 raw x
+// instead of limbs, and the warp takes it element by element: lane j forms
+// w_j = s q_j + b and x_j w_j in fp32, a fixed butterfly adds the 32 products,
+// and the owning lane adds the sum -- a plain fp32 dot for that lane-chunk, so
+// an outlier whose weight is zero adds exactly nothing and sets no grid for the
+// others.
 // A chunk holding NaN or +-Inf gets the scale NaN, so the row's result is NaN.
 //
 // Order of every operation depends on K alone, never on the rows a launch
@@ -159,16 +161,17 @@ __device__ __forceinline__ float wide_dot(float xj, uint32_t word, int lane, flo
 // Fixed-point limbs of x for every lane-chunk, on the bf16 fields alone: x = sign *
 // M * 2^(e-134), M = 128 + mantissa (e >= 1) or the mantissa (e = 0, subnormal, read
 // with e = 1).  With emax the chunk's largest e, F = x * 2^(23-E), E = emax - 126,
-// is sign * M * 2^(e - emax + 15), a left shift when e >= emax - 15 (exact).
+// is sign * M * 2^(e - emax + 15): a left shift when e >= emax - 15 (exact), else
+// a right shift rounded to nearest even (an error below 2^-23 of the largest |x|,
+// the size of an fp32 rounding of a sum that holds the largest product).
 // A lane-chunk goes to the fp32 pass (its 32 raw x where its limbs would be, its
-// constants zero, its bit set in wmask[c]) when a nonzero x lies more than 2^15
-// below the largest (fixed point would round it), or when the largest exceeds
-// every other nonzero magnitude by 2^4 or more: a lone outlier, whose product
-// with a zero weight the integer form would carry as two large terms that
-// cancel.  cst gets (2^(E-23), X = 2^(E-23) sum F, 8 sum F, 0) per lane-chunk
-// (|sum F| < 2^28; the scale NaN when the chunk holds a NaN or an infinity).
-// Each warp's 32 lanes take the 32 lane-chunks of one chunk, so a ballot gives
-// the chunk's mask.
+// constants zero, its bit set in wmask[c]) when one or two values dominate it --
+// at most two nonzero x within 2^4 of the largest and some smaller nonzero x: an
+// outlier whose weight may be zero would otherwise set the grid of the others and
+// ride in both integer terms.  cst gets (2^(E-23), X = 2^(E-23) sum F, 8 sum F, 0)
+// per lane-chunk (|sum F| < 2^28; the scale NaN when the chunk holds a NaN or an
+// infinity).  Each warp's 32 lanes take the 32 lane-chunks of one chunk, so a
+// ballot gives the chunk's mask.
 __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, uint4 *cst, uint32_t *wmask,
                                            int W, int warp, int lane) {
     // one thread per lane-chunk, all of it in registers: no cross-lane step but
@@ -197,23 +200,21 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             }
         }
         bool bad = false;
-        int emax = 0, e2 = 0;   // the largest and second largest e of a nonzero x (0: none)
+        int emax = 0;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
             const uint32_t ef = (h >> 7) & 0xFFu;
             bad = bad || ef == 0xFFu;
-            const int e = (h & 0x7FFFu) == 0 ? 0 : (ef == 0 ? 1 : (int)ef);   // M != 0
-            e2 = max(e2, min(e, emax));
-            emax = max(emax, e);
+            const int e = ef == 0 ? 1 : (int)ef;
+            if ((h & 0x7FFFu) != 0) emax = max(emax, e);   // M != 0
         }
         uint32_t L[6][4];
 #pragma unroll
         for (int q = 0; q < 6; ++q)
 #pragma unroll
             for (int w = 0; w < 4; ++w) L[q][w] = 0u;
-        // a nonzero x below emax - 15 would be rounded; emax - e2 >= 5 is a lone outlier
-        bool fallback = e2 > 0 && emax - e2 >= 5;
+        int near = 0, below = 0;   // nonzero x within 2^4 of the largest (sh >= 12), and the rest
         int sf = 0;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
@@ -222,8 +223,17 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             const int e = ef == 0 ? 1 : (int)ef;
             const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
             const int sh = e - emax + 15;
-            fallback = fallback || (sh < 0 && M != 0);
-            int F = sh >= 0 ? M << sh : 0;
+            near += (M != 0 && sh >= 12) ? 1 : 0;
+            below += (M != 0 && sh < 12) ? 1 : 0;
+            int F;
+            if (sh >= 0) {
+                F = M << sh;
+            } else if (sh > -9) {
+                const int d = -sh;
+                F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
+            } else {
+                F = 0;
+            }
             if (h & 0x8000u) F = -F;
             sf += F;
             // value t of the lane-chunk: word t >> 3, byte (t & 7) >> 1 of limb vector 2 limb + (t & 1)
@@ -232,7 +242,7 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             L[2 + p][w] |= (uint32_t)((F >> 8) & 0xFF) << sft;
             L[4 + p][w] |= (uint32_t)((F >> 16) & 0xFF) << sft;
         }
-        fallback = fallback && !bad;
+        const bool fallback = !bad && near <= 2 && below > 0;
         uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
         if (fallback) {
 #pragma unroll

@@ -19,7 +19,9 @@ Variants:
            zero weights: the large value's product cancels to exactly zero;
   offset7  as window, but the zero weights are code 7 with bias -7 * scale, so
            any split of w into a code part and a bias part leaves two large
-           terms that cancel.
+           terms that cancel;
+  pair     as zero, with a second outlier of 2^9 (also of weight zero) in every
+           run: two dominating values.
 Each runs through every route of tf_qmm_rows: the M = 1 tile ring (with and
 without the fused GLU), the narrow-call kernel, the per-warp ring, the fp32 M = 1
 kernel (K not a multiple of 512), three rows on the streaming kernels, the
@@ -42,6 +44,7 @@ VARIANTS = {   # name: (small exponent range, code of the zero weights or None f
     "natural": ((-14, -10), None),
     "window": ((-5, -4), 8),
     "offset7": ((-5, -4), 7),
+    "pair": ((-14, -10), 8),
 }
 
 # name: (M, K, whole rows, segments, epilogue) -- the route each one takes is in its comment
@@ -70,6 +73,11 @@ def inputs(variant, M, K, N, seed):
     small, code = VARIANTS[variant]
     pos = synth.wide_positions(K, seed)
     x = synth.make_x_wide(M, K, small_exp=small, seed=seed, positions=pos)
+    if variant == "pair":   # a second outlier, 2^9, one place after the first within its run
+        pos2 = (pos // 32) * 32 + (pos % 32 + 1) % 32
+        x2 = synth.make_x_wide(M, K, big_exp=9, small_exp=small, seed=seed + 1, positions=pos2)
+        x[:, pos2] = x2[:, pos2]
+        pos = np.concatenate([pos, pos2])
     w = synth.make_weights(N, K, seed=seed, tag=synth.TAG_W2)
     if code is not None:
         w = synth.with_zero_weights(w, pos, offset=code)
