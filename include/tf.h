@@ -107,10 +107,10 @@ typedef enum {
  * depends on K alone -- never on the segments, their order, N_whole or a row's
  * position in a chunk -- so a row computed in a slice has the same bits as the
  * same row computed in the whole matrix (PR #1433 review: "a different sk is
- * a different fp32 order").  With M <= 4 (and K % 512 == 0, 16-byte aligned
+ * a different fp32 order").  With M <= 3 (and K % 512 == 0, 16-byte aligned
  * weights) each activation row's outputs are bit for bit those of a call with
- * that row alone; calls of 5 or more rows run on the tensor cores, whose rows
- * agree with one another but not bit for bit with the M <= 4 calls (both meet
+ * that row alone; calls of 4 or more rows run on the tensor cores, whose rows
+ * agree with one another but not bit for bit with the M <= 3 calls (both meet
  * the same 2-ulp bar).  A 32-value run of x dominated by one or two outliers
  * (no third value within 2^4 of its largest) is summed as a plain fp32 dot,
  * so an outlier whose weight is zero adds exactly nothing.

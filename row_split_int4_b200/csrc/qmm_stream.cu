@@ -1234,13 +1234,13 @@ static cudaError_t launch_split(const QmmArgs &a, cudaStream_t stream, int *ncan
     return launch_pdl(qmm_m1_split_kernel<kM>, dim3(blocks), dim3(kSWarps * 32), L.total, stream, a, maxcols, S);
 }
 
-// 2 to 4 activation rows on the streaming kernels: each row takes exactly the
+// 2 or 3 activation rows on the streaming kernels: each row takes exactly the
 // arithmetic it takes alone (the same lane-chunks, order and tree), so its bits
 // equal those of an M = 1 call; the codes, scales and biases of a tile are read
 // once for all the rows.  Long-K calls take the narrow-call kernel (two rows at
 // most: the limbs of more leave too little room for its rings); the others the
 // tile ring with as many rows per warp as still give every group a tile
-// (four rows by 16 for two activation rows, two by 8 for three or four).
+// (four rows by 16 for two activation rows, two by 8 for three).
 static int multi_tile_shape(const QmmArgs &a) {
     if (!encode_tiled_fn() || tile_stages(a.K, a.M) < 2) return 0;
     const int big = a.M == 2 ? 4 : 2;
@@ -1249,7 +1249,9 @@ static int multi_tile_shape(const QmmArgs &a) {
 }
 
 static bool stream_multi_eligible(const QmmArgs &a) {
-    if (a.M < 2 || a.M > 4) return false;
+    // four rows measured slower here than on the tensor cores (lm_head half 286 us
+    // against 260 us), so the streaming kernels take two and three
+    if (a.M < 2 || a.M > 3) return false;
     if (!a.glu && (a.K + kChunk - 1) / kChunk > 8) return split_stages(a) > 0;
     return multi_tile_shape(a) > 0;
 }
@@ -1270,7 +1272,6 @@ cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream, int *nca
     switch (a.M) {
         case 2: return launch_multi<2>(a, stream);
         case 3: return launch_multi<3>(a, stream);
-        case 4: return launch_multi<4>(a, stream);
         default: break;
     }
     const int shape = tile_ring_shape(a);

@@ -96,7 +96,7 @@ def test_ragged_shapes(tf, orc, K, N):
 
 def test_row_bits_do_not_depend_on_chunk(tf, orc):
     """A row's bits do not depend on where it sits in its chunk: calls of 5 or more
-    rows (the tensor cores) agree with one another, and calls of 2 to 4 rows (the
+    rows (the tensor cores) agree with one another, and calls of 2 or 3 rows (the
     streaming kernels, each row taking the one-row arithmetic) agree with one-row
     calls; every row is within tolerance of the oracle."""
     K, N = 5120, 96
@@ -109,7 +109,7 @@ def test_row_bits_do_not_depend_on_chunk(tf, orc):
         yM = qmm(tf, xt[m0:m0 + M], W, [(0, N)])
         assert bits_equal(yM, y16[m0:m0 + M]), (m0, M)
     ones = torch.cat([qmm(tf, xt[m:m + 1], W, [(0, N)]) for m in range(16)])
-    for m0, M in ((0, 2), (5, 3), (11, 4)):
+    for m0, M in ((0, 2), (5, 3)):
         yM = qmm(tf, xt[m0:m0 + M], W, [(0, N)])
         assert bits_equal(yM, ones[m0:m0 + M]), (m0, M)
     yo, y64, ad = orc.qmm_rows(x, *w.astuple(), np.arange(N), want_f64=True)
