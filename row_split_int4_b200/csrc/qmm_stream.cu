@@ -170,61 +170,52 @@ __device__ __forceinline__ float wide_dot(float xj, uint32_t word, int lane, flo
 // outlier whose weight may be zero would otherwise set the grid of the others and
 // ride in both integer terms.  cst gets (2^(E-23), X = 2^(E-23) sum F, 8 sum F, 0)
 // per lane-chunk (|sum F| < 2^28; the scale NaN when the chunk holds a NaN or an
-// infinity).  Each warp's 32 lanes take the 32 lane-chunks of one chunk, so a
-// ballot gives the chunk's mask.
+// infinity).
 __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, uint8_t *limbs, uint4 *cst, uint32_t *wmask,
                                            int W, int warp, int lane) {
-    // one thread per lane-chunk, all of it in registers: no cross-lane step but
-    // the ballot, so the whole CTA prepares up to W * 32 lane-chunks in one pass
+    // Four threads per lane-chunk, each with 8 of its values (one 16-byte load, one
+    // word of every limb vector), the lane-chunk's largest exponent, counts and sum
+    // joined by shuffles within the four; all threads of the CTA take part, so the
+    // preparation is short next to the first ring fill.
     const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
-    for (int lc = warp * 32 + lane; lc < nch * 32; lc += W * 32) {
-        const int c = lc >> 5, l = lc & 31;
-        const int k0 = c * kChunk + l * 32;
-        uint32_t hv[16];   // the 32 bf16 x of the lane-chunk, two per word (zero past K)
-        if (x16 && k0 + 32 <= K) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(x + k0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 v = src[i];
-                hv[4 * i] = v.x;
-                hv[4 * i + 1] = v.y;
-                hv[4 * i + 2] = v.z;
-                hv[4 * i + 3] = v.w;
-            }
+    uint8_t *wm8 = reinterpret_cast<uint8_t *>(wmask);   // byte j of chunk c: lane-chunks 8j .. 8j + 7
+    for (int u = warp * 32 + lane; u < nch * 128; u += W * 32) {
+        const int lc = u >> 2, w = u & 3, c = lc >> 5, l = lc & 31;
+        const int k0 = c * kChunk + l * 32 + w * 8;
+        uint32_t hv[4];   // values 8w .. 8w + 7 of the lane-chunk, two per word (zero past K)
+        if (x16 && k0 + 8 <= K) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(x + k0);
+            hv[0] = v.x;
+            hv[1] = v.y;
+            hv[2] = v.z;
+            hv[3] = v.w;
         } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const uint32_t lo = k0 + 2 * i < K ? x[k0 + 2 * i] : 0u;
                 const uint32_t hi = k0 + 2 * i + 1 < K ? x[k0 + 2 * i + 1] : 0u;
                 hv[i] = lo | (hi << 16);
             }
         }
-        bool bad = false;
-        int emax = 0;
+        int emax = 0, bad = 0;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
+        for (int t = 0; t < 8; ++t) {
             const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-            const uint32_t ef = (h >> 7) & 0xFFu;
-            bad = bad || ef == 0xFFu;
-            const int e = ef == 0 ? 1 : (int)ef;
-            if ((h & 0x7FFFu) != 0) emax = max(emax, e);   // M != 0
+            const int ef = (int)((h >> 7) & 0xFFu);
+            bad |= ef == 0xFF ? 1 : 0;
+            if ((h & 0x7FFFu) != 0) emax = max(emax, max(ef, 1));   // M != 0; a subnormal reads e = 1
         }
-        uint32_t L[6][4];
+        emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 1));
+        emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 2));
+        uint32_t L[6] = {0u, 0u, 0u, 0u, 0u, 0u};   // word w of limb vector 2 limb + parity
+        int cnt = 0, sf = 0;   // cnt: nonzero x within 2^4 of the largest (bits 0..7), smaller ones (8..15), bad (16..)
 #pragma unroll
-        for (int q = 0; q < 6; ++q)
-#pragma unroll
-            for (int w = 0; w < 4; ++w) L[q][w] = 0u;
-        int near = 0, below = 0;   // nonzero x within 2^4 of the largest (sh >= 12), and the rest
-        int sf = 0;
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
+        for (int t = 0; t < 8; ++t) {
             const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-            const uint32_t ef = (h >> 7) & 0xFFu;
-            const int e = ef == 0 ? 1 : (int)ef;
+            const int ef = (int)((h >> 7) & 0xFFu);
             const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
-            const int sh = e - emax + 15;
-            near += (M != 0 && sh >= 12) ? 1 : 0;
-            below += (M != 0 && sh < 12) ? 1 : 0;
+            const int sh = max(ef, 1) - emax + 15;
+            if (M != 0) cnt += sh >= 12 ? 1 : 256;
             int F;
             if (sh >= 0) {
                 F = M << sh;
@@ -236,30 +227,46 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             }
             if (h & 0x8000u) F = -F;
             sf += F;
-            // value t of the lane-chunk: word t >> 3, byte (t & 7) >> 1 of limb vector 2 limb + (t & 1)
-            const int w = t >> 3, p = t & 1, sft = 8 * ((t & 7) >> 1);
-            L[0 + p][w] |= (uint32_t)(F & 0xFF) << sft;
-            L[2 + p][w] |= (uint32_t)((F >> 8) & 0xFF) << sft;
-            L[4 + p][w] |= (uint32_t)((F >> 16) & 0xFF) << sft;
+            // value 8w + t: byte t >> 1 of word w of limb vectors 2 limb + (t & 1)
+            const int p = t & 1, sft = 8 * (t >> 1);
+            L[0 + p] |= (uint32_t)(F & 0xFF) << sft;
+            L[2 + p] |= (uint32_t)((F >> 8) & 0xFF) << sft;
+            L[4 + p] |= (uint32_t)((F >> 16) & 0xFF) << sft;
         }
-        const bool fallback = !bad && near <= 2 && below > 0;
+        cnt += bad << 16;
+        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 1);
+        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 2);
+        sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 1);
+        sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 2);
+        const bool any_bad = (cnt >> 16) != 0;
+        const bool fallback = !any_bad && (cnt & 0xFF) <= 2 && ((cnt >> 8) & 0xFF) > 0;
         uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
         if (fallback) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q * 32] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
-            cst[lc] = make_uint4(0u, 0u, 0u, 0u);
+            dst[w * 32] = make_uint4(hv[0], hv[1], hv[2], hv[3]);   // values 8w .. 8w + 7 in vector w
         } else {
 #pragma unroll
-            for (int q = 0; q < 6; ++q) dst[q * 32] = make_uint4(L[q][0], L[q][1], L[q][2], L[q][3]);
-            // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
-            const float scale = bad ? __int_as_float(0x7FC00000)
-                                    : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
-            const int sfv = bad ? 0 : sf;
-            cst[lc] = make_uint4(__float_as_uint(scale), __float_as_uint(__int2float_rn(sfv) * scale),
-                                 (uint32_t)sfv << 3, 0u);
+            for (int q = 0; q < 6; ++q) reinterpret_cast<uint32_t *>(dst + q * 32)[w] = L[q];
         }
-        const uint32_t wb = __ballot_sync(0xFFFFFFFFu, fallback);
-        if (l == 0) wmask[c] = wb;
+        if (w == 0) {
+            if (fallback) {
+                cst[lc] = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
+                const float scale = any_bad ? __int_as_float(0x7FC00000)
+                                            : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
+                const int sfv = any_bad ? 0 : sf;
+                cst[lc] = make_uint4(__float_as_uint(scale), __float_as_uint(__int2float_rn(sfv) * scale),
+                                     (uint32_t)sfv << 3, 0u);
+            }
+        }
+        // the warp's 32 threads hold 8 lane-chunks of chunk c (l of lane 0 a multiple of 8)
+        const uint32_t b = __ballot_sync(0xFFFFFFFFu, fallback && w == 0);
+        if (lane == 0) {
+            uint32_t m8 = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m8 |= ((b >> (4 * j)) & 1u) << j;
+            wm8[c * 4 + (l >> 3)] = (uint8_t)m8;
+        }
     }
 }
 
@@ -310,9 +317,8 @@ __device__ __forceinline__ void slice_fold(float &acc, float *tot, int c, int sc
 // covered by the slot) adds nothing there.  Full slots pass compile-time nc and
 // kend, so their bounds fold away.
 template <int kRU>
-__device__ __forceinline__ void slot_dot(float (&acc)[kRU], float *tot, const uint8_t *sl, const uint8_t *limbs,
-                                         const uint4 *cst, const uint32_t *wms, int c0, int nc, int kend, int nch, int sc,
-                                         int lane) {
+__device__ __forceinline__ void slot_dot(float (&acc)[kRU], const uint8_t *sl, const uint8_t *limbs, const uint4 *cst,
+                                         const uint32_t *wms, int c0, int nc, int kend, int lane) {
     const uint4 *ql = reinterpret_cast<const uint4 *>(sl) + lane;
     const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kRU * kSlotQ);
     const uint16_t *sc16 = sc0 + (lane >> 1);
@@ -346,10 +352,6 @@ __device__ __forceinline__ void slot_dot(float (&acc)[kRU], float *tot, const ui
                 const float d = wide_dot(xj, word, lane, s, b);
                 if (lane == l) acc[r] += d;
             }
-        }
-        if (slice_end(c, sc, nch)) {
-#pragma unroll
-            for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot + r, c, sc, lane);
         }
     }
 }
@@ -480,15 +482,21 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
             failed = failed || !ok;
             const uint8_t *sl = ring + slot * kSlotBytes;
             if (j + 1 < nsl)
-                slot_dot<kRU>(acc, tot, sl, limbs, csts, wms, j * (kKS / kChunk), kKS / kChunk, kKS, nch, sc, lane);
+                slot_dot<kRU>(acc, sl, limbs, csts, wms, j * (kKS / kChunk), kKS / kChunk, kKS, lane);
             else
-                slot_dot<kRU>(acc, tot, sl, limbs, csts, wms, j * (kKS / kChunk), nc_last, len_last, nch, sc, lane);
+                slot_dot<kRU>(acc, sl, limbs, csts, wms, j * (kKS / kChunk), nc_last, len_last, lane);
             if (++slot == kStages) {
                 slot = 0;
                 par ^= 1u;
             }
             __syncwarp();
             if (issued < steps && !failed) issue_next();
+            // slices end at slot ends (slots of 2 chunks, slices of 4 or the whole K)
+            const int c_last = min(j * (kKS / kChunk) + kKS / kChunk, nch) - 1;
+            if (slice_end(c_last, sc, nch)) {
+#pragma unroll
+                for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot + r, c_last, sc, lane);
+            }
         }
         if (lane == 0) {
             if (a.glu) {
@@ -826,18 +834,23 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     }
                 }
             }
-            if (slice_end(c, sc, nch)) {
-#pragma unroll
-                for (int r = 0; r < kWR; ++r)
-#pragma unroll
-                    for (int m = 0; m < kM; ++m) slice_fold(acc[r][m], tot + r * kM + m, c, sc, lane);
-            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty0 + 8 * slot);
         if (++slot == S) {
             slot = 0;
             par ^= 1u;
+        }
+        // a slice ends only at the end of a slot (slices of 4 chunks, slots of 1, 2
+        // or 4), so its tree sum waits until the slot is back with the producer
+        {
+            const int c_last = min(h.y * kCps + kCps, nch) - 1;
+            if (slice_end(c_last, sc, nch)) {
+#pragma unroll
+                for (int r = 0; r < kWR; ++r)
+#pragma unroll
+                    for (int m = 0; m < kM; ++m) slice_fold(acc[r][m], tot + r * kM + m, c_last, sc, lane);
+            }
         }
         if (h.y == nsl - 1) {
             if (lane == 0) {
