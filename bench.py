@@ -395,7 +395,8 @@ KERNELS = {   # name: (rows, K, segments, epilogue)
 }
 
 
-ADJACENT = ("residual_add", "embed_rows", "lm_head8_half")
+ADJACENT = ("residual_add", "embed_rows", "lm_head8_half", "gather_act", "argmax_half", "head_half_fused", "pick",
+            "top2_half")
 
 
 def run_adjacent(args):
@@ -418,11 +419,52 @@ def run_adjacent(args):
         x = torch.randn(M, H, device="cuda", generator=g).to(torch.bfloat16)
         y = torch.empty(M, rows, dtype=torch.bfloat16, device="cuda")
         call, nbytes = (lambda: tf.tf_qmm8_rows(x, q8, sc, [(0, rows)], y)), rows * H + 2 * rows + 2 * M * H + 2 * M * rows
+    elif args.kernel == "gather_act":
+        # the activated frame's two 8,704-wide halves joined into the 17,408-wide frame
+        F = 17408
+        parts = [torch.randn(M, F // 2, device="cuda", generator=g).to(torch.bfloat16) for _ in range(2)]
+        frame = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+        call, nbytes = (lambda: tf.tf_gather_rows(frame, parts, [F // 2] * 2)), 4 * M * F
+    elif args.kernel in ("argmax_half", "top2_half"):
+        # one half of the head's logits, 124,160 wide
+        n = V // 2
+        lg = torch.randn(M, n, device="cuda", generator=g).to(torch.bfloat16)
+        if args.kernel == "argmax_half":
+            w = torch.empty(M, dtype=torch.int64, device="cuda")
+            scr = torch.empty(tf.tf_argmax_scratch_bytes(M, n), dtype=torch.uint8, device="cuda")
+            call = lambda: tf.tf_argmax_rows(lg, n, w, scr)   # noqa: E731
+        else:
+            w = torch.empty(M, 2, dtype=torch.int64, device="cuda")
+            scr = torch.empty(tf.tf_top2_scratch_bytes(M, n), dtype=torch.uint8, device="cuda")
+            call = lambda: tf.tf_top2_rows(lg, n, w, scr)   # noqa: E731
+        nbytes = 2 * M * n + 8 * M
+    elif args.kernel == "head_half_fused":
+        # one half of the lm_head with its argmax word (the qmm and the key kernel)
+        rows = V // 2
+        wq = torch.randint(0, 256, (V, H // 2), dtype=torch.uint8, device="cuda", generator=g)
+        sc = (0.001 + 0.019 * torch.rand(V, H // 64, device="cuda", generator=g)).to(torch.bfloat16)
+        bi = (-8 * sc.float() + 1e-3 * torch.randn(V, H // 64, device="cuda", generator=g)).to(torch.bfloat16)
+        x = torch.randn(M, H, device="cuda", generator=g).to(torch.bfloat16)
+        lg = torch.empty(M, rows, dtype=torch.bfloat16, device="cuda")
+        w = torch.empty(M, dtype=torch.int64, device="cuda")
+        scr = torch.empty(tf.tf_qmm_argmax_scratch_bytes(M, rows), dtype=torch.uint8, device="cuda")
+        call = lambda: tf.tf_qmm_argmax_rows(x, wq, sc, bi, (rows, rows), rows, lg, w, scr)   # noqa: E731
+        nbytes = qmm_bytes(H, rows, M=M)
+    elif args.kernel == "pick":
+        words = torch.randint(0, 2**40, (2, M), dtype=torch.int64, device="cuda", generator=g)
+        ids = torch.empty(M, dtype=torch.int32, device="cuda")
+        call, nbytes = (lambda: tf.tf_pick(words, ids)), 16 * M + 4 * M
     else:
         table = torch.randn(V, H, device="cuda", generator=g).to(torch.bfloat16)
         ids = torch.randint(0, V, (M,), device="cuda", generator=g, dtype=torch.int32)
         out = torch.empty(M, H, dtype=torch.bfloat16, device="cuda")
         call, nbytes = (lambda: tf.tf_embed_rows(table, V, ids, out)), 4 * M * H
+    call()
+    if not args.no_graph:   # one call in a CUDA graph: a replay has no host work per kernel
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            call()
+        call = gr.replay
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.reps)]
     for a, b in ev:
         a.record()

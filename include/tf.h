@@ -30,9 +30,11 @@
  *  - Kernels are launched with programmatic dependent launch: a kernel may
  *    be scheduled while the kernel before it on the stream still runs, and
  *    waits (griddepcontrol.wait) for that kernel to finish before it reads
- *    any of its arguments' arrays or writes any output.  Before that wait it
- *    only asks for weight bytes to be brought into L2, which cannot observe
- *    stale data, so callers see plain stream order.  Setting the environment
+ *    any of its arguments' arrays or writes any output, with one exception:
+ *    a qmm kernel may read weights (codes, scales, biases) before that wait.
+ *    The library never writes weights, and a kernel of the caller's lets the
+ *    next kernel start only once it has ended, so weights it wrote are in
+ *    place; callers see plain stream order.  Setting the environment
  *    variable TF_PDL=0 before the first call launches without it.
  *  - Outputs must not overlap inputs.
  */

@@ -179,93 +179,106 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
     // preparation is short next to the first ring fill.
     const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
     uint8_t *wm8 = reinterpret_cast<uint8_t *>(wmask);   // byte j of chunk c: lane-chunks 8j .. 8j + 7
-    for (int u = warp * 32 + lane; u < nch * 128; u += W * 32) {
-        const int lc = u >> 2, w = u & 3, c = lc >> 5, l = lc & 31;
-        const int k0 = c * kChunk + l * 32 + w * 8;
-        uint32_t hv[4];   // values 8w .. 8w + 7 of the lane-chunk, two per word (zero past K)
-        if (x16 && k0 + 8 <= K) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(x + k0);
-            hv[0] = v.x;
-            hv[1] = v.y;
-            hv[2] = v.z;
-            hv[3] = v.w;
-        } else {
+    const int nu = nch * 128, stride = W * 32;
+    // a thread's units in batches of four, each batch's loads issued together
+    for (int ub = warp * 32 + lane; ub < nu; ub += 4 * stride) {
+        uint32_t xb[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t lo = k0 + 2 * i < K ? x[k0 + 2 * i] : 0u;
-                const uint32_t hi = k0 + 2 * i + 1 < K ? x[k0 + 2 * i + 1] : 0u;
-                hv[i] = lo | (hi << 16);
-            }
-        }
-        int emax = 0, bad = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-            const int ef = (int)((h >> 7) & 0xFFu);
-            bad |= ef == 0xFF ? 1 : 0;
-            if ((h & 0x7FFFu) != 0) emax = max(emax, max(ef, 1));   // M != 0; a subnormal reads e = 1
-        }
-        emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 1));
-        emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 2));
-        uint32_t L[6] = {0u, 0u, 0u, 0u, 0u, 0u};   // word w of limb vector 2 limb + parity
-        int cnt = 0, sf = 0;   // cnt: nonzero x within 2^4 of the largest (bits 0..7), smaller ones (8..15), bad (16..)
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-            const int ef = (int)((h >> 7) & 0xFFu);
-            const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
-            const int sh = max(ef, 1) - emax + 15;
-            if (M != 0) cnt += sh >= 12 ? 1 : 256;
-            int F;
-            if (sh >= 0) {
-                F = M << sh;
-            } else if (sh > -9) {
-                const int d = -sh;
-                F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
+        for (int b = 0; b < 4; ++b) {
+            const int u = ub + b * stride;
+            const int lc = u >> 2, w = u & 3, c = lc >> 5, l = lc & 31;
+            const int k0 = c * kChunk + l * 32 + w * 8;
+            if (u < nu && x16 && k0 + 8 <= K) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(x + k0);
+                xb[b][0] = v.x;
+                xb[b][1] = v.y;
+                xb[b][2] = v.z;
+                xb[b][3] = v.w;
             } else {
-                F = 0;
-            }
-            if (h & 0x8000u) F = -F;
-            sf += F;
-            // value 8w + t: byte t >> 1 of word w of limb vectors 2 limb + (t & 1)
-            const int p = t & 1, sft = 8 * (t >> 1);
-            L[0 + p] |= (uint32_t)(F & 0xFF) << sft;
-            L[2 + p] |= (uint32_t)((F >> 8) & 0xFF) << sft;
-            L[4 + p] |= (uint32_t)((F >> 16) & 0xFF) << sft;
-        }
-        cnt += bad << 16;
-        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 1);
-        cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 2);
-        sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 1);
-        sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 2);
-        const bool any_bad = (cnt >> 16) != 0;
-        const bool fallback = !any_bad && (cnt & 0xFF) <= 2 && ((cnt >> 8) & 0xFF) > 0;
-        uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
-        if (fallback) {
-            dst[w * 32] = make_uint4(hv[0], hv[1], hv[2], hv[3]);   // values 8w .. 8w + 7 in vector w
-        } else {
 #pragma unroll
-            for (int q = 0; q < 6; ++q) reinterpret_cast<uint32_t *>(dst + q * 32)[w] = L[q];
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t lo = u < nu && k0 + 2 * i < K ? x[k0 + 2 * i] : 0u;
+                    const uint32_t hi = u < nu && k0 + 2 * i + 1 < K ? x[k0 + 2 * i + 1] : 0u;
+                    xb[b][i] = lo | (hi << 16);
+                }
+            }
         }
-        if (w == 0) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int u = ub + b * stride;
+            if (u >= nu) break;   // warp-uniform: nu is a multiple of 32
+            const int lc = u >> 2, w = u & 3, c = lc >> 5, l = lc & 31;
+            const uint32_t *hv = xb[b];   // values 8w .. 8w + 7 of the lane-chunk, two per word (zero past K)
+            int emax = 0, bad = 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
+                const int ef = (int)((h >> 7) & 0xFFu);
+                bad |= ef == 0xFF ? 1 : 0;
+                if ((h & 0x7FFFu) != 0) emax = max(emax, max(ef, 1));   // M != 0; a subnormal reads e = 1
+            }
+            emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 1));
+            emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 2));
+            uint32_t L[6] = {0u, 0u, 0u, 0u, 0u, 0u};   // word w of limb vector 2 limb + parity
+            int cnt = 0, sf = 0;   // cnt: nonzero x within 2^4 of the largest (bits 0..7), smaller ones (8..15), bad (16..)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
+                const int ef = (int)((h >> 7) & 0xFFu);
+                const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
+                const int sh = max(ef, 1) - emax + 15;
+                if (M != 0) cnt += sh >= 12 ? 1 : 256;
+                int F;
+                if (sh >= 0) {
+                    F = M << sh;
+                } else if (sh > -9) {
+                    const int d = -sh;
+                    F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
+                } else {
+                    F = 0;
+                }
+                if (h & 0x8000u) F = -F;
+                sf += F;
+                // value 8w + t: byte t >> 1 of word w of limb vectors 2 limb + (t & 1)
+                const int p = t & 1, sft = 8 * (t >> 1);
+                L[0 + p] |= (uint32_t)(F & 0xFF) << sft;
+                L[2 + p] |= (uint32_t)((F >> 8) & 0xFF) << sft;
+                L[4 + p] |= (uint32_t)((F >> 16) & 0xFF) << sft;
+            }
+            cnt += bad << 16;
+            cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 1);
+            cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 2);
+            sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 1);
+            sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 2);
+            const bool any_bad = (cnt >> 16) != 0;
+            const bool fallback = !any_bad && (cnt & 0xFF) <= 2 && ((cnt >> 8) & 0xFF) > 0;
+            uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
             if (fallback) {
-                cst[lc] = make_uint4(0u, 0u, 0u, 0u);
+                dst[w * 32] = make_uint4(hv[0], hv[1], hv[2], hv[3]);   // values 8w .. 8w + 7 in vector w
             } else {
-                // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
-                const float scale = any_bad ? __int_as_float(0x7FC00000)
-                                            : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
-                const int sfv = any_bad ? 0 : sf;
-                cst[lc] = make_uint4(__float_as_uint(scale), __float_as_uint(__int2float_rn(sfv) * scale),
-                                     (uint32_t)sfv << 3, 0u);
-            }
-        }
-        // the warp's 32 threads hold 8 lane-chunks of chunk c (l of lane 0 a multiple of 8)
-        const uint32_t b = __ballot_sync(0xFFFFFFFFu, fallback && w == 0);
-        if (lane == 0) {
-            uint32_t m8 = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) m8 |= ((b >> (4 * j)) & 1u) << j;
-            wm8[c * 4 + (l >> 3)] = (uint8_t)m8;
+                for (int q = 0; q < 6; ++q) reinterpret_cast<uint32_t *>(dst + q * 32)[w] = L[q];
+            }
+            if (w == 0) {
+                if (fallback) {
+                    cst[lc] = make_uint4(0u, 0u, 0u, 0u);
+                } else {
+                    // 2^(E-23) = 2^(emax-149); normal for emax >= 23, the exact subnormal below
+                    const float scale = any_bad ? __int_as_float(0x7FC00000)
+                                                : (emax >= 23 ? __int_as_float((emax - 22) << 23) : ldexpf(1.0f, emax - 149));
+                    const int sfv = any_bad ? 0 : sf;
+                    cst[lc] = make_uint4(__float_as_uint(scale), __float_as_uint(__int2float_rn(sfv) * scale),
+                                         (uint32_t)sfv << 3, 0u);
+                }
+            }
+            // the warp's 32 threads hold 8 lane-chunks of chunk c (l of lane 0 a multiple of 8)
+            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, fallback && w == 0);
+            if (lane == 0) {
+                uint32_t m8 = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) m8 |= ((bal >> (4 * j)) & 1u) << j;
+                wm8[c * 4 + (l >> 3)] = (uint8_t)m8;
+            }
         }
     }
 }
@@ -357,7 +370,8 @@ __device__ __forceinline__ void slot_dot(float (&acc)[kRU], const uint8_t *sl, c
 }
 
 // ------------------------------------------------------------------ kernel --
-template <int kRU>
+// kOne: the whole K is one slice, folded once after the unit's last slot.
+template <int kRU, bool kOne>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArgs a, int units) {
     constexpr int kSlotBytes = slot_bytes(kRU);
     constexpr int kStages = stages_for(kRU);
@@ -492,11 +506,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) qmm_m1_stream_kernel(QmmArg
             __syncwarp();
             if (issued < steps && !failed) issue_next();
             // slices end at slot ends (slots of 2 chunks, slices of 4 or the whole K)
-            const int c_last = min(j * (kKS / kChunk) + kKS / kChunk, nch) - 1;
-            if (slice_end(c_last, sc, nch)) {
+            if (!kOne) {
+                const int c_last = min(j * (kKS / kChunk) + kKS / kChunk, nch) - 1;
+                if (slice_end(c_last, sc, nch)) {
 #pragma unroll
-                for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot + r, c_last, sc, lane);
+                    for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot + r, c_last, sc, lane);
+                }
             }
+        }
+        if (kOne) {
+#pragma unroll
+            for (int r = 0; r < kRU; ++r) slice_fold(acc[r], tot + r, nch - 1, sc, lane);
         }
         if (lane == 0) {
             if (a.glu) {
@@ -609,7 +629,9 @@ __device__ __forceinline__ int tile_row(int w, int r) {
     return kGlu ? (r & 1) * (2 * kWR) + (kWR / 2) * w + (r >> 1) : kWR * w + r;
 }
 
-template <bool kGlu, int kWR, int kM>
+// kOne: the whole K is one slice (at most 8 chunks), so the slice's tree sum is
+// the tile's last step and needs no per-slot test.
+template <bool kGlu, int kWR, int kM, bool kOne>
 __global__ void __launch_bounds__(kTThreads, 1)
     qmm_m1_tile_kernel(QmmArgs a, TilePlan plan, const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap bmap, int S) {
@@ -722,32 +744,16 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
     };
 
-    // While the kernel before this one may still run, each producer asks for the
-    // first ring's worth of one of the CTA's first four tiles (the four the groups
-    // claim first) to be brought into L2; weights are never written by a kernel
-    // of the library, and an L2 prefetch cannot see stale data in any case.
-    if (producer && lane == 0 && t0 + grp < t1) {
-        int r_a, r_b, col, ncol;
-        tile_rows(t0 + grp, r_a, r_b, col, ncol);
-        for (int c = 0; c < S && c < nsl; ++c) {
-            const int cq = c * (Sh::q / Sh::qelem), cs = c * (Sh::sb / 2);
-            l2_prefetch_2d(&qmap, cq, r_a);
-            l2_prefetch_2d(&smap, cs, r_a);
-            l2_prefetch_2d(&bmap, cs, r_a);
-            if (kGlu) {
-                l2_prefetch_2d(&qmap, cq, r_b);
-                l2_prefetch_2d(&smap, cs, r_b);
-                l2_prefetch_2d(&bmap, cs, r_b);
-            }
-        }
-    }
-    pdl_wait();
-    pdl_trigger();
-    // the whole ring goes out before the limb preparation (one tile-chunk a slot);
-    // all warps prepare the limbs, then the producers keep the rings full
+    // The whole ring goes out first (one tile-chunk a slot), before the wait for
+    // the kernel this one may overlap: the weights are never written by a kernel
+    // of the library, and a kernel from elsewhere does not release this one
+    // before it ends.  Then all warps prepare the limbs, and the producers keep
+    // the rings full.
     if (producer && lane == 0)
         for (int i = 0; i < S; ++i) issue_next();
     __syncwarp();
+    pdl_wait();
+    pdl_trigger();
     const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
 #pragma unroll
     for (int m = 0; m < kM; ++m)
@@ -768,6 +774,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         for (int m = 0; m < kM; ++m) acc[r][m] = 0.0f;
     float *tot = reinterpret_cast<float *>(smem + L.tot_off) + (producer ? 0 : warp * 8);   // lane 0's, [r][m]
     const int sc = slice_chunks(nch);
+    (void)sc;
     uint64_t best = 0;
     int slot = 0;
     uint32_t par = 0;
@@ -843,7 +850,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         // a slice ends only at the end of a slot (slices of 4 chunks, slots of 1, 2
         // or 4), so its tree sum waits until the slot is back with the producer
-        {
+        if (!kOne) {
             const int c_last = min(h.y * kCps + kCps, nch) - 1;
             if (slice_end(c_last, sc, nch)) {
 #pragma unroll
@@ -853,6 +860,20 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
         }
         if (h.y == nsl - 1) {
+            if (kOne) {   // the single slice's fold, as slice_fold does it
+                float tr[kWR * kM];
+#pragma unroll
+                for (int r = 0; r < kWR; ++r)
+#pragma unroll
+                    for (int m = 0; m < kM; ++m) {
+                        tr[r * kM + m] = warp_sum_to_lane0(acc[r][m]);
+                        acc[r][m] = 0.0f;
+                    }
+                if (lane == 0) {
+#pragma unroll
+                    for (int i = 0; i < kWR * kM; ++i) tot[i] = tr[i];
+                }
+            }
             if (lane == 0) {
                 int r_a, r_b, col, ncol;
                 tile_rows(h.x, r_a, r_b, col, ncol);
@@ -1113,7 +1134,9 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream, int 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     if (g_stream_smem_set[dev][ri] < L.total) {
-        cudaError_t e = cudaFuncSetAttribute(qmm_m1_stream_kernel<RU>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+        cudaError_t e = cudaFuncSetAttribute(qmm_m1_stream_kernel<RU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(qmm_m1_stream_kernel<RU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
         if (e != cudaSuccess) return e;
         g_stream_smem_set[dev][ri] = 226 * 1024;
     }
@@ -1123,7 +1146,9 @@ static cudaError_t launch_ru(const QmmArgs &a, int ri, cudaStream_t stream, int 
     const int need = (units + W - 1) / W;
     if (need < blocks) blocks = need;
     if (ncand) *ncand = blocks * W;
-    return launch_pdl(qmm_m1_stream_kernel<RU>, dim3(blocks), dim3(W * 32), L.total, stream, a, units);
+    if (slice_chunks(L.nch) == L.nch)
+        return launch_pdl(qmm_m1_stream_kernel<RU, true>, dim3(blocks), dim3(W * 32), L.total, stream, a, units);
+    return launch_pdl(qmm_m1_stream_kernel<RU, false>, dim3(blocks), dim3(W * 32), L.total, stream, a, units);
 }
 
 // ---------------------------------------------------------- tile ring host --
@@ -1202,13 +1227,19 @@ static cudaError_t launch_tile(const QmmArgs &a, cudaStream_t stream, int *ncand
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     if (!smem_set[dev]) {
         cudaError_t e =
-            cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu, kWR, kM>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+            cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu, kWR, kM, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 226 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(qmm_m1_tile_kernel<kGlu, kWR, kM, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     226 * 1024);
         if (e != cudaSuccess) return e;
         smem_set[dev] = true;
     }
     const int blocks = plan.ntiles < num_sms() ? plan.ntiles : num_sms();
     if (ncand) *ncand = blocks * (kTWarps + kTGroups);
-    return launch_pdl(qmm_m1_tile_kernel<kGlu, kWR, kM>, dim3(blocks), dim3(kTThreads), L.total, stream, a, plan, qmap,
+    if (slice_chunks(L.nch) == L.nch)
+        return launch_pdl(qmm_m1_tile_kernel<kGlu, kWR, kM, true>, dim3(blocks), dim3(kTThreads), L.total, stream, a, plan,
+                          qmap, smap, bmap, S);
+    return launch_pdl(qmm_m1_tile_kernel<kGlu, kWR, kM, false>, dim3(blocks), dim3(kTThreads), L.total, stream, a, plan, qmap,
                       smap, bmap, S);
 }
 

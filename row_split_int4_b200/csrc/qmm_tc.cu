@@ -19,10 +19,10 @@
 // straddles two segments; with TF_EPI_GLU its rows 0-63 are gate rows and
 // 64-127 the up rows of the same outputs.  Two CTAs per SM for N <= 32 (each
 // with half of tensor memory), one CTA per SM above; 10 to 22 warps:
-//   * warp 0, one thread: per group one TMA copy of the activation tile
-//     [N x 64] (128-byte swizzle) and two of the tile's packed codes
-//     [2 x 64 rows x 32 B] into a ring of 8 to 16 slots in shared memory.  No
-//     multicast.
+//   * warp 0, three threads: per four groups one TMA copy of the activation
+//     tiles [4 x N x 64] and two of the tile's packed codes [2 x 64 rows x
+//     128 B] (both with the 128-byte swizzle) into a ring of 2 to 4 slots in
+//     shared memory, each copy from a lane of its own.  No multicast.
 //   * 4 or 8 decoder warps, one thread per weight row (= tensor-memory lane):
 //     the row's codes -> bf16 pairs, stored into an A stage in tensor memory
 //     (tcgen05.st), software-pipelined so that a store drains while the next
@@ -61,25 +61,31 @@ namespace tf {
 constexpr int kTcRows = 128;                    // weight rows per tile (MMA M)
 constexpr int kTcK = 64;                        // K per group / pipeline stage
 constexpr int kTcXbSlots = 8;                   // X_g slots in shared memory
+constexpr int kTcGps = 4;                       // groups per ring slot
 // Per MMA N: CTAs per SM (two for N <= 32, each with half of tensor memory),
-// decoder and scale warps, and pipeline depths.  Ring slot: the activation tile
-// (N x 128 B) and the codes (4 KB).  Tensor memory: tc_dbufs(N) D buffers of N
-// columns from column 0, tc_astages(N) A stages of 32 columns at the top.
+// decoder and scale warps, and pipeline depths.  Ring slot: four groups, the
+// activation tiles [4][N][128 B] and the codes [128 rows][128 B], both with the
+// 128-byte swizzle.  The roles hand work on in steps of tc_bg(N) groups (one
+// barrier wait and one release per step: for small N a barrier round costs
+// about as much as a group's work).  Tensor memory: tc_dbufs(N) D stages of
+// tc_bg(N) x N columns from column 0, tc_astages(N) A stages of tc_bg(N) x 32
+// columns at the top.
 __host__ __device__ constexpr int tc_ctas_per_sm(int n) { return n <= 32 ? 2 : 1; }
 __host__ __device__ constexpr uint32_t tc_tmem_cols(int n) { return n <= 32 ? 256u : 512u; }
 __host__ __device__ constexpr int tc_dec_warps(int n) { return n == 64 ? 8 : 4; }
 // Scale warps: per tensor-memory lane quarter one warp per 32 activation rows.
 __host__ __device__ constexpr int tc_scale_warps(int n) { return 4 * (n < 32 ? 1 : n / 32); }
 __host__ __device__ constexpr int tc_threads(int n) { return 32 * (2 + tc_dec_warps(n) + tc_scale_warps(n)); }
-__host__ __device__ constexpr int tc_slot_bytes(int n) { return n * kTcK * 2 + kTcRows * kTcK / 2; }
-__host__ __device__ constexpr int tc_ring(int n) { return n == 16 ? 16 : (n == 32 ? 12 : (n == 64 ? 12 : 8)); }
-__host__ __device__ constexpr int tc_astages(int n) { return n == 64 ? 8 : 4; }
-__host__ __device__ constexpr int tc_dbufs(int n) {
-    return (int)(tc_tmem_cols(n) - 32 * tc_astages(n)) / n < 8 ? (int)(tc_tmem_cols(n) - 32 * tc_astages(n)) / n : 8;
+__host__ __device__ constexpr int tc_slot_bytes(int n) { return kTcGps * (n * kTcK * 2 + kTcRows * kTcK / 2); }
+__host__ __device__ constexpr int tc_ring(int n) { return n == 16 ? 4 : (n == 32 ? 3 : (n == 64 ? 4 : 2)); }
+__host__ __device__ constexpr int tc_bg(int n) { return n <= 32 ? 2 : 1; }
+__host__ __device__ constexpr int tc_astages(int n) { return n <= 32 ? 2 : (n == 64 ? 8 : 4); }
+__host__ __device__ constexpr int tc_dfit(int n) {
+    return (int)(tc_tmem_cols(n) - 32 * tc_bg(n) * tc_astages(n)) / (tc_bg(n) * n);
 }
+__host__ __device__ constexpr int tc_dbufs(int n) { return tc_dfit(n) < 8 ? tc_dfit(n) : 8; }
 constexpr int kTcMaxN = 128;                    // activation rows per call
 constexpr int kTcMaxSplit = 8;                  // CTAs per cluster
-constexpr int kTcCBytes = kTcRows * kTcK / 2;   // 4 KB of codes per group
 constexpr int kTcXbBytes = kTcXbSlots * kTcMaxN * 4;
 constexpr int kTcBarBytes = 1024;               // mbarriers, TMEM address, failure flag
 __host__ __device__ constexpr int tc_num_bars(int n) {
@@ -98,7 +104,9 @@ struct TcChecks {
     static_assert(tc_slot_bytes(N) % 1024 == 0, "ring slots keep the 1 KB alignment of the swizzled tile");
     static_assert(N * kTcRows * 4 <= tc_ring(N) * tc_slot_bytes(N), "partial sums must fit in the ring");
     static_assert(tc_num_bars(N) * 8 + 8 <= kTcBarBytes, "barrier area");
-    static_assert(tc_dbufs(N) >= 2 && tc_dbufs(N) * N + 32 * tc_astages(N) <= (int)tc_tmem_cols(N), "tensor memory map");
+    static_assert(tc_dbufs(N) >= 2 && tc_bg(N) * (tc_dbufs(N) * N + 32 * tc_astages(N)) <= (int)tc_tmem_cols(N),
+                  "tensor memory map");
+    static_assert(kTcGps % tc_bg(N) == 0 && kTcXbSlots % tc_bg(N) == 0 && 8 % tc_bg(N) == 0, "steps of whole groups");
     static_assert(tc_smem_bytes(N) <= 227 * 1024, "shared memory");
     static_assert(tc_ctas_per_sm(N) == 1 || (tc_smem_bytes(N) + 1024) * 3 > 228 * 1024, "at most two CTAs per SM");
     static_assert(tc_ctas_per_sm(N) == 2 || (tc_smem_bytes(N) + 1024) * 2 > 228 * 1024, "one CTA per SM");
@@ -140,6 +148,11 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
 __device__ __forceinline__ void tc_tma_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
     asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
                  "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_tma_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
                  : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -303,15 +316,16 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     constexpr int NT = N / (SW / 4);          // activation rows per scale thread (16 or 32)
     constexpr int CH = 16;                    // columns per tcgen05.ld
     constexpr int R = tc_ring(N), NA = tc_astages(N), ND = tc_dbufs(N);
-    constexpr int SLOT = tc_slot_bytes(N), XBYTES = N * kTcK * 2, RING = R * SLOT;
+    constexpr int SLOT = tc_slot_bytes(N), XG = N * kTcK * 2, XBYTES = kTcGps * XG, RING = R * SLOT;
     constexpr uint32_t TCOLS = tc_tmem_cols(N);
-    constexpr uint32_t ACOL = TCOLS - 32 * NA;        // first A-stage column
+    constexpr int BG = tc_bg(N), XS = kTcXbSlots / BG;   // groups per step; X_g slots of a step's size
+    constexpr uint32_t ACOL = TCOLS - 32 * BG * NA;   // first A-stage column
     constexpr int DW = tc_dec_warps(N);               // decoder warps
     constexpr int VW = 32 * 4 / DW;                   // bf16 pairs per decoder thread and group: 32 or 16
     (void)sizeof(TcChecks<N>);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *ring = smem;                                               // [slot][x | codes]
+    uint8_t *ring = smem;                                               // [slot][x: 4 groups | codes]
     float *part = reinterpret_cast<float *>(smem);                      // at the end: [N][128] fp32
     float *xbar = reinterpret_cast<float *>(smem + RING);       // [slot][128] fp32
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + RING + kTcXbBytes);
@@ -400,148 +414,162 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA
-        if (lane == 0) {
+        // Per slot (four groups) three copies, each from a lane of its own:
+        // lane 0 the activation tiles, lanes 1 and 2 the codes of tile rows
+        // 0-63 and 64-127.  A tensor copy holds the thread that issues it for
+        // a fixed time, so copies from three lanes overlap where one lane's
+        // would queue.
+        if (lane < 3) {
             const uint32_t bytes = (uint32_t)SLOT;
+            const int nsl = nst / kTcGps;
             int issued = 0;
-            for (int li = 0; li < nst; ++li) {
-                const int s = li % R;
-                if (li >= R) {
-                    const uint32_t par = ((li / R) - 1) & 1;
-                    if (!tc_wait(xfree(s), par, fail) || !tc_wait(cfree(s), par, fail)) { *fail = 1; break; }
+            for (int j = 0; j < nsl; ++j) {
+                const int s = j % R;
+                bool ok = true;
+                if (j >= R) {
+                    const uint32_t par = ((j / R) - 1) & 1;
+                    ok = tc_wait(xfree(s), par, fail) && tc_wait(cfree(s), par, fail);
                 }
-                if (*fail) break;
-                const int i = i0 + li;
+                if (!__all_sync(0x7u, ok && !*fail)) {
+                    if (lane == 0) *fail = 1;
+                    break;
+                }
+                const int i = i0 + kTcGps * j;
                 const uint32_t slot = tc_smem(ring + s * SLOT);
-                tc_expect_tx(full(s), bytes);
-                tc_tma_2d(slot, &xmap, i * kTcK, 0, full(s));
-                tc_tma_2d(slot + XBYTES, &cmap, i * (kTcK / 2), rowA, full(s));
-                tc_tma_2d(slot + XBYTES + kTcCBytes / 2, &cmap, i * (kTcK / 2), rowB, full(s));
-                issued = li + 1;
+                if (lane == 0) tc_expect_tx(full(s), bytes);
+                __syncwarp(0x7u);
+                if (lane == 0)
+                    tc_tma_3d(slot, &xmap, 0, 0, i, full(s));
+                else
+                    tc_tma_2d(slot + XBYTES + (lane - 1) * (kTcRows / 2) * (kTcGps * kTcK / 2), &cmap,
+                              i * (kTcK / 2), lane == 1 ? rowA : rowB, full(s));
+                issued = j + 1;
             }
             // every copy issued must land before the ring is reused or the CTA exits
-            for (int li = issued - R; li < issued; ++li)
-                if (li >= 0) tc_wait(full(li % R), (li / R) & 1, fail, 1 << 16);
+            if (lane == 0)
+                for (int j = issued - R; j < issued; ++j)
+                    if (j >= 0) tc_wait(full(j % R), (j / R) & 1, fail, 1 << 16);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t idesc = tc_idesc(N);
-            for (int li = 0; li < nst; ++li) {
-                const int s = li % R, sa = li % NA, sd = li % ND;
-                if (!tc_wait(full(s), (li / R) & 1, fail) || !tc_wait(afull(sa), (li / NA) & 1, fail) ||
-                    (li >= ND && !tc_wait(dfree(sd), ((li / ND) - 1) & 1, fail))) {
+            for (int k = 0; k < nst / BG; ++k) {   // steps of BG groups
+                const int sa = k % NA, sd = k % ND;
+                if (!tc_wait(afull(sa), (k / NA) & 1, fail) || (k >= ND && !tc_wait(dfree(sd), ((k / ND) - 1) & 1, fail))) {
                     *fail = 1;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t xb = tc_smem(ring + s * SLOT);
-                const uint32_t dt = tmem + (uint32_t)(N * sd), at = tmem + ACOL + 32u * sa;
+                bool ok = true;
 #pragma unroll
-                for (int kk = 0; kk < kTcK / 16; ++kk) tc_mma_ts(dt, at + 8 * kk, tc_desc(xb + kk * 32), idesc, kk > 0 ? 1u : 0u);
-                tc_commit(xfree(s));
+                for (int g = 0; g < BG; ++g) {
+                    const int li = k * BG + g, j = li / kTcGps, gs = li % kTcGps, s = j % R;
+                    if (gs == 0 && !tc_wait(full(s), (j / R) & 1, fail)) {   // the slot's first group
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t xb = tc_smem(ring + s * SLOT) + (uint32_t)(gs * XG);
+                    const uint32_t dt = tmem + (uint32_t)(BG * N * sd + N * g), at = tmem + ACOL + 32u * (BG * sa + g);
+#pragma unroll
+                    for (int kk = 0; kk < kTcK / 16; ++kk)
+                        tc_mma_ts(dt, at + 8 * kk, tc_desc(xb + kk * 32), idesc, kk > 0 ? 1u : 0u);
+                    if (gs == kTcGps - 1) tc_commit(xfree(s));   // the slot's last group
+                }
+                if (!ok) {
+                    *fail = 1;
+                    break;
+                }
                 tc_commit(aempty(sa));
                 tc_commit(dfull(sd));
             }
         }
     } else if (warp < 2 + DW) {
         // ------------------------------------------- codes -> A stages, and X_g
-        // Software-pipelined: group li is decoded into registers while the
-        // tensor-memory store of group li-1 drains; an A stage is published
-        // (afull) only after tcgen05.wait::st.  With 8 decoder warps each
-        // thread takes half of its row's 64 codes.
+        // Per step: wait for the A stage; per group wait for the slot (at its
+        // first group), turn the row's codes into bf16 pairs and store them into
+        // tensor memory; the stage is published (afull) once, after
+        // tcgen05.wait::st.  With 8 decoder warps each thread takes half of its
+        // row's 64 codes.  The four warps of the first half also form X_g.
         const int q = warp & 3, dh = (warp - 2) >> 2;   // lane quarter; part of the group's codes
         const int t = 32 * q + lane;                    // tile row == TMEM lane; also an activation row
         const uint32_t a_lane = tmem + ((uint32_t)(32 * q) << 16) + ACOL + (uint32_t)(dh * VW);
-        const bool xrole = dh == 0;                     // these four warps also form X_g
-        uint32_t va[VW], vb[VW];
-        bool ok = true;
-        int stored = 0;
-#define TC_PRODUCE(LI, V)                                                                                           \
-    {                                                                                                               \
-        const int s_ = (LI) % R, xs_ = (LI) % kTcXbSlots;                                                           \
-        ok = tc_wait(full(s_), ((LI) / R) & 1, fail);                                                               \
-        if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                         \
-            *fail = 1;                                                                                              \
-            break;                                                                                                  \
-        }                                                                                                           \
-        const uint8_t *slot_ = ring + s_ * SLOT;                                                                    \
-        const uint4 *cp_ = reinterpret_cast<const uint4 *>(slot_ + XBYTES + 32 * t);                                \
-        uint32_t w_[VW / 4];                                                                                        \
-        if (VW == 32) { /* lanes 4-7 of each eight read the second half first: no bank conflict */                 \
-            const int sw_ = (lane >> 2) & 1;                                                                        \
-            const uint4 ca_ = cp_[sw_], cb_ = cp_[sw_ ^ 1];                                                         \
-            const uint4 c0_ = sw_ ? cb_ : ca_, c1_ = sw_ ? ca_ : cb_;                                               \
-            w_[0] = c0_.x; w_[1] = c0_.y; w_[2] = c0_.z; w_[3] = c0_.w;                                             \
-            w_[VW / 4 - 4] = c1_.x; w_[VW / 4 - 3] = c1_.y; w_[VW / 4 - 2] = c1_.z; w_[VW / 4 - 1] = c1_.w;         \
-        } else {                                                                                                    \
-            const uint4 c0_ = cp_[dh];                                                                              \
-            w_[0] = c0_.x; w_[1] = c0_.y; w_[2] = c0_.z; w_[3] = c0_.w;                                             \
-        }                                                                                                           \
-        float xsum_ = 0.0f;                                                                                         \
-        if (xrole && t < N) { /* X_g of activation row t: 64 values, k ascending (8 chunks of 8) */                \
-            const uint8_t *xrow_ = slot_ + t * 128;                                                                 \
-            _Pragma("unroll") for (int c = 0; c < 8; ++c) {                                                         \
-                const uint4 v_ = *reinterpret_cast<const uint4 *>(xrow_ + ((c ^ (t & 7)) << 4));                    \
-                const float cs_ = tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(0.0f, v_.x), v_.y), v_.z), v_.w); \
-                xsum_ = c == 0 ? cs_ : xsum_ + cs_;                                                                 \
-            }                                                                                                       \
-        }                                                                                                           \
-        __syncwarp();                                                                                               \
-        if (lane == 0) tc_arrive(cfree(s_));                                                                        \
-        if (xrole) {                                                                                                \
-            ok = (LI) < kTcXbSlots || tc_wait(xbfree(xs_), (((LI) / kTcXbSlots) - 1) & 1, fail);                    \
-            if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                     \
-                *fail = 1;                                                                                          \
-                break;                                                                                              \
-            }                                                                                                       \
-            if (t < N) xbar[xs_ * kTcMaxN + t] = xsum_;                                                             \
-            __syncwarp();                                                                                           \
-            if (lane == 0) tc_arrive(xbfull(xs_));                                                                  \
-        }                                                                                                           \
-        _Pragma("unroll") for (int c = 0; c < VW / 4; ++c) {                                                        \
-            const uint32_t ws_ = w_[c] >> 4;                                                                        \
-            V[4 * c + 0] = tc_code_pair<0>(w_[c], ws_);                                                             \
-            V[4 * c + 1] = tc_code_pair<1>(w_[c], ws_);                                                             \
-            V[4 * c + 2] = tc_code_pair<2>(w_[c], ws_);                                                             \
-            V[4 * c + 3] = tc_code_pair<3>(w_[c], ws_);                                                             \
-        }                                                                                                           \
-    }
-#define TC_PUBLISH(LI)                                                                                              \
-    {                                                                                                               \
-        tc_wait_st();                                                                                               \
-        tc_fence_before();                                                                                          \
-        __syncwarp();                                                                                               \
-        if (lane == 0) tc_arrive(afull((LI) % NA));                                                                 \
-    }
-#define TC_STORE(LI, V)                                                                                             \
-    {                                                                                                               \
-        const int sa_ = (LI) % NA;                                                                                  \
-        ok = (LI) < NA || tc_wait(aempty(sa_), (((LI) / NA) - 1) & 1, fail);                                        \
-        if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                         \
-            *fail = 1;                                                                                              \
-            break;                                                                                                  \
-        }                                                                                                           \
-        tc_fence_after();                                                                                           \
-        tc_st<VW>(a_lane + 32u * sa_, V);                                                                           \
-        stored = (LI) + 1;                                                                                          \
-    }
-        for (int li = 0; li < nst; li += 2) {   // nst is a multiple of 8
-            TC_PRODUCE(li, va)
-            if (li > 0) TC_PUBLISH(li - 1)
-            TC_STORE(li, va)
-            TC_PRODUCE(li + 1, vb)
-            TC_PUBLISH(li)
-            TC_STORE(li + 1, vb)
-        }
-        if (stored == nst && nst > 0) {
-            tc_wait_st();
+        const bool xrole = dh == 0;
+        uint32_t v[VW];
+        for (int k = 0; k < nst / BG; ++k) {
+            const int sa = k % NA, xs = k % XS;
+            bool ok = k < NA || tc_wait(aempty(sa), ((k / NA) - 1) & 1, fail);
+            if (__any_sync(0xFFFFFFFFu, !ok)) {
+                *fail = 1;
+                break;
+            }
+            tc_fence_after();
+            float xsum[BG];
+#pragma unroll
+            for (int g = 0; g < BG; ++g) {
+                const int li = k * BG + g, j = li / kTcGps, gs = li % kTcGps, s = j % R;
+                if (gs == 0) {
+                    ok = tc_wait(full(s), (j / R) & 1, fail);
+                    if (__any_sync(0xFFFFFFFFu, !ok)) break;
+                }
+                const uint8_t *slot = ring + s * SLOT;
+                // row t's 128 bytes of codes, 16-byte chunk c at position c ^ (t & 7)
+                // (the copy's swizzle); group gs is chunks 2 gs and 2 gs + 1, so eight
+                // neighbouring rows read eight distinct bank quads
+                const uint4 *cp = reinterpret_cast<const uint4 *>(slot + XBYTES + 128 * t);
+                uint32_t w[VW / 4];
+                if (VW == 32) {
+                    const uint4 c0 = cp[(2 * gs) ^ (t & 7)], c1 = cp[(2 * gs + 1) ^ (t & 7)];
+                    w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
+                    w[VW / 4 - 4] = c1.x; w[VW / 4 - 3] = c1.y; w[VW / 4 - 2] = c1.z; w[VW / 4 - 1] = c1.w;
+                } else {
+                    const uint4 c0 = cp[(2 * gs + dh) ^ (t & 7)];
+                    w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
+                }
+                xsum[g] = 0.0f;
+                if (xrole && t < N) {   // X_g of activation row t: 64 values, k ascending (8 chunks of 8)
+                    const uint8_t *xrow = slot + gs * XG + t * 128;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 xv = *reinterpret_cast<const uint4 *>(xrow + ((c ^ (t & 7)) << 4));
+                        const float cs = tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(0.0f, xv.x), xv.y), xv.z), xv.w);
+                        xsum[g] = c == 0 ? cs : xsum[g] + cs;
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < VW / 4; ++c) {
+                    const uint32_t ws = w[c] >> 4;
+                    v[4 * c + 0] = tc_code_pair<0>(w[c], ws);
+                    v[4 * c + 1] = tc_code_pair<1>(w[c], ws);
+                    v[4 * c + 2] = tc_code_pair<2>(w[c], ws);
+                    v[4 * c + 3] = tc_code_pair<3>(w[c], ws);
+                }
+                __syncwarp();
+                if (lane == 0 && gs == kTcGps - 1) tc_arrive(cfree(s));   // the slot's codes are read
+                tc_st<VW>(a_lane + 32u * (uint32_t)(BG * sa + g), v);
+                tc_wait_st();
+            }
+            if (__any_sync(0xFFFFFFFFu, !ok)) {
+                *fail = 1;
+                break;
+            }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) tc_arrive(afull((nst - 1) % NA));
+            if (lane == 0) tc_arrive(afull(sa));
+            if (xrole) {
+                ok = k < XS || tc_wait(xbfree(xs), ((k / XS) - 1) & 1, fail);
+                if (__any_sync(0xFFFFFFFFu, !ok)) {
+                    *fail = 1;
+                    break;
+                }
+                if (t < N) {
+#pragma unroll
+                    for (int g = 0; g < BG; ++g) xbar[(xs * BG + g) * kTcMaxN + t] = xsum[g];
+                }
+                __syncwarp();
+                if (lane == 0) tc_arrive(xbfull(xs));
+            }
         }
-#undef TC_PRODUCE
-#undef TC_PUBLISH
-#undef TC_STORE
     } else {
         // ------------------------------------------------ y += s D_g + b X_g
         const int q = warp & 3, h = (warp - 2 - DW) >> 2;   // lane quarter, block of NT rows
@@ -567,21 +595,25 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
                 sn = __ldg(reinterpret_cast<const uint4 *>(srow + 8 * (p + 1)));
                 bn = __ldg(reinterpret_cast<const uint4 *>(brow + 8 * (p + 1)));
             }
+// Group J (0..7) of the period; the step's barriers are waited for at its
+// first group and released after its last.
 #define TC_GROUP(J)                                                                                                 \
     {                                                                                                               \
-        const int sd = li % ND, xs = li % kTcXbSlots;                                                         \
-        const bool ok = tc_wait(dfull(sd), (li / ND) & 1, fail) && tc_wait(xbfull(xs), (li / kTcXbSlots) & 1, fail); \
-        if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                         \
-            *fail = 1;                                                                                              \
-            break;                                                                                                  \
+        const int k = li / BG, sd = k % ND, xs = k % XS, g = (J) % BG;                                              \
+        if (g == 0) {                                                                                               \
+            const bool ok = tc_wait(dfull(sd), (k / ND) & 1, fail) && tc_wait(xbfull(xs), (k / XS) & 1, fail);     \
+            if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                     \
+                *fail = 1;                                                                                          \
+                break;                                                                                              \
+            }                                                                                                       \
+            tc_fence_after();                                                                                       \
         }                                                                                                           \
-        tc_fence_after();                                                                                           \
         /* D holds sum (q - 8) x: y += s D + (b + 8 s) X */                                                       \
         const float sf = tc_pick_bf16<J>(s8), bf = fmaf(8.0f, sf, tc_pick_bf16<J>(b8));                             \
-        const float *xg = xb_h + xs * kTcMaxN;                                                                      \
+        const float *xg = xb_h + (xs * BG + g) * kTcMaxN;                                                           \
         _Pragma("unroll") for (int c = 0; c < NT; c += CH) {                                                        \
             uint32_t d[CH];                                                                                         \
-            tc_ld<CH>(d_lane + (uint32_t)(N * sd) + c, d);                                                                   \
+            tc_ld<CH>(d_lane + (uint32_t)(BG * N * sd + N * g) + c, d);                                             \
             tc_wait_ld();                                                                                           \
             _Pragma("unroll") for (int j = 0; j < CH; j += 4) {                                                     \
                 const float4 xv = *reinterpret_cast<const float4 *>(xg + c + j);                                    \
@@ -591,11 +623,13 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
                          bf, xv.z, xv.w);                                                                           \
             }                                                                                                       \
         }                                                                                                           \
-        tc_fence_before();                                                                                          \
-        __syncwarp();                                                                                               \
-        if (lane == 0) {                                                                                            \
-            tc_arrive(dfree(sd));                                                                                   \
-            tc_arrive(xbfree(xs));                                                                                  \
+        if (g == BG - 1) {                                                                                          \
+            tc_fence_before();                                                                                      \
+            __syncwarp();                                                                                           \
+            if (lane == 0) {                                                                                        \
+                tc_arrive(dfree(sd));                                                                               \
+                tc_arrive(xbfree(xs));                                                                              \
+            }                                                                                                       \
         }                                                                                                           \
         ++li;                                                                                                       \
     }
@@ -748,11 +782,13 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
 
     CUtensorMap xmap, cmap;
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)a.M};
-        const cuuint64_t strides[1] = {(cuuint64_t)a.ldx * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)n_mma};
-        const cuuint32_t estr[2] = {1, 1};
-        if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(a.x), dims, strides, box, estr,
+        // [group][row][64 values]: four groups' activation tiles in one copy,
+        // each tile the MMA's B operand as it stands (rows past M read as zero)
+        const cuuint64_t dims[3] = {(cuuint64_t)kTcK, (cuuint64_t)a.M, (cuuint64_t)(a.K / kTcK)};
+        const cuuint64_t strides[2] = {(cuuint64_t)a.ldx * 2, (cuuint64_t)kTcK * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)kTcK, (cuuint32_t)n_mma, (cuuint32_t)kTcGps};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(a.x), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -760,10 +796,10 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
     {
         const cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.n_whole};
         const cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
-        const cuuint32_t box[2] = {(cuuint32_t)(kTcK / 2), 64u};
+        const cuuint32_t box[2] = {(cuuint32_t)(kTcGps * kTcK / 2), 64u};   // four groups' codes of 64 rows
         const cuuint32_t estr[2] = {1, 1};
         if (g_encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(a.wq), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }

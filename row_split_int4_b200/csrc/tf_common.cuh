@@ -88,8 +88,10 @@ __host__ __forceinline__ bool aligned(const void *p, uintptr_t a) {
 // exited).  pdl_wait() blocks the calling thread until the kernels before it
 // have finished and their writes are visible.  Each kernel calls pdl_wait()
 // before it reads any array it was given or writes any output, with one
-// exception: it may ask for weights to be brought into L2 first (a prefetch
-// reads L2, which every write reaches, so it can never see stale data).  Each
+// exception: a qmm kernel may read weights first (into L2 or shared memory).
+// No kernel of the library writes weights, and a kernel from elsewhere never
+// calls launch_dependents, so the kernel after it starts only once it has
+// ended and the weights it wrote are in place.  Each
 // qmm kernel calls pdl_trigger() once its own pdl_wait() has returned, so that
 // the next one queues behind it but no further; the short kernels between them
 // (gather, argmax, pick, ...) call it first thing, so that the qmm after them
