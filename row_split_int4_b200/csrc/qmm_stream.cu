@@ -932,21 +932,22 @@ __global__ void __launch_bounds__(kTThreads, 1)
 // the GPU: a warp per row at the full K would run two rounds on a few warps
 // while the rest idle.  Here each CTA owns a contiguous run of output columns
 // and its warps share the (column, K-slice) pairs of that run, round robin.  A
-// pair is one row over one slice (up to 4,096 K: 2 KB of codes and 128 B each of
-// scales and biases), streamed through the warp's own ring by three 1-D bulk
-// copies (one lane each); the warp leaves the slice's tree sum in shared memory,
+// pair is one row over one slice (up to 4,096 K: 2 KB of codes), streamed
+// through the warp's own ring by one 1-D bulk copy; the scales and biases of
+// the CTA's rows come in once, two copies a row, at the start (the copy engine
+// takes a fixed time per copy, so many small copies would hold up the rest of
+// the CTA's copies).  The warp leaves the slice's tree sum in shared memory,
 // and once every pair is done each column's slice sums are added in ascending
 // order.  That is the reduction order of every M = 1 kernel (see the top of this
 // file), so the bits are theirs.
 constexpr int kSWarps = 16;
 constexpr int kSMaxStages = 4;
 constexpr int kSItemQ = 4 * kChunk / 2;          // code bytes of one row-slice
-constexpr int kSItemS = 4 * kChunk / 32;         // scale (or bias) bytes of one row-slice
-constexpr int kSSlot = kSItemQ + 2 * kSItemS;    // 2,304
+constexpr int kSSlot = kSItemQ;                  // 2,048
 
 struct SplitLayout {
     int nch, nsl;
-    size_t limb_off, cst_off, wm_off, part_off, bar_off, ring_off, total;
+    size_t limb_off, cst_off, wm_off, part_off, sb_off, bar_off, ring_off, total;
 };
 
 // M activation rows (limbs, sums and scales of each), `stages` slots per warp.
@@ -958,8 +959,9 @@ __host__ __device__ inline SplitLayout split_layout(int K, int maxcols, int M, i
     L.cst_off = round_up(L.limb_off + (size_t)M * L.nch * 32 * kLimbBytes, 128);
     L.wm_off = L.cst_off + (size_t)M * L.nch * 32 * 16;
     L.part_off = round_up(L.wm_off + (size_t)M * L.nch * 4, 128);
-    L.bar_off = round_up(L.part_off + (size_t)maxcols * L.nsl * M * 4, 128);
-    L.ring_off = round_up(L.bar_off + (size_t)kSWarps * kSMaxStages * 8, 128);
+    L.sb_off = round_up(L.part_off + (size_t)maxcols * L.nsl * M * 4, 128);   // [maxcols][G] scales, then biases
+    L.bar_off = round_up(L.sb_off + (size_t)2 * maxcols * (K / kGroup) * 2, 128);
+    L.ring_off = round_up(L.bar_off + (size_t)(kSWarps * kSMaxStages + 1) * 8, 128);
     L.total = L.ring_off + (size_t)kSWarps * stages * kSSlot;
     return L;
 }
@@ -978,6 +980,9 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     uint8_t *ring = smem + L.ring_off + (size_t)warp * kSStages * kSSlot;
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bar0 = smem_addr(smem + L.bar_off) + (uint32_t)(warp * kSMaxStages * 8);
+    const uint32_t sbar = smem_addr(smem + L.bar_off) + (uint32_t)(kSWarps * kSMaxStages * 8);
+    uint16_t *s_all = reinterpret_cast<uint16_t *>(smem + L.sb_off);
+    uint16_t *b_all = s_all + (size_t)maxcols * G;
 
     // this CTA's columns and the warp's (column, slice) pairs: i = warp + t * kSWarps
     const int c0 = (int)((long long)blockIdx.x * a.seg.ncols / gridDim.x);
@@ -985,53 +990,43 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     const int nitems = (c1 - c0) * nsl;
     const int my_items = nitems > warp ? (nitems - warp + kSWarps - 1) / kSWarps : 0;
 
-    // lane 0 copies the codes of a pair, lane 1 its scales, lane 2 its biases
-    auto piece = [&](int t, const uint8_t *&src, uint32_t &bytes, uint32_t &dst_off, uint32_t &tx) {
+    // lane 0 copies the codes of a pair
+    auto issue = [&](int t) {
+        const int slot = t % kSStages;
+        const uint32_t bar = bar0 + 8 * slot;
         const int i = warp + t * kSWarps;
         const int col = c0 + i / nsl, j = i % nsl;
         const int len = min(4 * kChunk, K - j * 4 * kChunk);   // K of the slice (a multiple of 512)
         const size_t row = (size_t)seg_row(a.seg, col, 0, 0);
-        tx = (uint32_t)(len / 2 + len / 16);
-        if (lane == 0) {
-            src = a.wq + row * (size_t)(K / 2) + (size_t)j * kSItemQ;
-            bytes = (uint32_t)(len / 2);
-            dst_off = 0;
-        } else {
-            const uint16_t *base = lane == 1 ? a.scales : a.biases;
-            src = reinterpret_cast<const uint8_t *>(base + row * (size_t)G + (size_t)j * (4 * kChunk / kGroup));
-            bytes = (uint32_t)(len / 32);
-            dst_off = lane == 1 ? kSItemQ : kSItemQ + kSItemS;
-        }
-    };
-    auto issue = [&](int t) {
-        const int slot = t % kSStages;
-        const uint32_t bar = bar0 + 8 * slot;
-        const uint8_t *src = nullptr;
-        uint32_t bytes = 0, dst_off = 0, tx = 0;
-        piece(t, src, bytes, dst_off, tx);
-        if (lane == 0) mbar_expect_tx(bar, tx);
-        __syncwarp();
-        if (lane < 3) bulk_g2s(ring_s + slot * kSSlot + dst_off, src, bytes, bar);
+        mbar_expect_tx(bar, (uint32_t)(len / 2));
+        bulk_g2s(ring_s + slot * kSSlot, a.wq + row * (size_t)(K / 2) + (size_t)j * kSItemQ, (uint32_t)(len / 2), bar);
     };
 
-    if (lane == 0) {
+    if (lane == 0)
         for (int st = 0; st < kSStages; ++st) mbar_init(bar0 + 8 * st, 1);
+    if (tid == 0) {
+        mbar_init(sbar, 1);
+        fence_mbar_init();
+        mbar_expect_tx(sbar, (uint32_t)(2 * (c1 - c0) * G * 2));
+    } else if (lane == 0) {
         fence_mbar_init();
     }
+    __syncthreads();
+    // Weights before the wait for the kernel this one may overlap (the library
+    // never writes weights, and a kernel from elsewhere ends before this one
+    // starts): the rows' scales and biases, then the warp's first pairs.
+    for (int i = tid; i < 2 * (c1 - c0); i += blockDim.x) {
+        const int col = c0 + (i >> 1);
+        const size_t row = (size_t)seg_row(a.seg, col, 0, 0);
+        const uint16_t *src = ((i & 1) ? a.biases : a.scales) + row * (size_t)G;
+        uint16_t *dst = ((i & 1) ? b_all : s_all) + (size_t)(col - c0) * G;
+        bulk_g2s(smem_addr(dst), src, (uint32_t)(G * 2), sbar);
+    }
+    if (lane == 0)
+        for (int t = 0; t < kSStages && t < my_items; ++t) issue(t);
     __syncwarp();
-    // While the kernel before this one may still run: the warp's first pairs into
-    // L2 (weights are never written by the library's kernels; an L2 prefetch cannot
-    // see stale data in any case).
-    if (lane < 3)
-        for (int t = 0; t < kSStages && t < my_items; ++t) {
-            const uint8_t *src = nullptr;
-            uint32_t bytes = 0, dst_off = 0, tx = 0;
-            piece(t, src, bytes, dst_off, tx);
-            l2_prefetch(src, bytes);
-        }
     pdl_wait();
     pdl_trigger();
-    for (int t = 0; t < kSStages && t < my_items; ++t) issue(t);
     const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
 #pragma unroll
     for (int m = 0; m < kM; ++m)
@@ -1040,7 +1035,7 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     __syncthreads();
 
     const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
-    bool failed = false;
+    bool failed = !__all_sync(0xFFFFFFFFu, wait_slot(sbar, 0, kSpinLimit));
     for (int t = 0; t < my_items; ++t) {
         const int slot = t % kSStages;
         const bool ok = __all_sync(0xFFFFFFFFu, wait_slot(bar0 + 8 * slot, (uint32_t)((t / kSStages) & 1),
@@ -1050,7 +1045,9 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
         const int col = c0 + i / nsl, j = i % nsl;
         const int ch = min(4, nch - 4 * j);
         const uint8_t *sl = ring + slot * kSSlot;
-        const uint16_t *sc0 = reinterpret_cast<const uint16_t *>(sl + kSItemQ);
+        // the slice's scales and biases of this row: 16 groups a chunk
+        const uint16_t *srow = s_all + (size_t)(col - c0) * G + j * (4 * kChunk / kGroup);
+        const uint16_t *brow = b_all + (size_t)(col - c0) * G + j * (4 * kChunk / kGroup);
         float acc[kM];
 #pragma unroll
         for (int m = 0; m < kM; ++m) acc[m] = 0.0f;
@@ -1058,8 +1055,8 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
             const int c = 4 * j + cc;
             const bool live = lane * 32 < K - c * kChunk;   // lanes past the end of a short last chunk add nothing
             const uint4 qv = reinterpret_cast<const uint4 *>(sl)[cc * 32 + lane];
-            const float sv = bf16_bits_to_f32(sc0[cc * 16 + (lane >> 1)]);
-            const float bv = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (lane >> 1)]);
+            const float sv = bf16_bits_to_f32(srow[cc * 16 + (lane >> 1)]);
+            const float bv = bf16_bits_to_f32(brow[cc * 16 + (lane >> 1)]);
 #pragma unroll
             for (int m = 0; m < kM; ++m) {
                 LaneChunk lc;
@@ -1070,8 +1067,8 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
                     const int l = __ffs(mm) - 1;
                     const float xj = wide_x(limbs + m * lc_n * kLimbBytes, c, l, lane);
                     const uint32_t word = reinterpret_cast<const uint32_t *>(sl)[(cc * 32 + l) * 4 + (lane >> 3)];
-                    const float s = bf16_bits_to_f32(sc0[cc * 16 + (l >> 1)]);
-                    const float b = bf16_bits_to_f32(sc0[kSItemS / 2 + cc * 16 + (l >> 1)]);
+                    const float s = bf16_bits_to_f32(srow[cc * 16 + (l >> 1)]);
+                    const float b = bf16_bits_to_f32(brow[cc * 16 + (l >> 1)]);
                     const float d = wide_dot(xj, word, lane, s, b);
                     if (lane == l) acc[m] += d;
                 }
@@ -1083,10 +1080,12 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
             if (lane == 0) part[((col - c0) * nsl + j) * kM + m] = failed ? __int_as_float(0x7FC00000) : v;
         }
         __syncwarp();
-        if (t + kSStages < my_items && !failed) issue(t + kSStages);
+        if (lane == 0 && t + kSStages < my_items && !failed) issue(t + kSStages);
     }
-    if (failed)   // copies still in flight get a bounded chance to land before exit
+    if (failed) {   // copies still in flight get a bounded chance to land before exit
         for (int st = 0; st < kSStages; ++st) wait_slot(bar0 + 8 * st, 0, 1024);
+        wait_slot(sbar, 0, 1024);
+    }
     __syncthreads();
 
     // each column and activation row: its slice sums in ascending order
