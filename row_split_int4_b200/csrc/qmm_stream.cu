@@ -209,47 +209,55 @@ __device__ __forceinline__ void prep_limbs(const uint16_t *x, int K, int nch, ui
             if (u >= nu) break;   // warp-uniform: nu is a multiple of 32
             const int lc = u >> 2, w = u & 3, c = lc >> 5, l = lc & 31;
             const uint32_t *hv = xb[b];   // values 8w .. 8w + 7 of the lane-chunk, two per word (zero past K)
-            int emax = 0, bad = 0;
+            // largest magnitude field of the 8 values: the exponent sits above the
+            // mantissa, so the largest field has the largest e (a subnormal reads e = 1)
+            uint32_t mx = 0;
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-                const int ef = (int)((h >> 7) & 0xFFu);
-                bad |= ef == 0xFF ? 1 : 0;
-                if ((h & 0x7FFFu) != 0) emax = max(emax, max(ef, 1));   // M != 0; a subnormal reads e = 1
-            }
+            for (int i = 0; i < 4; ++i) mx = __vmaxu2(mx, hv[i] & 0x7FFF7FFFu);
+            mx = max(mx & 0xFFFFu, mx >> 16);
+            int emax = mx == 0 ? 0 : max((int)(mx >> 7), 1);
+            const int bad = (mx >> 7) == 0xFFu ? 1 : 0;   // an infinity or a NaN
             emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 1));
             emax = max(emax, __shfl_xor_sync(0xFFFFFFFFu, emax, 2));
-            uint32_t L[6] = {0u, 0u, 0u, 0u, 0u, 0u};   // word w of limb vector 2 limb + parity
-            int cnt = 0, sf = 0;   // cnt: nonzero x within 2^4 of the largest (bits 0..7), smaller ones (8..15), bad (16..)
+            // F = x 2^(23-E) = x 2^(149-emax), by two exact power-of-two products in fp32
+            // (the first only when 2^(149-emax) would not be a normal fp32), then one
+            // conversion rounded to nearest even: exactly the integer shift above for
+            // every x (sign * M * 2^sh, |F| < 2^23; below 1/2 when sh <= -9)
+            const float pre = emax >= 22 ? 1.0f : __int_as_float(191 << 23);   // 2^64
+            const float scl = __int_as_float((emax >= 22 ? 276 - emax : 212 - emax) << 23);
+            int F[8];
+            // cnt: nonzero x within 2^4 of the largest (bits 0..7), smaller ones (8..15),
+            // bad (16..); the sum of F in wrapping arithmetic (an infinity converts to
+            // 2^31 - 1; such a lane-chunk's sum is never used)
+            int cnt = 0;
+            uint32_t sfu = 0;
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
-                const uint32_t h = (hv[t >> 1] >> (16 * (t & 1))) & 0xFFFFu;
-                const int ef = (int)((h >> 7) & 0xFFu);
-                const int M = ef == 0 ? (int)(h & 0x7Fu) : (int)(0x80u | (h & 0x7Fu));
-                const int sh = max(ef, 1) - emax + 15;
-                if (M != 0) cnt += sh >= 12 ? 1 : 256;
-                int F;
-                if (sh >= 0) {
-                    F = M << sh;
-                } else if (sh > -9) {
-                    const int d = -sh;
-                    F = (M + (1 << (d - 1)) - 1 + ((M >> d) & 1)) >> d;
-                } else {
-                    F = 0;
-                }
-                if (h & 0x8000u) F = -F;
-                sf += F;
-                // value 8w + t: byte t >> 1 of word w of limb vectors 2 limb + (t & 1)
-                const int p = t & 1, sft = 8 * (t >> 1);
-                L[0 + p] |= (uint32_t)(F & 0xFF) << sft;
-                L[2 + p] |= (uint32_t)((F >> 8) & 0xFF) << sft;
-                L[4 + p] |= (uint32_t)((F >> 16) & 0xFF) << sft;
+                const uint32_t hw = hv[t >> 1];
+                const uint32_t h = (t & 1) ? hw >> 16 : hw & 0xFFFFu;
+                const float xf = __uint_as_float((t & 1) ? hw & 0xFFFF0000u : hw << 16);
+                F[t] = __float2int_rn((xf * pre) * scl);
+                const uint32_t mag = h & 0x7FFFu;
+                if (mag != 0) cnt += max((int)(mag >> 7), 1) >= emax - 3 ? 1 : 256;   // sh >= 12
+                sfu += (uint32_t)F[t];
+            }
+            // value 8w + t: byte t >> 1 of word w of limb vectors 2 limb + (t & 1); byte
+            // `limb` of the two's complement F
+            uint32_t L[6];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t lo = __byte_perm(F[p], F[p + 2], 0x5140), hi = __byte_perm(F[p + 4], F[p + 6], 0x5140);
+                const uint32_t lo2 = __byte_perm(F[p], F[p + 2], 0x7362), hi2 = __byte_perm(F[p + 4], F[p + 6], 0x7362);
+                L[0 + p] = __byte_perm(lo, hi, 0x5410);
+                L[2 + p] = __byte_perm(lo, hi, 0x7632);
+                L[4 + p] = __byte_perm(lo2, hi2, 0x5410);
             }
             cnt += bad << 16;
             cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 1);
             cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, 2);
-            sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 1);
-            sf += __shfl_xor_sync(0xFFFFFFFFu, sf, 2);
+            sfu += __shfl_xor_sync(0xFFFFFFFFu, sfu, 1);
+            sfu += __shfl_xor_sync(0xFFFFFFFFu, sfu, 2);
+            const int sf = (int)sfu;
             const bool any_bad = (cnt >> 16) != 0;
             const bool fallback = !any_bad && (cnt & 0xFF) <= 2 && ((cnt >> 8) & 0xFF) > 0;
             uint4 *dst = reinterpret_cast<uint4 *>(limbs) + (size_t)c * 6 * 32 + l;
@@ -291,20 +299,30 @@ __device__ __forceinline__ void fused_head_keys(const QmmArgs &a, uint64_t best,
 
 // The word of one slice from the qmm grid's ncand warp keys: max over them (the
 // argmax order is the keys' unsigned order, so any tree gives the same key), the
-// winning value read back from the logits.  One CTA.
-__global__ void __launch_bounds__(1024) argmax_keys_kernel(const uint64_t *cand, int ncand, const uint16_t *logits,
-                                                           uint32_t id_base, uint64_t *word) {
+// winning value read back from the logits.  One CTA of kKeyThreads threads, small
+// enough (threads, registers, shared memory) to sit beside a qmm CTA on its SM:
+// the qmm launched after it then starts on every SM at once.
+constexpr int kKeyThreads = 128;
+__global__ void __launch_bounds__(kKeyThreads) argmax_keys_kernel(const uint64_t *cand, int ncand, const uint16_t *logits,
+                                                                  uint32_t id_base, uint64_t *word) {
     pdl_trigger();
     pdl_wait();
-    uint64_t v = 0;
-    for (int i = threadIdx.x; i < ncand; i += blockDim.x) v = umax64(v, cand[i]);
-    v = warp_max64(v);
-    __shared__ uint64_t red[32];
+    uint64_t v0 = 0, v1 = 0, v2 = 0, v3 = 0;   // four loads in flight per thread
+    int i = threadIdx.x;
+    for (; i + 3 * kKeyThreads < ncand; i += 4 * kKeyThreads) {
+        v0 = umax64(v0, cand[i]);
+        v1 = umax64(v1, cand[i + kKeyThreads]);
+        v2 = umax64(v2, cand[i + 2 * kKeyThreads]);
+        v3 = umax64(v3, cand[i + 3 * kKeyThreads]);
+    }
+    for (; i < ncand; i += kKeyThreads) v0 = umax64(v0, cand[i]);
+    uint64_t v = warp_max64(umax64(umax64(v0, v1), umax64(v2, v3)));
+    __shared__ uint64_t red[kKeyThreads / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) red[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        v = lane < (int)(blockDim.x >> 5) ? red[lane] : 0ull;
+        v = lane < kKeyThreads / 32 ? red[lane] : 0ull;
         v = warp_max64(v);
         if (lane == 0) *word = word_of_key(v, logits, id_base);
     }
@@ -1331,7 +1349,7 @@ cudaError_t launch_qmm_m1_stream(const QmmArgs &a, cudaStream_t stream, int *nca
 
 cudaError_t launch_argmax_keys(const uint64_t *cand, int ncand, const uint16_t *logits, uint32_t id_base, uint64_t *word,
                                cudaStream_t stream) {
-    return launch_pdl(argmax_keys_kernel, dim3(1), dim3(1024), 0, stream, cand, ncand, logits, id_base, word);
+    return launch_pdl(argmax_keys_kernel, dim3(1), dim3(kKeyThreads), 0, stream, cand, ncand, logits, id_base, word);
 }
 
 int qmm_m1_stream_max_cand() { return num_sms() * kMaxWarps; }
