@@ -762,13 +762,15 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
     };
 
-    // The whole ring goes out first (one tile-chunk a slot), before the wait for
-    // the kernel this one may overlap: the weights are never written by a kernel
-    // of the library, and a kernel from elsewhere does not release this one
-    // before it ends.  Then all warps prepare the limbs, and the producers keep
-    // the rings full.
+    // The first three slots of each ring go out first (one tile-chunk a slot),
+    // before the wait for the kernel this one may overlap: the weights are never
+    // written by a kernel of the library, and a kernel from elsewhere does not
+    // release this one before it ends.  Every CTA's first copies arrive as one
+    // burst, and a smaller burst lands each group's first slot sooner (measured:
+    // 71.1 -> 69.1 us on the lm_head half against sending the whole ring).  Then
+    // all warps prepare the limbs, and the producers keep the rings full.
     if (producer && lane == 0)
-        for (int i = 0; i < S; ++i) issue_next();
+        for (int i = 0; i < 3 && i < S; ++i) issue_next();
     __syncwarp();
     pdl_wait();
     pdl_trigger();
@@ -1069,7 +1071,8 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
         float acc[kM];
 #pragma unroll
         for (int m = 0; m < kM; ++m) acc[m] = 0.0f;
-        for (int cc = 0; cc < ch; ++cc) {
+        // one chunk of the pair (a full slice's four unrolled)
+        auto chunk = [&](int cc) {
             const int c = 4 * j + cc;
             const bool live = lane * 32 < K - c * kChunk;   // lanes past the end of a short last chunk add nothing
             const uint4 qv = reinterpret_cast<const uint4 *>(sl)[cc * 32 + lane];
@@ -1091,6 +1094,12 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
                     if (lane == l) acc[m] += d;
                 }
             }
+        };
+        if (ch == 4) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) chunk(cc);
+        } else {
+            for (int cc = 0; cc < ch; ++cc) chunk(cc);
         }
 #pragma unroll
         for (int m = 0; m < kM; ++m) {
