@@ -1013,17 +1013,19 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     const int nitems = (c1 - c0) * nsl;
     const int my_items = nitems > warp ? (nitems - warp + kSWarps - 1) / kSWarps : 0;
 
-    // lane 0 copies the codes of a pair
-    auto issue = [&](int t) {
+    // the codes of pair t of warp w into slot t % kSStages of w's ring
+    auto issue_for = [&](int w, int t) {
         const int slot = t % kSStages;
-        const uint32_t bar = bar0 + 8 * slot;
-        const int i = warp + t * kSWarps;
+        const uint32_t bar = smem_addr(smem + L.bar_off) + (uint32_t)(w * kSMaxStages * 8) + 8 * slot;
+        const uint32_t ring_w = smem_addr(smem + L.ring_off + (size_t)w * kSStages * kSSlot);
+        const int i = w + t * kSWarps;
         const int col = c0 + i / nsl, j = i % nsl;
         const int len = min(4 * kChunk, K - j * 4 * kChunk);   // K of the slice (a multiple of 512)
         const size_t row = (size_t)seg_row(a.seg, col, 0, 0);
         mbar_expect_tx(bar, (uint32_t)(len / 2));
-        bulk_g2s(ring_s + slot * kSSlot, a.wq + row * (size_t)(K / 2) + (size_t)j * kSItemQ, (uint32_t)(len / 2), bar);
+        bulk_g2s(ring_w + slot * kSSlot, a.wq + row * (size_t)(K / 2) + (size_t)j * kSItemQ, (uint32_t)(len / 2), bar);
     };
+    auto issue = [&](int t) { issue_for(warp, t); };   // lane 0 of the pair's warp
 
     if (lane == 0)
         for (int st = 0; st < kSStages; ++st) mbar_init(bar0 + 8 * st, 1);
@@ -1037,24 +1039,34 @@ __global__ void __launch_bounds__(kSWarps * 32, 1) qmm_m1_split_kernel(QmmArgs a
     __syncthreads();
     // Weights before the wait for the kernel this one may overlap (the library
     // never writes weights, and a kernel from elsewhere ends before this one
-    // starts): the rows' scales and biases, then the warp's first pairs.
-    for (int i = tid; i < 2 * (c1 - c0); i += blockDim.x) {
-        const int col = c0 + (i >> 1);
-        const size_t row = (size_t)seg_row(a.seg, col, 0, 0);
-        const uint16_t *src = ((i & 1) ? a.biases : a.scales) + row * (size_t)G;
-        uint16_t *dst = ((i & 1) ? b_all : s_all) + (size_t)(col - c0) * G;
-        bulk_g2s(smem_addr(dst), src, (uint32_t)(G * 2), sbar);
+    // starts): the last warp sends the rows' scales and biases and every warp's
+    // first pairs (lane w those of warp w), while the other warps prepare the
+    // limbs -- the copy engine takes a fixed time per copy, so the copies and the
+    // preparation overlap instead of following one another.
+    constexpr int kIssuer = kSWarps - 1;
+    if (warp == kIssuer) {
+        for (int i = lane; i < 2 * (c1 - c0); i += 32) {
+            const int col = c0 + (i >> 1);
+            const size_t row = (size_t)seg_row(a.seg, col, 0, 0);
+            const uint16_t *src = ((i & 1) ? a.biases : a.scales) + row * (size_t)G;
+            uint16_t *dst = ((i & 1) ? b_all : s_all) + (size_t)(col - c0) * G;
+            bulk_g2s(smem_addr(dst), src, (uint32_t)(G * 2), sbar);
+        }
+        if (lane < kSWarps) {
+            const int items_w = nitems > lane ? (nitems - lane + kSWarps - 1) / kSWarps : 0;
+            for (int t = 0; t < kSStages && t < items_w; ++t) issue_for(lane, t);
+        }
+        __syncwarp();
     }
-    if (lane == 0)
-        for (int t = 0; t < kSStages && t < my_items; ++t) issue(t);
-    __syncwarp();
     pdl_wait();
     pdl_trigger();
     const size_t lc_n = (size_t)nch * 32;   // lane-chunks of one activation row
+    if (warp != kIssuer) {
 #pragma unroll
-    for (int m = 0; m < kM; ++m)
-        prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, csts + m * lc_n, wms + m * nch,
-                   kSWarps, warp, lane);
+        for (int m = 0; m < kM; ++m)
+            prep_limbs(a.x + (size_t)m * a.ldx, K, nch, limbs + m * lc_n * kLimbBytes, csts + m * lc_n, wms + m * nch,
+                       kSWarps - 1, warp, lane);
+    }
     __syncthreads();
 
     const uint4 *limb_l = reinterpret_cast<const uint4 *>(limbs) + lane;
