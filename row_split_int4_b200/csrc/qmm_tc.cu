@@ -78,8 +78,8 @@ __host__ __device__ constexpr int tc_scale_warps(int n) { return 4 * (n < 32 ? 1
 __host__ __device__ constexpr int tc_threads(int n) { return 32 * (2 + tc_dec_warps(n) + tc_scale_warps(n)); }
 __host__ __device__ constexpr int tc_slot_bytes(int n) { return kTcGps * (n * kTcK * 2 + kTcRows * kTcK / 2); }
 __host__ __device__ constexpr int tc_ring(int n) { return n == 16 ? 4 : (n == 32 ? 3 : (n == 64 ? 4 : 2)); }
-__host__ __device__ constexpr int tc_bg(int n) { return n <= 32 ? 2 : 1; }
-__host__ __device__ constexpr int tc_astages(int n) { return n <= 32 ? 2 : (n == 64 ? 8 : 4); }
+__host__ __device__ constexpr int tc_bg(int n) { return n <= 64 ? 2 : 1; }
+__host__ __device__ constexpr int tc_astages(int n) { return n <= 32 ? 2 : (n == 64 ? 3 : 4); }
 __host__ __device__ constexpr int tc_dfit(int n) {
     return (int)(tc_tmem_cols(n) - 32 * tc_bg(n) * tc_astages(n)) / (tc_bg(n) * n);
 }
