@@ -1217,15 +1217,17 @@ static TilePlan tile_plan(const QmmArgs &a, int rows) {
 }
 
 // The tile ring takes the call when the driver offers the tensor-map encoder, two
-// slots per group fit beside the limbs, and the tiles keep every group busy: 16-row
-// tiles with at least four per SM, else (not GLU, K >= 8,192) 4-row tiles with at
-// least two per SM; otherwise the per-warp kernel's finer units balance better.
+// slots per group fit beside the limbs, and there are tiles enough: 16-row tiles
+// with at least two per SM (attn_out's 320 tiles: 15.9 -> 13.8 us against the
+// per-warp ring, though half the groups of a CTA get no tile), else (not GLU,
+// K >= 8,192) 4-row tiles with at least two per SM; otherwise the per-warp
+// kernel's finer units balance better.
 // (With a short K the 4-chunk slots run mostly empty -- at K = 5,120 a tile's second
 // slot holds one chunk -- and the per-warp ring measured faster there.)  Returns the
 // rows per compute warp of the tile shape, 0 for the per-warp kernel.
 static int tile_ring_shape(const QmmArgs &a) {
     if (!encode_tiled_fn() || tile_stages(a.K, 1) < 2) return 0;
-    if (tile_plan(a, TileShape<4>::rows).ntiles >= 4 * num_sms()) return 4;
+    if (tile_plan(a, TileShape<4>::rows).ntiles >= 2 * num_sms()) return 4;
     if (!a.glu && a.K >= 8192 && tile_plan(a, TileShape<1>::rows).ntiles >= 2 * num_sms()) return 1;
     return 0;
 }
