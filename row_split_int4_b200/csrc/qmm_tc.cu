@@ -78,7 +78,7 @@ __host__ __device__ constexpr int tc_scale_warps(int n) { return 4 * (n < 32 ? 1
 __host__ __device__ constexpr int tc_threads(int n) { return 32 * (2 + tc_dec_warps(n) + tc_scale_warps(n)); }
 __host__ __device__ constexpr int tc_slot_bytes(int n) { return kTcGps * (n * kTcK * 2 + kTcRows * kTcK / 2); }
 __host__ __device__ constexpr int tc_ring(int n) { return n == 16 ? 4 : (n == 32 ? 3 : (n == 64 ? 4 : 2)); }
-__host__ __device__ constexpr int tc_bg(int n) { return n <= 64 ? 2 : 1; }
+__host__ __device__ constexpr int tc_bg(int) { return 2; }
 __host__ __device__ constexpr int tc_astages(int n) { return n <= 32 ? 2 : (n == 64 ? 3 : 4); }
 __host__ __device__ constexpr int tc_dfit(int n) {
     return (int)(tc_tmem_cols(n) - 32 * tc_bg(n) * tc_astages(n)) / (tc_bg(n) * n);
@@ -104,7 +104,7 @@ struct TcChecks {
     static_assert(tc_slot_bytes(N) % 1024 == 0, "ring slots keep the 1 KB alignment of the swizzled tile");
     static_assert(N * kTcRows * 4 <= tc_ring(N) * tc_slot_bytes(N), "partial sums must fit in the ring");
     static_assert(tc_num_bars(N) * 8 + 8 <= kTcBarBytes, "barrier area");
-    static_assert(tc_dbufs(N) >= 2 && tc_bg(N) * (tc_dbufs(N) * N + 32 * tc_astages(N)) <= (int)tc_tmem_cols(N),
+    static_assert(tc_dbufs(N) >= 1 && tc_bg(N) * (tc_dbufs(N) * N + 32 * tc_astages(N)) <= (int)tc_tmem_cols(N),
                   "tensor memory map");
     static_assert(kTcGps % tc_bg(N) == 0 && kTcXbSlots % tc_bg(N) == 0 && 8 % tc_bg(N) == 0, "steps of whole groups");
     static_assert(tc_smem_bytes(N) <= 227 * 1024, "shared memory");
