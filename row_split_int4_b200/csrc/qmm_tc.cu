@@ -115,6 +115,7 @@ struct TcChecks {
 // Plan of one launch, computed on the host.
 struct TcPlan {
     int ks;                        // CTAs per cluster (K slices)
+    int persist;                   // 1: each CTA walks tiles blockIdx.x, + gridDim.x, ... (ks == 1, no GLU)
     int periods;                   // K / 512: eight groups each
     int ntiles;
     int tstart[TF_MAX_SEGS + 1];   // first tile of each segment (TF_EPI_NONE)
@@ -309,7 +310,7 @@ __device__ __forceinline__ float tc_pick_bf16(const uint4 &v) {
     return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 
-template <int N>
+template <int N, bool kPersist>
 __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     qmm_tc_kernel(QmmArgs a, const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap, TcPlan plan) {
     constexpr int SW = tc_scale_warps(N);     // scale warps
@@ -337,9 +338,14 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     pdl_trigger();
     const int ks = plan.ks;
     const int rank = (int)tc_cluster_rank();
-    const int tile = blockIdx.x / ks;
     const int p0 = rank * plan.periods / ks, p1 = (rank + 1) * plan.periods / ks;
-    const int i0 = 8 * p0, nst = 8 * (p1 - p0);          // this CTA's groups [i0, i0 + nst)
+    const int i0 = 8 * p0, nst = 8 * (p1 - p0);          // this CTA's groups [i0, i0 + nst) of a tile
+    // The CTA's tiles: one (blockIdx.x / ks), or with kPersist every
+    // gridDim.x-th from blockIdx.x, the roles running on through them without a
+    // new start (barrier phases and ring slots count on across tiles).
+    const int ntl = kPersist ? (plan.ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 1;
+    auto tile_of = [&](int it) { return kPersist ? (int)blockIdx.x + it * (int)gridDim.x : (int)blockIdx.x / ks; };
+    const int ntot = ntl * nst;                          // groups this CTA runs through
     const uint32_t bar_s = tc_smem(bars);
     // barrier addresses: full[R] xfree[R] cfree[R] afull[A] aempty[A] dfull[D] dfree[D] xbfull[X] xbfree[X]
     auto full = [=](int s) { return bar_s + 8u * s; };
@@ -352,33 +358,36 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     auto xbfull = [=](int s) { return bar_s + 8u * (3 * R + 2 * NA + 2 * ND + s); };
     auto xbfree = [=](int s) { return bar_s + 8u * (3 * R + 2 * NA + 2 * ND + kTcXbSlots + s); };
 
-    // The tile's rows: box A (tile rows 0-63) and box B (64-127) of the whole
+    // A tile's rows: box A (tile rows 0-63) and box B (64-127) of the whole
     // matrix, how many of each box are valid, and the output column of tile row 0.
-    int rowA, rowB, validA, validB, col_base;
-    if (a.glu) {
-        rowA = a.seg.row0[0] + 64 * tile;
-        rowB = a.seg.row0[1] + 64 * tile;
-        validA = validB = min(64, a.seg.ncols - 64 * tile);
-        col_base = 64 * tile;
-    } else {
-        // the segment holding this tile (unrolled, so the parameter arrays are not indexed at run time)
-        int tfirst = 0, nr = 0, r0 = 0, c0 = 0;
+    auto tile_info = [&](int tile, int &rowA, int &rowB, int &validA, int &validB, int &col_base) {
+        if (a.glu) {
+            rowA = a.seg.row0[0] + 64 * tile;
+            rowB = a.seg.row0[1] + 64 * tile;
+            validA = validB = min(64, a.seg.ncols - 64 * tile);
+            col_base = 64 * tile;
+        } else {
+            // the segment holding this tile (unrolled, so the parameter arrays are not indexed at run time)
+            int tfirst = 0, nr = 0, r0 = 0, c0 = 0;
 #pragma unroll
-        for (int j = 0; j < TF_MAX_SEGS; ++j)
-            if (j < a.seg.nseg && tile >= plan.tstart[j]) {
-                tfirst = plan.tstart[j];
-                nr = a.seg.nrows[j];
-                r0 = a.seg.row0[j];
-                c0 = a.seg.col0[j];
-            }
-        const int local = tile - tfirst;
-        const int nv = min(kTcRows, nr - kTcRows * local);
-        rowA = r0 + kTcRows * local;
-        rowB = rowA + 64;
-        validA = min(64, nv);
-        validB = nv - validA;
-        col_base = c0 + kTcRows * local;
-    }
+            for (int j = 0; j < TF_MAX_SEGS; ++j)
+                if (j < a.seg.nseg && tile >= plan.tstart[j]) {
+                    tfirst = plan.tstart[j];
+                    nr = a.seg.nrows[j];
+                    r0 = a.seg.row0[j];
+                    c0 = a.seg.col0[j];
+                }
+            const int local = tile - tfirst;
+            const int nv = min(kTcRows, nr - kTcRows * local);
+            rowA = r0 + kTcRows * local;
+            rowB = rowA + 64;
+            validA = min(64, nv);
+            validB = nv - validA;
+            col_base = c0 + kTcRows * local;
+        }
+    };
+    int rowA, rowB, validA, validB, col_base;   // the first (or only) tile's
+    tile_info(tile_of(0), rowA, rowB, validA, validB, col_base);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < R; ++s) {
@@ -423,8 +432,13 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             const uint32_t bytes = (uint32_t)SLOT;
             const int nsl = nst / kTcGps;
             int issued = 0;
-            for (int j = 0; j < nsl; ++j) {
+            int tr_a = rowA, tr_b = rowB;
+            for (int j = 0; j < ntl * nsl; ++j) {   // slots over the CTA's tiles
                 const int s = j % R;
+                if (j > 0 && j % nsl == 0) {   // the next tile's rows
+                    int va, vb, cb;
+                    tile_info(tile_of(j / nsl), tr_a, tr_b, va, vb, cb);
+                }
                 bool ok = true;
                 if (j >= R) {
                     const uint32_t par = ((j / R) - 1) & 1;
@@ -434,7 +448,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
                     if (lane == 0) *fail = 1;
                     break;
                 }
-                const int i = i0 + kTcGps * j;
+                const int i = i0 + kTcGps * (j % nsl);
                 const uint32_t slot = tc_smem(ring + s * SLOT);
                 if (lane == 0) tc_expect_tx(full(s), bytes);
                 __syncwarp(0x7u);
@@ -442,7 +456,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
                     tc_tma_3d(slot, &xmap, 0, 0, i, full(s));
                 else
                     tc_tma_2d(slot + XBYTES + (lane - 1) * (kTcRows / 2) * (kTcGps * kTcK / 2), &cmap,
-                              i * (kTcK / 2), lane == 1 ? rowA : rowB, full(s));
+                              i * (kTcK / 2), lane == 1 ? tr_a : tr_b, full(s));
                 issued = j + 1;
             }
             // every copy issued must land before the ring is reused or the CTA exits
@@ -454,7 +468,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         // ---------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t idesc = tc_idesc(N);
-            for (int k = 0; k < nst / BG; ++k) {   // steps of BG groups
+            for (int k = 0; k < ntot / BG; ++k) {   // steps of BG groups
                 const int sa = k % NA, sd = k % ND;
                 if (!tc_wait(afull(sa), (k / NA) & 1, fail) || (k >= ND && !tc_wait(dfree(sd), ((k / ND) - 1) & 1, fail))) {
                     *fail = 1;
@@ -496,7 +510,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         const uint32_t a_lane = tmem + ((uint32_t)(32 * q) << 16) + ACOL + (uint32_t)(dh * VW);
         const bool xrole = dh == 0;
         uint32_t v[VW];
-        for (int k = 0; k < nst / BG; ++k) {
+        for (int k = 0; k < ntot / BG; ++k) {
             const int sa = k % NA, xs = k % XS;
             bool ok = k < NA || tc_wait(aempty(sa), ((k / NA) - 1) & 1, fail);
             if (__any_sync(0xFFFFFFFFu, !ok)) {
@@ -575,13 +589,19 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         const int q = warp & 3, h = (warp - 2 - DW) >> 2;   // lane quarter, block of NT rows
         const int t = 32 * q + lane;                   // tile row == TMEM lane
         const int G = a.K / kGroup;
-        const bool valid = t < 64 ? t < validA : (t - 64) < validB;
-        const int row = t < 64 ? rowA + t : rowB + (t - 64);
-        const uint16_t *srow = valid ? a.scales + (size_t)row * G : nullptr;
-        const uint16_t *brow = valid ? a.biases + (size_t)row * G : nullptr;
         const uint32_t d_lane = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(h * NT);
         const float *xb_h = xbar + h * NT;
         float acc[NT];
+#pragma unroll
+        for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
+        int li = 0;   // groups folded so far, over all of the CTA's tiles
+        for (int it = 0; it < ntl && !*fail; ++it) {
+        int tra = rowA, trb = rowB, tva = validA, tvb = validB, tcb = col_base;
+        if (it > 0) tile_info(tile_of(it), tra, trb, tva, tvb, tcb);
+        const bool valid = t < 64 ? t < tva : (t - 64) < tvb;
+        const int row = t < 64 ? tra + t : trb + (t - 64);
+        const uint16_t *srow = valid ? a.scales + (size_t)row * G : nullptr;
+        const uint16_t *brow = valid ? a.biases + (size_t)row * G : nullptr;
 #pragma unroll
         for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
         uint4 s8 = make_uint4(0, 0, 0, 0), b8 = s8, sn = s8, bn = s8;
@@ -589,7 +609,6 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             s8 = __ldg(reinterpret_cast<const uint4 *>(srow + 8 * p0));
             b8 = __ldg(reinterpret_cast<const uint4 *>(brow + 8 * p0));
         }
-        int li = 0;
         for (int p = p0; p < p1 && !*fail; ++p) {
             if (srow && p + 1 < p1) {   // next period's eight scales and biases
                 sn = __ldg(reinterpret_cast<const uint4 *>(srow + 8 * (p + 1)));
@@ -640,15 +659,33 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             s8 = sn;
             b8 = bn;
         }
-        // this CTA's partial sums -> shared memory, as part[m][t]
+        if (kPersist && valid) {   // the whole K is here: the tile's outputs go straight out
 #pragma unroll
-        for (int j = 0; j < NT; ++j) part[(h * NT + j) * kTcRows + t] = acc[j];
+            for (int j = 0; j < NT; ++j)
+                if (h * NT + j < a.M) a.y[(size_t)(h * NT + j) * a.ldy + tcb + t] = f32_to_bf16_rne(acc[j]);
+        }
+        }
+        // this CTA's partial sums -> shared memory, as part[m][t]
+        if (!kPersist) {
+#pragma unroll
+            for (int j = 0; j < NT; ++j) part[(h * NT + j) * kTcRows + t] = acc[j];
+        }
     }
     __syncwarp();
     tc_fence_before();
     tc_cluster_sync();   // every partial sum and failure flag of the cluster is in place
 
-    if (warp >= 2 + DW) {
+    if (kPersist && warp >= 2 + DW) {
+        if (*fail) {   // a wait gave up: every output of the CTA's tiles reads NaN
+            const int tid = threadIdx.x - 32 * (2 + DW);
+            for (int it = 0; it < ntl; ++it) {
+                int ra, rb, va, vb, cb;
+                tile_info(tile_of(it), ra, rb, va, vb, cb);
+                const int nv = va + vb;
+                for (int e = tid; e < nv * a.M; e += 32 * SW) a.y[(size_t)(e / nv) * a.ldy + cb + e % nv] = (uint16_t)TF_NAN_BF16;
+            }
+        }
+    } else if (warp >= 2 + DW) {
         const int tid = threadIdx.x - 32 * (2 + DW);   // 0 .. 32 SW - 1
         constexpr int RT = 32 * SW;                              // reducing threads
         int bad = 0;
@@ -730,20 +767,24 @@ bool qmm_tc_eligible(const QmmArgs &a) {
            aligned(a.biases, 16);
 }
 
-template <int N>
+template <int N, bool kPersist>
 static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const CUtensorMap &cmap, const TcPlan &plan,
                                cudaStream_t stream) {
     static bool smem_set[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     if (!smem_set[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(qmm_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes(N));
+        const cudaError_t e =
+            cudaFuncSetAttribute(qmm_tc_kernel<N, kPersist>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes(N));
         if (e != cudaSuccess) return e;
         smem_set[dev] = true;
     }
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3((unsigned)(plan.ntiles * plan.ks));
+    // persistent: one CTA per resident slot, each walking every gridDim.x-th tile
+    const int slots = tc_ctas_per_sm(N) * num_sms();
+    const int ctas = kPersist ? (plan.ntiles < slots ? plan.ntiles : slots) : plan.ntiles * plan.ks;
+    cfg.gridDim = dim3((unsigned)ctas);
     cfg.blockDim = dim3(tc_threads(N));
     cfg.dynamicSmemBytes = tc_smem_bytes(N);
     cfg.stream = stream;
@@ -756,7 +797,15 @@ static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, qmm_tc_kernel<N>, a, xmap, cmap, plan);
+    return cudaLaunchKernelEx(&cfg, qmm_tc_kernel<N, kPersist>, a, xmap, cmap, plan);
+}
+
+template <int N>
+static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const CUtensorMap &cmap, const TcPlan &plan,
+                               cudaStream_t stream) {
+    if constexpr (N <= 64)
+        if (plan.persist) return launch_tc_n<N, true>(a, xmap, cmap, plan, stream);
+    return launch_tc_n<N, false>(a, xmap, cmap, plan, stream);
 }
 
 cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
@@ -779,6 +828,9 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
         plan.ntiles = n;
     }
     if (plan.ntiles == 0) return cudaSuccess;
+    // One K slice and plain outputs: CTAs stay resident and walk the tiles.  At
+    // N = 128 the fold's registers run short and the walk measured slower.
+    plan.persist = plan.ks == 1 && !a.glu && n_mma <= 64;
 
     CUtensorMap xmap, cmap;
     {

@@ -6,7 +6,8 @@ The kernel copies four 64-value groups of activations at a time as one 3-D tile
 as zero) and the codes four groups wide; these cases check that both copies land
 where the MMA and the decoders read them: M from 4 to 128 (N = 16, 32, 64 and 128),
 a ragged last 128-row tile, rows padded to ldx = K + 64 (bits equal to the
-unpadded call) and the fused gate*SiLU(up) epilogue, each against the oracle
+unpadded call), the fused gate*SiLU(up) epilogue, and more tiles than resident
+CTAs with one K slice (persistent CTAs walking several tiles), each against the oracle
 (TensorFold PR #1433, step-1 body: each rank reduces its rows over the full K in
 fp32; step-2 body: the GLU of the gate and up halves).
 """
@@ -77,3 +78,26 @@ def test_tc_glu_odd_rows(tf, orc, M):
         yo, y64, ad = orc.qmm_rows(x, *w.astuple(), np.arange(r0, r0 + F), nthreads=NT, want_f64=True)
         check_values(host_bits(t), yo, y64, ad, K, f"tensor cores M={M} rows {r0}..")
     check_values(host_bits(act), orc.glu(host_bits(g), host_bits(u)), what=f"tensor cores M={M} GLU")
+
+
+@pytest.mark.parametrize("M", [16, 33, 64, 128])
+def test_tc_persistent_tiles(tf, orc, M):
+    """More 128-row tiles than resident CTAs, with the K range in one slice: each
+    CTA walks several tiles (every gridDim-th), its copy ring, tensor-memory
+    stages and barrier phases running on across them (MMA widths up to 64; at
+    128 the same shape runs one tile per CTA).  Two segments with ragged ends put
+    tile starts off the 128-row grid of the whole matrix."""
+    K = 512
+    segs = [(0, 20000), (25000, 19000)]   # 157 + 149 tiles, both segments end in a partial tile
+    N = 44000
+    w = synth.make_weights(N, K, seed=200 + M)
+    W = DevWeights(w)
+    x = synth.make_x(M, K, seed=200 + M)
+    xt = padded(dev(x))
+    y = host_bits(qmm(tf, xt, W, segs))
+    torch.cuda.synchronize()
+    cols = np.arange(sum(n for _, n in segs))
+    whole = np.concatenate([np.arange(r0, r0 + n) for r0, n in segs])
+    pick = np.unique(np.concatenate([cols[::5], cols[-300:], cols[19800:20200]]))   # every fifth, both tails
+    yo, y64, ad = orc.qmm_rows(x, *w.astuple(), whole[pick], nthreads=NT, want_f64=True)
+    check_values(y[:, pick], yo, y64, ad, K, f"tensor cores M={M}, persistent")
