@@ -11,12 +11,14 @@ for M > 1 (where the call runs the two kernels one after the other).  The
 picked id of the two fused halves must equal the pick over the whole
 vocabulary, and the words must equal the oracle's scan of the GPU's logits.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
 
 import synth
-from gpu_util import DevWeights, bits_equal, dev, empty_bf16, host_bits, need_gpu
+from gpu_util import DevWeights, bits_equal, check_values, dev, empty_bf16, host_bits, need_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -198,3 +200,28 @@ def test_fused_full_head_planted(tf, orc, whole_head, kind):
         for row, a, b, c in reversed(saved):
             W.wq[row], W.scales[row], W.biases[row] = a, b, c
         torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("kind", ["natural", "nan"])
+def test_fused_narrow_long_k(tf, orc, kind):
+    """A head too narrow for the tile ring with a long K (3,000 rows, K = 17,920:
+    the narrow-call kernel, whose warps leave the keys): the fused call's logits and words
+    equal the unfused call's, for both halves and the whole, with a NaN row
+    planted; and the logits are within the V bar of the oracle on sampled rows."""
+    V, K = 3000, 17920
+    w = synth.make_weights(V, K, seed=15, tag=synth.TAG_HEAD)
+    if kind == "nan":
+        wq, sc, bi = (a.copy() for a in w.astuple())
+        sc[2200] = 0x7FC0
+        w = synth.QWeights(wq, sc, bi)
+    W = DevWeights(w)
+    x_bits = synth.make_x(1, K, seed=15, tag=synth.TAG_X)
+    x = dev(x_bits)
+    for seg in (tf.tf_split_rows(V, 2, 0), tf.tf_split_rows(V, 2, 1), (0, V)):
+        lu, wu = unfused(tf, x, W, seg, seg[0])
+        lf, wf = fused(tf, x, W, seg, seg[0])
+        torch.cuda.synchronize()
+        assert bits_equal(lf, lu) and torch.equal(wf, wu), seg
+    rows = np.unique(np.concatenate([np.arange(0, V, 23), [V - 1, 2200]]))
+    yo, y64, ad = orc.qmm_rows(x_bits, *w.astuple(), rows, nthreads=os.cpu_count() or 1, want_f64=True)
+    check_values(host_bits(lf)[:, rows], yo, y64, ad, K, f"narrow long-K head ({kind})")

@@ -159,3 +159,38 @@ def test_few_rows_equal_one_row_calls(tf, orc, M, shape):
         sampled(orc, x, w, host_bits(g), np.arange(segs[0][0], segs[0][0] + ncols), K, f"gate M={M}")
     else:
         sampled(orc, x, w, host_bits(y), columns_of(segs), K, f"{shape} M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_narrow_call_many_columns(tf, orc, M):
+    """The narrow-call kernel with many (row, slice) pairs per warp: K = 17,920
+    (17.5 chunks, slices of 4, 4, 4, 4 and 1.5 chunks) over 4,000 columns from
+    three segments, so each CTA's ~27 columns give its warps more pairs than ring
+    slots, and a CTA's run of rows can cross a segment boundary.  Every column is
+    checked against the oracle, and bit for bit against the same rows on the
+    16-row tile ring (the whole 6,000-row matrix) and, for two activation rows,
+    against one-row calls."""
+    K, N = 17920, 6000
+    segs = [(0, 1500), (4000, 1500), (2000, 1000)]
+    w = synth.make_weights(N, K, seed=70 + M, tag=synth.TAG_W2)
+    W = DevWeights(w)
+    x = synth.make_x(M, K, seed=80 + M)
+    xt = dev(x)
+    cols = columns_of(segs)
+    y = empty_bf16(M, len(cols))
+    tf.tf_qmm_rows(xt, *W.t(), segs, y)
+    whole = empty_bf16(M, N) if M == 1 else None
+    if M == 1:
+        tf.tf_qmm_rows(xt, *W.t(), [(0, N)], whole)
+    ones = []
+    for m in range(M if M > 1 else 0):
+        o = empty_bf16(1, len(cols))
+        tf.tf_qmm_rows(xt[m:m + 1], *W.t(), segs, o)
+        ones.append(o)
+    torch.cuda.synchronize()
+    if M == 1:
+        assert bits_equal(y, whole[:, torch.as_tensor(cols, device="cuda")]), "narrow call != tile ring"
+    for m, o in enumerate(ones):
+        assert bits_equal(y[m:m + 1], o), f"activation row {m}: two-row call != one-row call"
+    yo, y64, ad = orc.qmm_rows(x, *w.astuple(), cols, nthreads=NT, want_f64=True)
+    check_values(host_bits(y), yo, y64, ad, K, f"narrow call M={M}")
