@@ -1,0 +1,135 @@
+"""Seeded random calls of tf_qmm_rows over every route, against the oracle.
+
+Each case draws its shape from a route's range: the M = 1 tile ring (more than
+296 sixteen-row tiles), the narrow-call kernel (K above 8,192, fewer rows), the
+per-warp ring (few rows), the tensor cores (M = 4..128), and the fallbacks for a K
+that is not a multiple of 512; with one to three row segments of the whole matrix
+or the fused gate*SiLU(up) epilogue, and activation rows padded in memory or not.
+Every case is checked against the oracle (V: 2 bf16 ulps, or the fp32
+accumulation floor where the sum cancels) on all of its columns, or on 384
+sampled ones plus both ends of every segment for the larger cases (TensorFold
+PR #1433, step-1 body: each rank reduces its rows over the full K; step-2 body:
+the GLU of the gate and up halves).  A last set draws fused heads
+(tf_qmm_argmax_rows) of random slices: logits against the oracle, the word bit
+for bit against the oracle's argmax scan of the GPU's logits (step-1 body:
+pair_argmax over each rank's half).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import DevWeights, check_values, dev, empty_bf16, host_bits, need_gpu
+
+pytestmark = pytest.mark.gpu
+NT = os.cpu_count() or 1
+ROUTES = ["tile", "split", "warp", "tc", "odd_k", "glu_tile", "glu_tc", "glu_odd_k"]
+CASES = 8   # per route
+
+
+@pytest.fixture(scope="module")
+def tf():
+    need_gpu()
+    import row_split_int4_b200 as tf
+    return tf
+
+
+def draw(route: str, i: int):
+    """(M, K, N_whole, segs, glu, pad) of case i of a route."""
+    rng = np.random.default_rng([1433, ROUTES.index(route), i])
+    pick = lambda seq: seq[int(rng.integers(len(seq)))]   # noqa: E731
+    glu = route.startswith("glu")
+    if route in ("tile", "glu_tile"):
+        M, K = int(rng.integers(1, 4)), pick([1024, 2048, 3072])
+        N = int(rng.integers(4800, 7000)) if not glu else 2 * int(rng.integers(2400, 3600))
+    elif route == "split":
+        M, K, N = int(rng.integers(1, 3)), pick([9216, 10240, 12800]), int(rng.integers(100, 3000))
+    elif route == "warp":
+        M, K, N = 1, pick([512, 1536, 4096]), int(rng.integers(1, 2000))
+    elif route in ("tc", "glu_tc"):
+        M, K = int(rng.integers(4, 129)), pick([512, 2048, 5120])
+        N = int(rng.integers(1, 1500)) if not glu else 2 * int(rng.integers(1, 700))
+    else:   # K not a multiple of 512
+        M, K = int(rng.integers(1, 41)), pick([576, 1088, 2112])
+        N = int(rng.integers(1, 800)) if not glu else 2 * int(rng.integers(1, 400))
+    if glu:
+        F = N // 2
+        segs = [(0, F), (F, F)]
+    else:
+        cuts = np.sort(rng.choice(np.arange(1, N), size=min(2, N - 1), replace=False)) if N > 2 else np.array([], int)
+        bounds = [0, *cuts.tolist(), N]
+        spans = [(bounds[j], bounds[j + 1] - bounds[j]) for j in range(len(bounds) - 1)]
+        nseg = int(rng.integers(1, len(spans) + 1))
+        segs = [spans[j] for j in rng.permutation(len(spans))[:nseg]]
+    return M, K, N, segs, glu, bool(rng.integers(2))
+
+
+@pytest.mark.parametrize("route,i", [(r, i) for r in ROUTES for i in range(CASES)])
+def test_random_call(tf, orc, route, i):
+    M, K, N, segs, glu, pad = draw(route, i)
+    w = synth.make_weights(N, K, seed=1000 + 31 * ROUTES.index(route) + i)
+    W = DevWeights(w)
+    x = synth.make_x(M, K, seed=2000 + 31 * ROUTES.index(route) + i)
+    xt = dev(x)
+    if pad:   # the same rows with leading dimension K + 64
+        buf = torch.zeros(M, K + 64, dtype=torch.bfloat16, device="cuda")
+        buf[:, :K] = xt
+        xt = buf[:, :K]
+    ncols = segs[0][1] if glu else sum(n for _, n in segs)
+    y = empty_bf16(M, ncols)
+    tf.tf_qmm_rows(xt, *W.t(), segs, y, epi=tf.TF_EPI_GLU if glu else 0)
+    torch.cuda.synchronize()
+    yb = host_bits(y)
+    what = f"{route} case {i}: M={M} K={K} N={N} segs={segs} pad={pad}"
+    if glu:
+        F = segs[0][1]
+        # The GPU's gate and up rows (the unfused calls) are held to V against the
+        # oracle, and the fused result to the oracle's GLU of those same rows: the
+        # GLU of bf16 values within V of the oracle's may round differently.
+        g = empty_bf16(M, F)
+        u = empty_bf16(M, F)
+        tf.tf_qmm_rows(xt, *W.t(), [segs[0]], g)
+        tf.tf_qmm_rows(xt, *W.t(), [segs[1]], u)
+        torch.cuda.synchronize()
+        for t, r0, part in ((g, 0, "gate"), (u, F, "up")):
+            yo, y64, ad = orc.qmm_rows(x, *w.astuple(), np.arange(r0, r0 + F), nthreads=NT, want_f64=True)
+            check_values(host_bits(t), yo, y64, ad, K, f"{what} {part} rows")
+        check_values(yb, orc.glu(host_bits(g), host_bits(u)), what=what + " GLU")
+        return
+    cols = np.concatenate([np.arange(r0, r0 + n) for r0, n in segs])
+    pos = np.arange(cols.size)
+    if M * cols.size * K > 4e8:   # sample: 384 columns plus both ends of every segment
+        rng = np.random.default_rng([7, i])
+        ends, o = [], 0
+        for _, n in segs:
+            ends += [o, o + n - 1]
+            o += n
+        pos = np.unique(np.concatenate([rng.choice(cols.size, 384, replace=False), ends]))
+    yo, y64, ad = orc.qmm_rows(x, *w.astuple(), cols[pos], nthreads=NT, want_f64=True)
+    check_values(yb[:, pos], yo, y64, ad, K, what)
+
+
+@pytest.mark.parametrize("i", range(CASES))
+def test_random_fused_head(tf, orc, i):
+    rng = np.random.default_rng([1437, i])
+    M, K = int(rng.integers(1, 4)), int(rng.choice([512, 2048, 5120]))
+    N = int(rng.integers(2, 9000))
+    r0 = int(rng.integers(0, N - 1))
+    n = int(rng.integers(1, N - r0 + 1))
+    w = synth.make_weights(N, K, seed=3000 + i, tag=synth.TAG_HEAD)
+    W = DevWeights(w)
+    x = synth.make_x(M, K, seed=3000 + i)
+    xt = dev(x)
+    logits = empty_bf16(M, n)
+    words = torch.full((M,), -1, dtype=torch.int64, device="cuda")
+    scratch = torch.empty(tf.tf_qmm_argmax_scratch_bytes(M, n), dtype=torch.uint8, device="cuda")
+    tf.tf_qmm_argmax_rows(xt, *W.t(), (r0, n), r0, logits, words, scratch)
+    torch.cuda.synchronize()
+    lb = host_bits(logits)
+    what = f"fused head case {i}: M={M} K={K} rows {r0}..{r0 + n}"
+    assert np.array_equal(host_bits(words), orc.argmax_rows(lb, r0)), what
+    pos = np.arange(n) if M * n * K <= 4e8 else np.unique(np.concatenate([rng.choice(n, 384, replace=False), [0, n - 1]]))
+    yo, y64, ad = orc.qmm_rows(x, *w.astuple(), r0 + pos, nthreads=NT, want_f64=True)
+    check_values(lb[:, pos], yo, y64, ad, K, what)
