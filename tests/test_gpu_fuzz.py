@@ -12,7 +12,8 @@ PR #1433, step-1 body: each rank reduces its rows over the full K; step-2 body:
 the GLU of the gate and up halves).  A last set draws fused heads
 (tf_qmm_argmax_rows) of random slices: logits against the oracle, the word bit
 for bit against the oracle's argmax scan of the GPU's logits (step-1 body:
-pair_argmax over each rank's half).
+pair_argmax over each rank's half); random int8 heads (the b70 lab's runtime INT8
+LM-head) and random argmax calls with planted ties, signed zeros and non-finites.
 """
 import os
 
@@ -133,3 +134,48 @@ def test_random_fused_head(tf, orc, i):
     pos = np.arange(n) if M * n * K <= 4e8 else np.unique(np.concatenate([rng.choice(n, 384, replace=False), [0, n - 1]]))
     yo, y64, ad = orc.qmm_rows(x, *w.astuple(), r0 + pos, nthreads=NT, want_f64=True)
     check_values(lb[:, pos], yo, y64, ad, K, what)
+
+
+@pytest.mark.parametrize("i", range(CASES))
+def test_random_int8_head(tf, orc, i):
+    """tf_qmm8_rows on random slices, K a multiple of 32 or not (the general kernel)."""
+    rng = np.random.default_rng([27, i])
+    M, K = int(rng.integers(1, 5)), int(rng.choice([512, 1000, 2048, 5120]))
+    N = int(rng.integers(2, 6000))
+    r0 = int(rng.integers(0, N - 1))
+    n = int(rng.integers(1, N - r0 + 1))
+    w = synth.make_weights8(N, K, seed=4000 + i)
+    q8, sc = synth.weights8_to_device(w)
+    x = synth.make_x(M, K, seed=4000 + i)
+    y = empty_bf16(M, n)
+    tf.tf_qmm8_rows(dev(x), q8, sc, [(r0, n)], y)
+    torch.cuda.synchronize()
+    pos = np.arange(n) if M * n * K <= 4e8 else np.unique(np.concatenate([rng.choice(n, 384, replace=False), [0, n - 1]]))
+    yo, y64, ad = orc.qmm8_rows(x, w.q8, w.scales, r0 + pos, nthreads=NT, want_f64=True)
+    check_values(host_bits(y)[:, pos], yo, y64, ad, K, f"int8 head case {i}: M={M} K={K} rows {r0}..{r0 + n}")
+
+
+@pytest.mark.parametrize("i", range(CASES))
+def test_random_argmax(tf, orc, i):
+    """tf_argmax_rows on random logits with planted ties, signed zeros and
+    non-finites: the words bit for bit against the oracle's scan."""
+    rng = np.random.default_rng([33, i])
+    M, n = int(rng.integers(1, 20)), int(rng.integers(1, 300000))
+    v = synth.to_bf16_bits(rng.standard_normal((M, n)).astype(np.float32))
+    for m in range(M):
+        kind = int(rng.integers(5))
+        if kind == 1 and n > 1:   # an exact tie for the top at two places
+            top = int(np.argmax(synth.bf16_bits_to_f32(v[m])))
+            v[m, int(rng.integers(n))] = v[m, top]
+        elif kind == 2:
+            v[m, int(rng.integers(n))] = 0x7FC0   # NaN
+        elif kind == 3:
+            v[m, int(rng.integers(n))] = int(rng.choice([0x7F80, 0xFF80]))   # +-Inf
+        elif kind == 4:
+            v[m, :] = int(rng.choice([0x0000, 0x8000]))   # all +0 or all -0
+    id_base = int(rng.integers(0, 2 ** 30))
+    words = torch.empty(M, dtype=torch.int64, device="cuda")
+    scratch = torch.empty(tf.tf_argmax_scratch_bytes(M, n), dtype=torch.uint8, device="cuda")
+    tf.tf_argmax_rows(dev(v), id_base, words, scratch)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(words), orc.argmax_rows(v, id_base)), f"argmax case {i}: M={M} n={n}"
