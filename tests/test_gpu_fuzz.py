@@ -13,7 +13,10 @@ the GLU of the gate and up halves).  A last set draws fused heads
 (tf_qmm_argmax_rows) of random slices: logits against the oracle, the word bit
 for bit against the oracle's argmax scan of the GPU's logits (step-1 body:
 pair_argmax over each rank's half); random int8 heads (the b70 lab's runtime INT8
-LM-head) and random argmax calls with planted ties, signed zeros and non-finites.
+LM-head), random argmax calls with planted ties, signed zeros and non-finites, and
+random row splits of such logits through the gather, the per-part argmax words and
+top twos, the pick and the merged top two (step-1 body: stage, gather,
+pair_argmax, pair_pick).
 """
 import os
 
@@ -65,6 +68,24 @@ def draw(route: str, i: int):
         nseg = int(rng.integers(1, len(spans) + 1))
         segs = [spans[j] for j in rng.permutation(len(spans))[:nseg]]
     return M, K, N, segs, glu, bool(rng.integers(2))
+
+
+def planted_logits(rng, M, n):
+    """Random bf16 logits [M, n], each row planted with a top tie, a NaN, an
+    infinity, all signed zeros, or nothing."""
+    v = synth.to_bf16_bits(rng.standard_normal((M, n)).astype(np.float32))
+    for m in range(M):
+        kind = int(rng.integers(5))
+        if kind == 1 and n > 1:
+            top = int(np.argmax(synth.bf16_bits_to_f32(v[m])))
+            v[m, int(rng.integers(n))] = v[m, top]
+        elif kind == 2:
+            v[m, int(rng.integers(n))] = 0x7FC0
+        elif kind == 3:
+            v[m, int(rng.integers(n))] = int(rng.choice([0x7F80, 0xFF80]))
+        elif kind == 4:
+            v[m, :] = int(rng.choice([0x0000, 0x8000]))
+    return v
 
 
 @pytest.mark.parametrize("route,i", [(r, i) for r in ROUTES for i in range(CASES)])
@@ -161,21 +182,53 @@ def test_random_argmax(tf, orc, i):
     non-finites: the words bit for bit against the oracle's scan."""
     rng = np.random.default_rng([33, i])
     M, n = int(rng.integers(1, 20)), int(rng.integers(1, 300000))
-    v = synth.to_bf16_bits(rng.standard_normal((M, n)).astype(np.float32))
-    for m in range(M):
-        kind = int(rng.integers(5))
-        if kind == 1 and n > 1:   # an exact tie for the top at two places
-            top = int(np.argmax(synth.bf16_bits_to_f32(v[m])))
-            v[m, int(rng.integers(n))] = v[m, top]
-        elif kind == 2:
-            v[m, int(rng.integers(n))] = 0x7FC0   # NaN
-        elif kind == 3:
-            v[m, int(rng.integers(n))] = int(rng.choice([0x7F80, 0xFF80]))   # +-Inf
-        elif kind == 4:
-            v[m, :] = int(rng.choice([0x0000, 0x8000]))   # all +0 or all -0
+    v = planted_logits(rng, M, n)
     id_base = int(rng.integers(0, 2 ** 30))
     words = torch.empty(M, dtype=torch.int64, device="cuda")
     scratch = torch.empty(tf.tf_argmax_scratch_bytes(M, n), dtype=torch.uint8, device="cuda")
     tf.tf_argmax_rows(dev(v), id_base, words, scratch)
     torch.cuda.synchronize()
     assert np.array_equal(host_bits(words), orc.argmax_rows(v, id_base)), f"argmax case {i}: M={M} n={n}"
+
+
+@pytest.mark.parametrize("i", range(CASES))
+def test_random_seam(tf, orc, i):
+    """A random row split of random logits into 1-4 parts: the gather of the
+    parts, each part's argmax word and top two, the pick and the merged top two,
+    all bit for bit against the oracle (PR #1433 step-1 body: stage, gather,
+    pair_argmax, pair_pick)."""
+    rng = np.random.default_rng([1432, i])
+    M, n, nparts = int(rng.integers(1, 9)), int(rng.integers(4, 60000)), int(rng.integers(1, 5))
+    v = planted_logits(rng, M, n)
+    cuts = np.sort(rng.choice(np.arange(1, n), size=nparts - 1, replace=False)) if nparts > 1 else np.array([], int)
+    bounds = [0, *cuts.tolist(), n]
+    parts = [v[:, bounds[j]:bounds[j + 1]].copy() for j in range(nparts)]
+    widths = [p.shape[1] for p in parts]
+    dparts = [dev(p) for p in parts]
+    dst = empty_bf16(M, n)
+    tf.tf_gather_rows(dst, dparts, widths)
+    words = torch.empty(nparts, M, dtype=torch.int64, device="cuda")
+    tops = torch.empty(nparts, M, 2, dtype=torch.int64, device="cuda")
+    for j, p in enumerate(dparts):
+        w = torch.empty(M, dtype=torch.int64, device="cuda")
+        scr = torch.empty(tf.tf_argmax_scratch_bytes(M, widths[j]), dtype=torch.uint8, device="cuda")
+        tf.tf_argmax_rows(p, bounds[j], w, scr)
+        words[j] = w
+        t2 = torch.empty(M, 2, dtype=torch.int64, device="cuda")
+        scr2 = torch.empty(tf.tf_top2_scratch_bytes(M, widths[j]), dtype=torch.uint8, device="cuda")
+        tf.tf_top2_rows(p, bounds[j], t2, scr2)
+        tops[j] = t2
+    ids = torch.empty(M, dtype=torch.int32, device="cuda")
+    tf.tf_pick(words, ids)
+    merged = torch.empty(M, 2, dtype=torch.int64, device="cuda")
+    tf.tf_top2_merge(tops, merged)
+    torch.cuda.synchronize()
+    what = f"seam case {i}: M={M} n={n} parts={widths}"
+    assert np.array_equal(host_bits(dst), orc.gather_rows(parts, M)), what + " gather"
+    o_words = np.stack([orc.argmax_rows(p, bounds[j]) for j, p in enumerate(parts)])
+    o_tops = np.stack([orc.top2_rows(p, bounds[j]) for j, p in enumerate(parts)])
+    assert np.array_equal(host_bits(words), o_words), what + " words"
+    assert np.array_equal(host_bits(tops), o_tops), what + " top two"
+    assert np.array_equal(host_bits(ids), orc.pick(o_words)), what + " pick"
+    assert np.array_equal(host_bits(merged), orc.top2_merge(o_tops)), what + " merged top two"
+    assert np.array_equal(orc.pick(o_words), orc.pick(orc.argmax_rows(v, 0)[None, :])), what + " split != whole"
