@@ -315,7 +315,9 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     qmm_tc_kernel(QmmArgs a, const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap, TcPlan plan) {
     constexpr int SW = tc_scale_warps(N);     // scale warps
     constexpr int NT = N / (SW / 4);          // activation rows per scale thread (16 or 32)
-    constexpr int CH = 16;                    // columns per tcgen05.ld
+    // columns per tcgen05.ld: the persistent walk at N = 128 keeps the tile's
+    // state in registers beside its 32 sums, so its loads take 8 columns at a time
+    constexpr int CH = (kPersist && N == 128) ? 8 : 16;
     constexpr int R = tc_ring(N), NA = tc_astages(N), ND = tc_dbufs(N);
     constexpr int SLOT = tc_slot_bytes(N), XG = N * kTcK * 2, XBYTES = kTcGps * XG, RING = R * SLOT;
     constexpr uint32_t TCOLS = tc_tmem_cols(N);
@@ -803,8 +805,7 @@ static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const 
 template <int N>
 static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const CUtensorMap &cmap, const TcPlan &plan,
                                cudaStream_t stream) {
-    if constexpr (N <= 64)
-        if (plan.persist) return launch_tc_n<N, true>(a, xmap, cmap, plan, stream);
+    if (plan.persist) return launch_tc_n<N, true>(a, xmap, cmap, plan, stream);
     return launch_tc_n<N, false>(a, xmap, cmap, plan, stream);
 }
 
@@ -828,9 +829,8 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
         plan.ntiles = n;
     }
     if (plan.ntiles == 0) return cudaSuccess;
-    // One K slice and plain outputs: CTAs stay resident and walk the tiles.  At
-    // N = 128 the fold's registers run short and the walk measured slower.
-    plan.persist = plan.ks == 1 && !a.glu && n_mma <= 64;
+    // One K slice and plain outputs: CTAs stay resident and walk the tiles.
+    plan.persist = plan.ks == 1 && !a.glu;
 
     CUtensorMap xmap, cmap;
     {

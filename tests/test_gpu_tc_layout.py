@@ -84,9 +84,9 @@ def test_tc_glu_odd_rows(tf, orc, M):
 def test_tc_persistent_tiles(tf, orc, M):
     """More 128-row tiles than resident CTAs, with the K range in one slice: each
     CTA walks several tiles (every gridDim-th), its copy ring, tensor-memory
-    stages and barrier phases running on across them (MMA widths up to 64; at
-    128 the same shape runs one tile per CTA).  Two segments with ragged ends put
-    tile starts off the 128-row grid of the whole matrix."""
+    stages and barrier phases running on across them (MMA widths 16, 64 and 128,
+    the last with narrower tensor-memory loads).  Two segments with ragged ends
+    put tile starts off the 128-row grid of the whole matrix."""
     K = 512
     segs = [(0, 20000), (25000, 19000)]   # 157 + 149 tiles, both segments end in a partial tile
     N = 44000
