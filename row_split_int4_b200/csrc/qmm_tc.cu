@@ -88,6 +88,10 @@ constexpr int kTcMaxN = 128;                    // activation rows per call
 constexpr int kTcMaxSplit = 8;                  // CTAs per cluster
 constexpr int kTcXbBytes = kTcXbSlots * kTcMaxN * 4;
 constexpr int kTcBarBytes = 1024;               // mbarriers, TMEM address, failure flag
+constexpr int kTcSmemMax = 227 * 1024;          // dynamic shared memory of one CTA
+constexpr int kTcSmemSM = 228 * 1024;           // shared memory of an SM (1 KB of it reserved per CTA)
+// X_g table of a persistent CTA: every group of K, fp32 per activation row of the MMA
+__host__ __device__ constexpr int tc_xtab_bytes(int n, int periods) { return 8 * periods * n * 4; }
 __host__ __device__ constexpr int tc_num_bars(int n) {
     return 3 * tc_ring(n) + 2 * tc_astages(n) + 2 * tc_dbufs(n) + 2 * kTcXbSlots;
 }
@@ -116,6 +120,7 @@ struct TcChecks {
 struct TcPlan {
     int ks;                        // CTAs per cluster (K slices)
     int persist;                   // 1: each CTA walks tiles blockIdx.x, + gridDim.x, ... (ks == 1, no GLU)
+    int xtab;                      // 1 (persistent only): X_g of every group kept in shared memory after the first tile
     int periods;                   // K / 512: eight groups each
     int ntiles;
     int tstart[TF_MAX_SEGS + 1];   // first tile of each segment (TF_EPI_NONE)
@@ -334,6 +339,12 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + RING + kTcXbBytes);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + tc_num_bars(N));
     volatile int *fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // X_g depends on the activations alone, the same for every tile: a persistent
+    // CTA forms it (through the X_g ring) on its first tile only and keeps it here,
+    // [group of the tile][activation row], for the tiles after
+    float *xtab = reinterpret_cast<float *>(smem + RING + kTcXbBytes + kTcBarBytes);
+    // (not at N = 128: there the table's registers would spill the fold's sums)
+    const bool xt = kPersist && N <= 64 && plan.xtab != 0;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
@@ -514,6 +525,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         uint32_t v[VW];
         for (int k = 0; k < ntot / BG; ++k) {
             const int sa = k % NA, xs = k % XS;
+            const bool ring_x = !xt || k * BG < nst;   // X_g formed here: every step, or the first tile's
             bool ok = k < NA || tc_wait(aempty(sa), ((k / NA) - 1) & 1, fail);
             if (__any_sync(0xFFFFFFFFu, !ok)) {
                 *fail = 1;
@@ -543,7 +555,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
                     w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
                 }
                 xsum[g] = 0.0f;
-                if (xrole && t < N) {   // X_g of activation row t: 64 values, k ascending (8 chunks of 8)
+                if (xrole && ring_x && t < N) {   // X_g of activation row t: 64 values, k ascending (8 chunks of 8)
                     const uint8_t *xrow = slot + gs * XG + t * 128;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
@@ -572,7 +584,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             tc_fence_before();
             __syncwarp();
             if (lane == 0) tc_arrive(afull(sa));
-            if (xrole) {
+            if (xrole && ring_x) {
                 ok = k < XS || tc_wait(xbfree(xs), ((k / XS) - 1) & 1, fail);
                 if (__any_sync(0xFFFFFFFFu, !ok)) {
                     *fail = 1;
@@ -580,7 +592,10 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
                 }
                 if (t < N) {
 #pragma unroll
-                    for (int g = 0; g < BG; ++g) xbar[(xs * BG + g) * kTcMaxN + t] = xsum[g];
+                    for (int g = 0; g < BG; ++g) {
+                        xbar[(xs * BG + g) * kTcMaxN + t] = xsum[g];
+                        if (xt) xtab[(k * BG + g) * N + t] = xsum[g];   // published by the arrive below
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) tc_arrive(xbfull(xs));
@@ -598,6 +613,8 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
         int li = 0;   // groups folded so far, over all of the CTA's tiles
         for (int it = 0; it < ntl && !*fail; ++it) {
+        const bool ring_x = !xt || it == 0;   // X_g through the ring (the table's first fill), else from the table
+        int lt = 0;                           // group within the tile
         int tra = rowA, trb = rowB, tva = validA, tvb = validB, tcb = col_base;
         if (it > 0) tile_info(tile_of(it), tra, trb, tva, tvb, tcb);
         const bool valid = t < 64 ? t < tva : (t - 64) < tvb;
@@ -622,7 +639,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     {                                                                                                               \
         const int k = li / BG, sd = k % ND, xs = k % XS, g = (J) % BG;                                              \
         if (g == 0) {                                                                                               \
-            const bool ok = tc_wait(dfull(sd), (k / ND) & 1, fail) && tc_wait(xbfull(xs), (k / XS) & 1, fail);     \
+            const bool ok = tc_wait(dfull(sd), (k / ND) & 1, fail) && (!ring_x || tc_wait(xbfull(xs), (k / XS) & 1, fail)); \
             if (__any_sync(0xFFFFFFFFu, !ok)) {                                                                     \
                 *fail = 1;                                                                                          \
                 break;                                                                                              \
@@ -631,7 +648,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         }                                                                                                           \
         /* D holds sum (q - 8) x: y += s D + (b + 8 s) X */                                                       \
         const float sf = tc_pick_bf16<J>(s8), bf = fmaf(8.0f, sf, tc_pick_bf16<J>(b8));                             \
-        const float *xg = xb_h + (xs * BG + g) * kTcMaxN;                                                           \
+        const float *xg = xt ? xtab + lt * N + h * NT : xb_h + (xs * BG + g) * kTcMaxN;                            \
         _Pragma("unroll") for (int c = 0; c < NT; c += CH) {                                                        \
             uint32_t d[CH];                                                                                         \
             tc_ld<CH>(d_lane + (uint32_t)(BG * N * sd + N * g) + c, d);                                             \
@@ -649,10 +666,11 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
             __syncwarp();                                                                                           \
             if (lane == 0) {                                                                                        \
                 tc_arrive(dfree(sd));                                                                               \
-                tc_arrive(xbfree(xs));                                                                              \
+                if (ring_x) tc_arrive(xbfree(xs));                                                                  \
             }                                                                                                       \
         }                                                                                                           \
         ++li;                                                                                                       \
+        ++lt;                                                                                                       \
     }
             do {
                 TC_GROUP(0) TC_GROUP(1) TC_GROUP(2) TC_GROUP(3) TC_GROUP(4) TC_GROUP(5) TC_GROUP(6) TC_GROUP(7)
@@ -777,7 +795,7 @@ static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const 
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
     if (!smem_set[dev]) {
         const cudaError_t e =
-            cudaFuncSetAttribute(qmm_tc_kernel<N, kPersist>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes(N));
+            cudaFuncSetAttribute(qmm_tc_kernel<N, kPersist>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemMax);
         if (e != cudaSuccess) return e;
         smem_set[dev] = true;
     }
@@ -788,7 +806,7 @@ static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const 
     const int ctas = kPersist ? (plan.ntiles < slots ? plan.ntiles : slots) : plan.ntiles * plan.ks;
     cfg.gridDim = dim3((unsigned)ctas);
     cfg.blockDim = dim3(tc_threads(N));
-    cfg.dynamicSmemBytes = tc_smem_bytes(N);
+    cfg.dynamicSmemBytes = tc_smem_bytes(N) + (plan.xtab ? tc_xtab_bytes(N, plan.periods) : 0);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -831,6 +849,11 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
     if (plan.ntiles == 0) return cudaSuccess;
     // One K slice and plain outputs: CTAs stay resident and walk the tiles.
     plan.persist = plan.ks == 1 && !a.glu;
+    // the X_g table where it fits beside the rest, keeping two CTAs per SM where there are two
+    if (plan.persist && n_mma <= 64) {
+        const int need = tc_smem_bytes(n_mma) + tc_xtab_bytes(n_mma, plan.periods);
+        plan.xtab = need <= kTcSmemMax && (tc_ctas_per_sm(n_mma) == 1 || 2 * (need + 1024) <= kTcSmemSM);
+    }
 
     CUtensorMap xmap, cmap;
     {
