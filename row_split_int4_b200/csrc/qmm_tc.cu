@@ -90,8 +90,8 @@ constexpr int kTcXbBytes = kTcXbSlots * kTcMaxN * 4;
 constexpr int kTcBarBytes = 1024;               // mbarriers, TMEM address, failure flag
 constexpr int kTcSmemMax = 227 * 1024;          // dynamic shared memory of one CTA
 constexpr int kTcSmemSM = 228 * 1024;           // shared memory of an SM (1 KB of it reserved per CTA)
-// X_g table of a persistent CTA: every group of K, fp32 per activation row of the MMA
-__host__ __device__ constexpr int tc_xtab_bytes(int n, int periods) { return 8 * periods * n * 4; }
+// X_g table of a CTA: its groups of K, fp32 per activation row of the MMA
+__host__ __device__ constexpr int tc_xtab_bytes(int n, int groups) { return groups * n * 4; }
 __host__ __device__ constexpr int tc_num_bars(int n) {
     return 3 * tc_ring(n) + 2 * tc_astages(n) + 2 * tc_dbufs(n) + 2 * kTcXbSlots;
 }
@@ -120,7 +120,8 @@ struct TcChecks {
 struct TcPlan {
     int ks;                        // CTAs per cluster (K slices)
     int persist;                   // 1: each CTA walks tiles blockIdx.x, + gridDim.x, ... (ks == 1, no GLU)
-    int xtab;                      // 1 (persistent only): X_g of every group kept in shared memory after the first tile
+    int xtab;                      // 1: the X_g of the CTA's groups in a shared-memory table (see the kernel)
+    int xgroups;                   // groups of K a CTA covers at most (its table's rows)
     int periods;                   // K / 512: eight groups each
     int ntiles;
     int tstart[TF_MAX_SEGS + 1];   // first tile of each segment (TF_EPI_NONE)
@@ -339,12 +340,18 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + RING + kTcXbBytes);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + tc_num_bars(N));
     volatile int *fail = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    // X_g depends on the activations alone, the same for every tile: a persistent
-    // CTA forms it (through the X_g ring) on its first tile only and keeps it here,
-    // [group of the tile][activation row], for the tiles after
+    // X_g depends on the activations alone, the same for every tile, so where it
+    // fits it goes into a table [group][activation row] in shared memory.  At
+    // N = 16 the scale warps fill it from x in global memory while the first copies,
+    // decodes and MMAs run, and no decoder forms X_g.  At N = 32 and 64 (filling it
+    // would take the scale warps too long) a persistent CTA forms X_g through the
+    // ring on its first tile only, writing the table too, and folds its later
+    // tiles from it.  Not at N = 128: the table's registers would spill the fold's
+    // sums.
     float *xtab = reinterpret_cast<float *>(smem + RING + kTcXbBytes + kTcBarBytes);
-    // (not at N = 128: there the table's registers would spill the fold's sums)
-    const bool xt = kPersist && N <= 64 && plan.xtab != 0;
+    constexpr bool kXFill = N == 16;                                    // the scale warps fill the table
+    constexpr bool kXFirst = !kXFill && kPersist && N <= 64;            // first-tile fill through the ring
+    const bool xt = (kXFill || kXFirst) && plan.xtab != 0;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
@@ -525,7 +532,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         uint32_t v[VW];
         for (int k = 0; k < ntot / BG; ++k) {
             const int sa = k % NA, xs = k % XS;
-            const bool ring_x = !xt || k * BG < nst;   // X_g formed here: every step, or the first tile's
+            const bool ring_x = !xt || (!kXFill && k * BG < nst);   // X_g formed here: no table, or its first tile
             bool ok = k < NA || tc_wait(aempty(sa), ((k / NA) - 1) & 1, fail);
             if (__any_sync(0xFFFFFFFFu, !ok)) {
                 *fail = 1;
@@ -594,7 +601,7 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
 #pragma unroll
                     for (int g = 0; g < BG; ++g) {
                         xbar[(xs * BG + g) * kTcMaxN + t] = xsum[g];
-                        if (xt) xtab[(k * BG + g) * N + t] = xsum[g];   // published by the arrive below
+                        if (!kXFill && xt) xtab[(k * BG + g) * N + t] = xsum[g];   // published by the arrive below
                     }
                 }
                 __syncwarp();
@@ -611,9 +618,32 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
         float acc[NT];
 #pragma unroll
         for (int j = 0; j < NT; ++j) acc[j] = 0.0f;
+        if (kXFill && xt) {   // the X_g table: the same sums, in the same order, as a decoder forms from a slot
+            const int ft = threadIdx.x - 32 * (2 + DW);
+            for (int e = ft; e < nst * N; e += 32 * SW) {
+                const int gl = e / N, tr = e % N;
+                float xs = 0.0f;
+                if (tr < a.M) {
+                    const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + (size_t)tr * a.ldx + (size_t)(i0 + gl) * kTcK);
+                    uint4 xv[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) xv[c] = __ldg(xr + c);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float cs =
+                            tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(tc_add_bf16x2(0.0f, xv[c].x), xv[c].y), xv[c].z), xv[c].w);
+                        xs = c == 0 ? cs : xs + cs;
+                    }
+                } else {   // a row past M reads as zero in the copies: its sum is +0
+                    xs = tc_add_bf16x2(0.0f, 0u);
+                }
+                xtab[gl * N + tr] = xs;
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(32 * SW) : "memory");   // the scale warps only
+        }
         int li = 0;   // groups folded so far, over all of the CTA's tiles
         for (int it = 0; it < ntl && !*fail; ++it) {
-        const bool ring_x = !xt || it == 0;   // X_g through the ring (the table's first fill), else from the table
+        const bool ring_x = !xt || (!kXFill && it == 0);   // X_g through the ring (and into the table), else from it
         int lt = 0;                           // group within the tile
         int tra = rowA, trb = rowB, tva = validA, tvb = validB, tcb = col_base;
         if (it > 0) tile_info(tile_of(it), tra, trb, tva, tvb, tcb);
@@ -806,7 +836,7 @@ static cudaError_t launch_tc_n(const QmmArgs &a, const CUtensorMap &xmap, const 
     const int ctas = kPersist ? (plan.ntiles < slots ? plan.ntiles : slots) : plan.ntiles * plan.ks;
     cfg.gridDim = dim3((unsigned)ctas);
     cfg.blockDim = dim3(tc_threads(N));
-    cfg.dynamicSmemBytes = tc_smem_bytes(N) + (plan.xtab ? tc_xtab_bytes(N, plan.periods) : 0);
+    cfg.dynamicSmemBytes = tc_smem_bytes(N) + (plan.xtab ? tc_xtab_bytes(N, plan.xgroups) : 0);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -850,8 +880,9 @@ cudaError_t launch_qmm_tc(const QmmArgs &a, cudaStream_t stream) {
     // One K slice and plain outputs: CTAs stay resident and walk the tiles.
     plan.persist = plan.ks == 1 && !a.glu;
     // the X_g table where it fits beside the rest, keeping two CTAs per SM where there are two
-    if (plan.persist && n_mma <= 64) {
-        const int need = tc_smem_bytes(n_mma) + tc_xtab_bytes(n_mma, plan.periods);
+    plan.xgroups = 8 * ((plan.periods + plan.ks - 1) / plan.ks);
+    if (n_mma == 16 || (plan.persist && n_mma <= 64)) {
+        const int need = tc_smem_bytes(n_mma) + tc_xtab_bytes(n_mma, plan.xgroups);
         plan.xtab = need <= kTcSmemMax && (tc_ctas_per_sm(n_mma) == 1 || 2 * (need + 1024) <= kTcSmemSM);
     }
 
