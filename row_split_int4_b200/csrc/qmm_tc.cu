@@ -27,7 +27,7 @@
 //     the row's codes -> bf16 pairs, stored into an A stage in tensor memory
 //     (tcgen05.st), software-pipelined so that a store drains while the next
 //     group is decoded; four of them, one thread per activation row, also form
-//     X_g from the activation tile.
+//     X_g from the activation tile, except where a table holds it (below).
 //   * warp 1, one thread: tcgen05.mma kind::f16, A from tensor memory, B (the
 //     activations) from shared memory, four K=16 steps per group into one of
 //     several D buffers; tcgen05.commit releases the ring slot and the A stage and
@@ -35,6 +35,14 @@
 //   * scale warps, per tensor-memory lane quarter one per 32 activation rows
 //     (4 to 16 warps): read D_g (tcgen05.ld), fold it and X_g into fp32
 //     accumulators held in registers, release the D buffer.
+//
+// Persistent CTAs.  When one slice covers K (and no GLU), one CTA per resident
+// slot walks every gridDim.x-th tile, its ring, stages and barrier phases
+// running on across tiles, and writes each tile's outputs itself.  X_g depends on
+// x alone, so where it fits a shared-memory table holds the X_g of all the CTA's
+// groups: at N = 16 the scale warps fill it from x in global memory at the start
+// (no decoder forms X_g), at N = 32 and 64 a persistent CTA forms X_g on its
+// first tile and folds the later ones from the table.  Same sums, same bits.
 //
 // Split K.  The groups are cut into `ks` slices, one per CTA of a thread-block
 // cluster of `ks` CTAs; ks and the cut depend on K and the whole matrix's row
