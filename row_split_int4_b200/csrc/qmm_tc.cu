@@ -330,8 +330,9 @@ __global__ void __launch_bounds__(tc_threads(N), tc_ctas_per_sm(N))
     constexpr int SW = tc_scale_warps(N);     // scale warps
     constexpr int NT = N / (SW / 4);          // activation rows per scale thread (16 or 32)
     // columns per tcgen05.ld: the persistent walk at N = 128 keeps the tile's
-    // state in registers beside its 32 sums, so its loads take 8 columns at a time
-    constexpr int CH = (kPersist && N == 128) ? 8 : 16;
+    // state in registers beside its 32 sums, so its loads take 8 columns at a time;
+    // one tile per CTA at N = 64 has the room to load its 32 in one go (one wait)
+    constexpr int CH = kPersist ? (N == 128 ? 8 : 16) : (N == 64 ? 32 : 16);
     constexpr int R = tc_ring(N), NA = tc_astages(N), ND = tc_dbufs(N);
     constexpr int SLOT = tc_slot_bytes(N), XG = N * kTcK * 2, XBYTES = kTcGps * XG, RING = R * SLOT;
     constexpr uint32_t TCOLS = tc_tmem_cols(N);
